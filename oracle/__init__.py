@@ -1,0 +1,236 @@
+"""CPU fp64 oracle for the R-SWA / SR-SWA decode-attention hot path.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package. The product path (``long_context_decode_swa_b200``) never imports it
+and shares no code with it.
+
+The arithmetic lives in ``rswa_oracle.c`` (plain C, fp64, OpenMP over
+independent (sequence, head) problems); this module compiles it with gcc on
+first use and marshals numpy arrays. bf16 tensors travel as their raw 16-bit
+patterns in ``np.uint16`` arrays. ``kv_cache_bytes`` is the one piece of
+arithmetic written here, in Python: the cache-size closed form.
+
+Parity status: every function is pinned by ``tests/test_oracle_*.py`` (see
+each function's docstring for its pins); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rswa_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BLOCK = 32  # SR-SWA block size (sparse_block_size)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle library with gcc (no GPU involved). Returns its path."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _L():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            I64 = ctypes.c_int64
+            Dbl = ctypes.c_double
+            lib.oracle_set_threads.argtypes = [I]
+            lib.oracle_get_threads.restype = I
+            lib.oracle_append.argtypes = [I, I, I, I, P, P, P, P, P, P, P]
+            lib.oracle_rswa_decode.argtypes = [I, I, I, I, I64, P, P, P, P, P, P, P, P, Dbl, P, P]
+            lib.oracle_rswa_prefill.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, P, P, Dbl, P, I, P, P]
+            lib.oracle_index_pool.argtypes = [I, I64, I, I, P, P, P]
+            lib.oracle_entmax15.argtypes = [I64, P, P]
+            lib.oracle_entmax15.restype = Dbl
+            lib.oracle_route.argtypes = [I, I64, I, I, P, P, P, Dbl, I, P, P, P, P, P]
+            lib.oracle_srswa_decode.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, I, P, P, P, P, Dbl, P, P]
+            _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a, ndim: int, name: str) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"{name}: expected bf16 bit patterns as uint16, got {a.dtype}")
+    if a.ndim != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got shape {a.shape}")
+    return a
+
+
+def _i32(a, name: str) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.int32:
+        raise TypeError(f"{name}: expected int32, got {a.dtype}")
+    return a
+
+
+def set_threads(n: int) -> None:
+    _L().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_L().oracle_get_threads())
+
+
+def append(ring_k, ring_v, k_new, v_new, wp, fill):
+    """Ring append, in place on ring_k/ring_v/wp/fill. Returns slot_out [B].
+
+    ring_* uint16 [B][H][n][D]; k_new/v_new uint16 [B][H][D]; wp/fill int32 [B].
+    """
+    for name, a in (("ring_k", ring_k), ("ring_v", ring_v), ("wp", wp), ("fill", fill)):
+        if not (isinstance(a, np.ndarray) and a.flags.c_contiguous):
+            raise ValueError(f"{name} must be a C-contiguous numpy array (updated in place)")
+    B, H, n, D = ring_k.shape
+    k_new = _u16(k_new, 3, "k_new")
+    v_new = _u16(v_new, 3, "v_new")
+    slot = np.zeros(B, np.int32)
+    _L().oracle_append(B, H, n, D, _p(ring_k), _p(ring_v), _p(k_new), _p(v_new), _p(wp), _p(fill), _p(slot))
+    return slot
+
+
+def rswa_decode(q, pk, pv, prefix_len, ring_k, ring_v, wp, fill, scale):
+    """R-SWA decode for every (b, h). Returns (out fp64 [B][H][D], lse fp64 [B][H])."""
+    q = _u16(q, 3, "q")
+    pk = _u16(pk, 4, "pk")
+    pv = _u16(pv, 4, "pv")
+    ring_k = _u16(ring_k, 4, "ring_k")
+    ring_v = _u16(ring_v, 4, "ring_v")
+    prefix_len, wp, fill = _i32(prefix_len, "prefix_len"), _i32(wp, "wp"), _i32(fill, "fill")
+    B, H, D = q.shape
+    cap = pk.shape[2]
+    n = ring_k.shape[2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _L().oracle_rswa_decode(B, H, D, n, cap, _p(q), _p(pk), _p(pv), _p(prefix_len), _p(ring_k), _p(ring_v),
+                            _p(wp), _p(fill), float(scale), _p(out), _p(lse))
+    return out, lse
+
+
+def rswa_prefill(q, k_out, v_out, pk, pv, prefix_len, scale, rows, n, ring_k=None, ring_v=None, wp=None, fill=None):
+    """R-SWA prefill for the listed query rows. Returns (out [B][H][R][D], lse [B][H][R]).
+
+    q/k_out/v_out uint16 [B][H][T][D]; ring (optional) holds the previous chunk.
+    """
+    q = _u16(q, 4, "q")
+    k_out = _u16(k_out, 4, "k_out")
+    v_out = _u16(v_out, 4, "v_out")
+    pk = _u16(pk, 4, "pk")
+    pv = _u16(pv, 4, "pv")
+    B, H, T, D = q.shape
+    cap = pk.shape[2]
+    prefix_len = _i32(prefix_len, "prefix_len")
+    rows = _i32(np.asarray(rows, np.int32), "rows")
+    if rows.size and (rows.min() < 0 or rows.max() >= T):
+        raise ValueError("row index out of range")
+    if ring_k is not None:
+        ring_k = _u16(ring_k, 4, "ring_k")
+        ring_v = _u16(ring_v, 4, "ring_v")
+        wp, fill = _i32(wp, "wp"), _i32(fill, "fill")
+        if ring_k.shape[2] != n:
+            raise ValueError("ring slots != n")
+    R = rows.size
+    out = np.zeros((B, H, R, D), np.float64)
+    lse = np.zeros((B, H, R), np.float64)
+    _L().oracle_rswa_prefill(B, H, D, int(n), cap, T, _p(q), _p(k_out), _p(v_out), _p(pk), _p(pv), _p(prefix_len),
+                             _p(ring_k), _p(ring_v), _p(wp), _p(fill), float(scale), _p(rows), R, _p(out), _p(lse))
+    return out, lse
+
+
+def index_pool(k_idx, prefix_len, blk: int = BLOCK):
+    """Block index keys: kbar fp64 [B][ceil(cap/blk)][DI] (mean of valid token keys)."""
+    k_idx = _u16(k_idx, 3, "k_idx")
+    prefix_len = _i32(prefix_len, "prefix_len")
+    B, cap, DI = k_idx.shape
+    nb_cap = (cap + blk - 1) // blk
+    kbar = np.zeros((B, nb_cap, DI), np.float64)
+    _L().oracle_index_pool(B, cap, DI, blk, _p(k_idx), _p(prefix_len), _p(kbar))
+    return kbar
+
+
+def entmax15(x):
+    """Exact 1.5-entmax of x (x already = z/2). Returns (p fp64, tau)."""
+    x = np.ascontiguousarray(np.asarray(x, np.float64).ravel())
+    p = np.zeros_like(x)
+    tau = _L().oracle_entmax15(x.size, _p(x), _p(p))
+    return p, float(tau)
+
+
+def route(q_idx, kbar, prefix_len, topk: int = 16, idx_scale: float = 1.0, blk: int = BLOCK):
+    """Router: returns dict(blk_idx int32 [B][topk], blk_logp fp64, probs fp64 [B][NBcap], tau fp64 [B], z fp64)."""
+    q_idx = np.ascontiguousarray(q_idx, np.float32)
+    kbar = np.ascontiguousarray(kbar, np.float64)
+    prefix_len = _i32(prefix_len, "prefix_len")
+    B, nb_cap, DI = kbar.shape
+    if q_idx.shape != (B, DI):
+        raise ValueError("q_idx shape")
+    blk_idx = np.zeros((B, topk), np.int32)
+    blk_logp = np.zeros((B, topk), np.float64)
+    probs = np.zeros((B, nb_cap), np.float64)
+    tau = np.zeros(B, np.float64)
+    z = np.zeros((B, nb_cap), np.float64)
+    _L().oracle_route(B, nb_cap, DI, blk, _p(q_idx), _p(kbar), _p(prefix_len), float(idx_scale), int(topk),
+                      _p(blk_idx), _p(blk_logp), _p(probs), _p(tau), _p(z))
+    return dict(blk_idx=blk_idx, blk_logp=blk_logp, probs=probs, tau=tau, z=z)
+
+
+def srswa_decode(q, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, scale, blk: int = BLOCK):
+    """SR-SWA gathered-block decode. Returns (out fp64 [B][H][D], lse fp64 [B][H])."""
+    q = _u16(q, 3, "q")
+    pk = _u16(pk, 4, "pk")
+    pv = _u16(pv, 4, "pv")
+    ring_k = _u16(ring_k, 4, "ring_k")
+    ring_v = _u16(ring_v, 4, "ring_v")
+    prefix_len, wp, fill = _i32(prefix_len, "prefix_len"), _i32(wp, "wp"), _i32(fill, "fill")
+    blk_idx = _i32(blk_idx, "blk_idx")
+    blk_logp = np.ascontiguousarray(blk_logp, np.float64)
+    B, H, D = q.shape
+    topk = blk_idx.shape[1]
+    cap = pk.shape[2]
+    n = ring_k.shape[2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _L().oracle_srswa_decode(B, H, D, n, cap, blk, _p(q), _p(pk), _p(pv), _p(prefix_len), _p(blk_idx),
+                             _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp), _p(fill), float(scale),
+                             _p(out), _p(lse))
+    return out, lse
+
+
+def kv_cache_bytes(ref_tokens: int, T: int, heads: int, head_dim: int, layers: int, bytes_per_elem: int,
+                   window: int | None) -> int:
+    """KV-cache bytes after T generated tokens.
+
+    Cached tokens are L_m + T for full attention (window=None) and
+    L_m + min(n, T) for R-SWA with window n ([R-SWA summary] §二.2); each token
+    stores K and V for every head of every layer.
+    """
+    cached = ref_tokens + (T if window is None else min(window, T))
+    return cached * 2 * heads * head_dim * bytes_per_elem * layers
+
+
+def bf16_bits_to_f64(a: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16) to float64 exactly."""
+    return (np.asarray(a, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -1,0 +1,491 @@
+/*
+ * rswa_oracle.c -- plain, slow, fp64 CPU statement of what the R-SWA / SR-SWA
+ * decode-attention hot path computes.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this library. The product (the CUDA
+ * library and its Python binding) never calls it, shares no code with it and
+ * has no CPU fallback through it.
+ *
+ * Every value is widened to double on load and every sum is taken in double,
+ * in the plain order of the definition. There is no tiling, no online softmax,
+ * no split; OpenMP only distributes independent (sequence, head) problems.
+ *
+ * Page names used in the citations below:
+ *   [R-SWA summary]   "百度Unlimited OCR" paper summary, lshu.cn/news/33052
+ *   [R-SWA tutorial]  "百度 Unlimited OCR 深度实战 ... R-SWA注意力革命", chenxutan.com/d/4055.html
+ *   [SR-SWA explainer] Unlimited-OCR-2 SR-SWA explainer, nxmr.cn/news/162408
+ *
+ * Layouts (row-major, all little-endian):
+ *   bf16 tensors are passed as their raw 16-bit patterns (uint16_t).
+ *   q, k_new, v_new        [B][H][D]
+ *   prefix K/V  pk, pv     [B][H][cap][D]   rows [0, prefix_len[b]) valid
+ *   ring K/V               [B][H][n][D]
+ *   wp, fill               [B]  next slot to write, number of valid slots
+ *   prefill q/k_out/v_out  [B][H][T][D]
+ *   k_idx                  [B][cap][DI]     per-token router index keys
+ *   q_idx                  [B][DI]          fp32 router query per sequence
+ *
+ * Parity status of each function is stated at the function.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* helpers                                                             */
+/* ------------------------------------------------------------------ */
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+static double bf16_to_double(uint16_t bits) {
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+static int64_t pos_mod(int64_t a, int64_t n) {
+  int64_t r = a % n;
+  return r < 0 ? r + n : r;
+}
+
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int oracle_get_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/*
+ * One attention read: softmax over an explicit key list.
+ *   s_j = scale * <q, k_j> + bias_j
+ *   o   = sum_j softmax(s)_j v_j ,  lse = log sum_j exp(s_j)
+ * The largest s_j is subtracted before exponentiating (exp(s - M) / sum
+ * exp(s - M) is the same quotient); lse adds M back. An empty key list gives
+ * o = 0 and lse = -inf.
+ * This is the attention formula of [R-SWA tutorial] §2.2.1 (softmax(Q K^T /
+ * sqrt(d)) V) over the key set R-SWA makes visible, with an additive bias
+ * slot for SR-SWA's log-probability term.
+ */
+typedef struct {
+  const uint16_t** krow;
+  const uint16_t** vrow;
+  double* bias;
+  double* s;
+  int64_t count;
+} keylist;
+
+static void keylist_init(keylist* L, int64_t max_keys) {
+  L->krow = (const uint16_t**)malloc(sizeof(*L->krow) * (size_t)(max_keys > 0 ? max_keys : 1));
+  L->vrow = (const uint16_t**)malloc(sizeof(*L->vrow) * (size_t)(max_keys > 0 ? max_keys : 1));
+  L->bias = (double*)malloc(sizeof(double) * (size_t)(max_keys > 0 ? max_keys : 1));
+  L->s = (double*)malloc(sizeof(double) * (size_t)(max_keys > 0 ? max_keys : 1));
+  L->count = 0;
+}
+
+static void keylist_free(keylist* L) {
+  free((void*)L->krow);
+  free((void*)L->vrow);
+  free(L->bias);
+  free(L->s);
+}
+
+static void keylist_push(keylist* L, const uint16_t* k, const uint16_t* v, double bias) {
+  L->krow[L->count] = k;
+  L->vrow[L->count] = v;
+  L->bias[L->count] = bias;
+  L->count++;
+}
+
+static void attend(const keylist* L, const uint16_t* q, int D, double scale, double* out, double* lse) {
+  double qd[1024];
+  for (int d = 0; d < D; ++d) qd[d] = bf16_to_double(q[d]);
+  for (int d = 0; d < D; ++d) out[d] = 0.0;
+  if (L->count == 0) {
+    *lse = -INFINITY;
+    return;
+  }
+  double M = -INFINITY;
+  for (int64_t j = 0; j < L->count; ++j) {
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d) dot += qd[d] * bf16_to_double(L->krow[j][d]);
+    L->s[j] = scale * dot + L->bias[j];
+    if (L->s[j] > M) M = L->s[j];
+  }
+  if (M == -INFINITY) { /* every key carries a -inf bias */
+    *lse = -INFINITY;
+    return;
+  }
+  double denom = 0.0;
+  for (int64_t j = 0; j < L->count; ++j) {
+    double w = exp(L->s[j] - M);
+    denom += w;
+    for (int d = 0; d < D; ++d) out[d] += w * bf16_to_double(L->vrow[j][d]);
+  }
+  for (int d = 0; d < D; ++d) out[d] /= denom;
+  *lse = M + log(denom);
+}
+
+/* ------------------------------------------------------------------ */
+/* a1: ring append                                                     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The sliding part of the cache is a ring of n slots per (sequence, head).
+ * A new token's K/V overwrite the slot at the write pointer, then the pointer
+ * advances cyclically and the valid count saturates at n
+ * ([SR-SWA explainer] "环形缓冲": the newest token overwrites the oldest slot
+ * in place and the write pointer wraps; [R-SWA tutorial] §3.3.2: a window of
+ * at most n entries to which each new K/V is appended, the oldest dropped).
+ * slot_out[b] receives the slot written (nullable).
+ * Pinned by: the closed form slot_s = (wp0 + s) mod n, fill = min(n, T)
+ * ([R-SWA summary] §二.2, C(T) = L_m + min(n, T)) and by a deque(maxlen=n)
+ * model of the ring's contents.
+ */
+void oracle_append(int B, int H, int n, int D, uint16_t* ring_k, uint16_t* ring_v, const uint16_t* k_new,
+                   const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out) {
+  for (int b = 0; b < B; ++b) {
+    int32_t slot = wp[b];
+    for (int h = 0; h < H; ++h) {
+      int64_t dst = (((int64_t)b * H + h) * n + slot) * D;
+      int64_t src = ((int64_t)b * H + h) * D;
+      memcpy(ring_k + dst, k_new + src, sizeof(uint16_t) * (size_t)D);
+      memcpy(ring_v + dst, v_new + src, sizeof(uint16_t) * (size_t)D);
+    }
+    wp[b] = (slot + 1 == n) ? 0 : slot + 1;
+    if (fill[b] < n) fill[b] = fill[b] + 1;
+    if (slot_out) slot_out[b] = slot;
+  }
+}
+
+/* The ring's valid slots: the fill[b] most recently written ones, i.e. the
+ * slots (wp - fill + i) mod n for i in [0, fill). Their order does not
+ * matter to a softmax. */
+static void push_ring(keylist* L, const uint16_t* ring_k, const uint16_t* ring_v, int64_t bh, int n, int D,
+                      int32_t wp, int32_t fill) {
+  for (int32_t i = 0; i < fill; ++i) {
+    int64_t slot = pos_mod((int64_t)wp - fill + i, n);
+    int64_t off = (bh * n + slot) * D;
+    keylist_push(L, ring_k + off, ring_v + off, 0.0);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* a2+a3: R-SWA decode (one query per sequence and head)               */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Each query attends to every prefix token (all page visual tokens plus the
+ * prompt, never evicted) and to the valid ring slots, which after this step's
+ * append include the query's own token
+ * ([R-SWA summary] §二.1; [R-SWA tutorial] §2.2.1 and §3.3.2, where the new
+ * K/V is appended to the window before the attention read).
+ * out [B][H][D], lse [B][H] (natural log).
+ * Pinned by: n >= T reduces to full causal attention; brute force against an
+ * explicit R-SWA mask on a flat timeline ([R-SWA tutorial] §3.3.1); m = 0 with
+ * one valid slot gives o = v_self; constant V gives o = V.
+ */
+void oracle_rswa_decode(int B, int H, int D, int n, int64_t cap, const uint16_t* q, const uint16_t* pk,
+                        const uint16_t* pv, const int32_t* prefix_len, const uint16_t* ring_k,
+                        const uint16_t* ring_v, const int32_t* wp, const int32_t* fill, double scale, double* out,
+                        double* lse) {
+  int64_t BH = (int64_t)B * H;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, cap + n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+      int64_t b = bh / H;
+      L.count = 0;
+      for (int64_t j = 0; j < prefix_len[b]; ++j) {
+        int64_t off = (bh * cap + j) * D;
+        keylist_push(&L, pk + off, pv + off, 0.0);
+      }
+      push_ring(&L, ring_k, ring_v, bh, n, D, wp[b], fill[b]);
+      attend(&L, q + bh * D, D, scale, out + bh * D, lse + bh);
+    }
+    keylist_free(&L);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* a4: R-SWA prefill rows                                              */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Output-side query i (0 <= i < T) of a chunk sees every prefix token and the
+ * output tokens j with i - n < j <= i: the most recent n outputs including
+ * itself ([R-SWA tutorial] §3.3.1 mask: reference positions always visible,
+ * only the most recent n output positions visible). Positions j < 0 belong
+ * to a previous chunk and are read from the ring (position -r is the r-th
+ * most recently written slot, (wp - r) mod n, present when r <= fill).
+ * Only the listed rows are computed: out [B][H][nrows][D], lse [B][H][nrows].
+ * Pinned by: n >= T with an empty ring reduces to causal attention over
+ * [prefix; outputs] with the prefix fully visible; row i equals a decode step
+ * after appending outputs 0..i; a two-chunk run equals a one-chunk run.
+ */
+void oracle_rswa_prefill(int B, int H, int D, int n, int64_t cap, int T, const uint16_t* q, const uint16_t* k_out,
+                         const uint16_t* v_out, const uint16_t* pk, const uint16_t* pv, const int32_t* prefix_len,
+                         const uint16_t* ring_k, const uint16_t* ring_v, const int32_t* wp, const int32_t* fill,
+                         double scale, const int32_t* rows, int nrows, double* out, double* lse) {
+  int64_t work = (int64_t)B * H * nrows;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, cap + n + 1);
+#pragma omp for schedule(dynamic, 8)
+    for (int64_t w = 0; w < work; ++w) {
+      int64_t bh = w / nrows;
+      int64_t r = w % nrows;
+      int64_t b = bh / H;
+      int64_t i = rows[r];
+      L.count = 0;
+      for (int64_t j = 0; j < prefix_len[b]; ++j) {
+        int64_t off = (bh * cap + j) * D;
+        keylist_push(&L, pk + off, pv + off, 0.0);
+      }
+      for (int64_t j = i - n + 1; j <= i; ++j) {
+        if (j >= 0) {
+          int64_t off = (bh * T + j) * D;
+          keylist_push(&L, k_out + off, v_out + off, 0.0);
+        } else if (ring_k != NULL) {
+          int64_t back = -j; /* 1 = most recent previous token */
+          if (back <= fill[b]) {
+            int64_t slot = pos_mod((int64_t)wp[b] - back, n);
+            int64_t off = (bh * n + slot) * D;
+            keylist_push(&L, ring_k + off, ring_v + off, 0.0);
+          }
+        }
+      }
+      attend(&L, q + (bh * T + i) * D, D, scale, out + (bh * nrows + r) * D, lse + bh * nrows + r);
+    }
+    keylist_free(&L);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* a5: block index keys                                                */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The history is cut into blocks of `blk` tokens ([SR-SWA explainer] 稀疏路由
+ * step 1, sparse_block_size 32). A block's index key is the mean of its
+ * tokens' index keys; a partial last block averages only its valid tokens.
+ * Blocks past the prefix are zero.
+ * kbar [B][ceil(cap/blk)][DI].
+ * Pinned by: constant keys within a block, antithetic pairs, and a partial
+ * last block whose invalid tail holds garbage.
+ */
+void oracle_index_pool(int B, int64_t cap, int DI, int blk, const uint16_t* k_idx, const int32_t* prefix_len,
+                       double* kbar) {
+  int64_t nb_cap = (cap + blk - 1) / blk;
+#pragma omp parallel for schedule(static)
+  for (int b = 0; b < B; ++b) {
+    int64_t m = prefix_len[b];
+    for (int64_t c = 0; c < nb_cap; ++c) {
+      double* dst = kbar + ((int64_t)b * nb_cap + c) * DI;
+      for (int d = 0; d < DI; ++d) dst[d] = 0.0;
+      int64_t t0 = c * blk;
+      int64_t t1 = t0 + blk < m ? t0 + blk : m;
+      if (t1 <= t0) continue;
+      for (int64_t t = t0; t < t1; ++t)
+        for (int d = 0; d < DI; ++d) dst[d] += bf16_to_double(k_idx[((int64_t)b * cap + t) * DI + d]);
+      for (int d = 0; d < DI; ++d) dst[d] /= (double)(t1 - t0);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* a7: exact 1.5-entmax                                                */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+  double x;
+  int64_t i;
+} xi_pair;
+
+static int cmp_desc(const void* a, const void* b) {
+  double xa = ((const xi_pair*)a)->x, xb = ((const xi_pair*)b)->x;
+  return (xa < xb) - (xa > xb);
+}
+
+/*
+ * 1.5-entmax of x (x is already (alpha - 1) z = z / 2):
+ *   p_i = max(x_i - tau, 0)^2 with tau fixed by sum_i p_i = 1.
+ * [SR-SWA explainer] 稀疏路由 step 3 names the 1.5-entmax; the form is the
+ * published alpha-entmax (Peters, Niculae & Martins, 2019, "Sparse
+ * Sequence-to-Sequence Models"), solved exactly by their sort-based method:
+ * sort x descending; for k = 1..K let M_k be the mean and S_k the sum of
+ * squares of the k largest, delta_k = (1 - (S_k - k M_k^2)) / k and
+ * tau_k = M_k - sqrt(delta_k); the support size is the largest k with
+ * delta_k >= 0 and tau_k < x_(k), and tau = tau_k there.
+ * Writes p[K] and returns tau. K = 0 returns NaN.
+ * Pinned by: bisection on sum max(x - tau, 0)^2 = 1, the two-element closed
+ * form, uniform inputs, shift invariance, non-negativity and unit sum.
+ */
+double oracle_entmax15(int64_t K, const double* x, double* p) {
+  if (K <= 0) return NAN;
+  xi_pair* s = (xi_pair*)malloc(sizeof(xi_pair) * (size_t)K);
+  for (int64_t i = 0; i < K; ++i) {
+    s[i].x = x[i];
+    s[i].i = i;
+  }
+  qsort(s, (size_t)K, sizeof(xi_pair), cmp_desc);
+  double sum = 0.0, sumsq = 0.0, tau = NAN;
+  for (int64_t k = 1; k <= K; ++k) {
+    double xk = s[k - 1].x;
+    sum += xk;
+    sumsq += xk * xk;
+    double M = sum / (double)k;
+    double delta = (1.0 - (sumsq - (double)k * M * M)) / (double)k;
+    if (delta < 0.0) continue;
+    double tk = M - sqrt(delta);
+    if (tk < xk) tau = tk;
+  }
+  for (int64_t i = 0; i < K; ++i) {
+    double r = x[i] - tau;
+    p[i] = r > 0.0 ? r * r : 0.0;
+  }
+  free(s);
+  return tau;
+}
+
+/* ------------------------------------------------------------------ */
+/* a6-a8: router: block scores, entmax, top-k, log bias                */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+  float z;
+  int64_t c;
+} zc_pair;
+
+/* Descending by the fp32 score; equal scores rank the smaller block first. */
+static int cmp_rank(const void* a, const void* b) {
+  const zc_pair* A = (const zc_pair*)a;
+  const zc_pair* Bp = (const zc_pair*)b;
+  if (A->z > Bp->z) return -1;
+  if (A->z < Bp->z) return 1;
+  return (A->c > Bp->c) - (A->c < Bp->c);
+}
+
+/*
+ * For each sequence b with NB = ceil(prefix_len[b] / blk) candidate blocks:
+ *   z_c   = idx_scale * <q_idx[b], kbar[b][c]>            (step 2: low-dim index score)
+ *   p     = 1.5-entmax(z / 2) over all NB candidates       (step 3)
+ *   sel   = the topk blocks by z, descending, ties to the smaller index (step 4)
+ *   logp  = ln p_c for each selected block (-inf where p_c = 0)   (偏置融合)
+ * ([SR-SWA explainer] 稀疏路由 steps 2-4 and the log-bias fusion; top-16 from
+ * sparse_topk_blocks.) Candidates are prefix blocks only: tokens in the ring
+ * window are not routed. If NB < topk the tail of blk_idx is -1 with logp
+ * -inf. The top-k order is decided on the score rounded to fp32, the
+ * precision the device router ranks in.
+ * Outputs: blk_idx [B][topk], blk_logp [B][topk], probs [B][NBcap] (nullable;
+ * zero past NB), tau [B] (nullable, tau of the x = z/2 problem),
+ * z_out [B][NBcap] (nullable).
+ */
+void oracle_route(int B, int64_t nb_cap, int DI, int blk, const float* q_idx, const double* kbar,
+                  const int32_t* prefix_len, double idx_scale, int topk, int32_t* blk_idx, double* blk_logp,
+                  double* probs, double* tau, double* z_out) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int b = 0; b < B; ++b) {
+    int64_t m = prefix_len[b];
+    int64_t NB = (m + blk - 1) / blk;
+    double* z = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
+    double* x = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
+    double* p = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
+    zc_pair* r = (zc_pair*)malloc(sizeof(zc_pair) * (size_t)(NB > 0 ? NB : 1));
+    for (int64_t c = 0; c < NB; ++c) {
+      double dot = 0.0;
+      for (int d = 0; d < DI; ++d) dot += (double)q_idx[(int64_t)b * DI + d] * kbar[((int64_t)b * nb_cap + c) * DI + d];
+      z[c] = idx_scale * dot;
+      x[c] = z[c] / 2.0;
+    }
+    double t = oracle_entmax15(NB, x, p);
+    for (int64_t c = 0; c < NB; ++c) {
+      r[c].z = (float)z[c];
+      r[c].c = c;
+    }
+    qsort(r, (size_t)NB, sizeof(zc_pair), cmp_rank);
+    for (int k = 0; k < topk; ++k) {
+      int64_t o = (int64_t)b * topk + k;
+      if (k < NB) {
+        int64_t c = r[k].c;
+        blk_idx[o] = (int32_t)c;
+        blk_logp[o] = p[c] > 0.0 ? log(p[c]) : -INFINITY;
+      } else {
+        blk_idx[o] = -1;
+        blk_logp[o] = -INFINITY;
+      }
+    }
+    if (probs)
+      for (int64_t c = 0; c < nb_cap; ++c) probs[(int64_t)b * nb_cap + c] = c < NB ? p[c] : 0.0;
+    if (z_out)
+      for (int64_t c = 0; c < nb_cap; ++c) z_out[(int64_t)b * nb_cap + c] = c < NB ? z[c] : 0.0;
+    if (tau) tau[b] = t;
+    free(z);
+    free(x);
+    free(p);
+    free(r);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* a9: SR-SWA gathered-block decode                                    */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Each query reads only its routed blocks plus the ring window
+ * ([SR-SWA explainer] "三者合起来": a fixed local window plus a fixed number
+ * of remote reference blocks). A token of selected block c scores
+ * scale * <q, k> + logp_c; ring tokens carry no bias; prefix tokens of
+ * unselected blocks are not read. Entries with blk_idx < 0 or logp = -inf are
+ * skipped. The route is shared by all heads of a sequence.
+ * out [B][H][D], lse [B][H].
+ * Pinned by: selecting every block with zero bias equals R-SWA decode; a
+ * uniform bias over all selected blocks with an empty ring is a no-op;
+ * brute force against a dense biased softmax on tiny inputs.
+ */
+void oracle_srswa_decode(int B, int H, int D, int n, int64_t cap, int blk, const uint16_t* q, const uint16_t* pk,
+                         const uint16_t* pv, const int32_t* prefix_len, const int32_t* blk_idx,
+                         const double* blk_logp, int topk, const uint16_t* ring_k, const uint16_t* ring_v,
+                         const int32_t* wp, const int32_t* fill, double scale, double* out, double* lse) {
+  int64_t BH = (int64_t)B * H;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, (int64_t)topk * blk + n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+      int64_t b = bh / H;
+      int64_t m = prefix_len[b];
+      L.count = 0;
+      for (int k = 0; k < topk; ++k) {
+        int64_t c = blk_idx[b * topk + k];
+        double bias = blk_logp[b * topk + k];
+        if (c < 0 || bias == -INFINITY) continue;
+        int64_t t1 = (c + 1) * blk < m ? (c + 1) * blk : m;
+        for (int64_t t = c * blk; t < t1; ++t) {
+          int64_t off = (bh * cap + t) * D;
+          keylist_push(&L, pk + off, pv + off, bias);
+        }
+      }
+      push_ring(&L, ring_k, ring_v, bh, n, D, wp[b], fill[b]);
+      attend(&L, q + bh * D, D, scale, out + bh * D, lse + bh);
+    }
+    keylist_free(&L);
+  }
+}
