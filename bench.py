@@ -1,0 +1,547 @@
+#!/usr/bin/env python
+"""Benchmark of the R-SWA / SR-SWA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+
+A step is one decode step of the whole batch through the C ABI:
+  configs 1, 2 (R-SWA):   rswa_append + rswa_decode
+  configs 4, 5 (SR-SWA):  rswa_append + srswa_route + srswa_decode
+(the router's block index keys are pooled once per prefix, before timing).
+The default workload is the batched R-SWA decode: 512 sequences, 16 heads,
+head_dim 128, a 10-page prefix (2560 visual + 32 prompt tokens) and a full
+128-slot ring with write pointers uniform in [0, 128).
+
+The K timed steps are captured in one CUDA graph and replayed once (after W
+eager warm-up steps and one untimed replay); CUDA events with external
+record nodes bracket every attention-kernel launch inside the graph, so the
+kernel's average duration is measured on its own stream inside the timed
+region. Inputs (the prefix K/V) are larger than L2, so no flush is needed
+between steps. Under torchrun every rank runs its own batch (weak scaling,
+no data-path collective); the timing is the max over ranks.
+
+--impl reference runs the CPU oracle (test infrastructure, fp64) on a bounded
+sample of each step's sequences on the host cores and reports the same
+metric, extrapolated from the sample.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode attn steps/s & achieved HBM GB/s (fraction of peak) on 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def workload(cfg: int) -> dict:
+    from long_context_decode_swa_b200 import synth
+    if cfg == 1:
+        m = synth.ocr_prefix_len(1)
+        return dict(kind="rswa", B=1, H=16, D=128, n=128, plen=[m], cap=m, wp0=37,
+                    name="R-SWA decode, 1 sequence, 16 heads, head_dim 128, prefix 288 (256 visual + 32 prompt), "
+                         "full 128-slot ring from slot 37")
+    if cfg == 2:
+        m = synth.ocr_prefix_len(10)
+        return dict(kind="rswa", B=512, H=16, D=128, n=128, plen=[m] * 512, cap=m, wp0=None,
+                    name="R-SWA batched decode, 512 sequences, 16 heads, head_dim 128, prefix 2592 "
+                         "(10 pages x 256 visual + 32 prompt), full 128-slot ring, wp ~ U[0,128)")
+    if cfg == 4:
+        return dict(kind="srswa", B=64, H=16, D=128, n=128, plen=[32768] * 64, cap=32768, wp0=None,
+                    name="SR-SWA decode, 64 sequences, 16 heads, head_dim 128, 32768-token history (1024 blocks "
+                         "of 32), index dim 32, 1.5-entmax top-16 + log-prob bias, full 128-slot ring")
+    if cfg == 5:
+        pages = synth.log_uniform_pages(16, 32, 400, seed=5005)
+        plen = [256 * p for p in pages]
+        return dict(kind="srswa", B=16, H=16, D=128, n=128, plen=plen, cap=102400, wp0=None,
+                    name="SR-SWA long-horizon decode, 16 sequences, 16 heads, head_dim 128, ragged histories "
+                         "8192-102400 tokens (log-uniform pages x 256), top-16 blocks + 128-slot ring")
+    raise SystemExit(f"config {cfg} is not a decode benchmark here")
+
+
+def algorithmic_bytes(w: dict, blk_rows=None) -> dict:
+    """Bytes the method must move per attention launch (and per route launch).
+
+    R-SWA: per (b, h): (prefix_len + ring fill) K and V rows of 256 B each, the
+    query (256 B), the f32 output (512 B) and lse (4 B).
+    SR-SWA: the same with the routed blocks' valid rows in place of the prefix.
+    Router: per sequence the block keys (128 B per block), q_idx (128 B) and the
+    top-k outputs (8 B each).
+    """
+    H, n = w["H"], w["n"]
+    per_q = 256 + 512 + 4
+    if w["kind"] == "rswa":
+        attn = sum((m + n) * 512 + per_q for m in w["plen"]) * H
+        return dict(attn=attn, route=0)
+    rows = blk_rows if blk_rows is not None else [16 * 32] * w["B"]
+    attn = sum((r + n) * 512 + per_q for r in rows) * H
+    route = sum(((m + 31) // 32) * 128 + 128 + 16 * 8 for m in w["plen"])
+    return dict(attn=attn, route=route)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self, t_begin: float, t_end: float) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            rows.append((ts, parts))
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        inside = [p for ts, p in rows if t_begin - 0.15 <= ts <= t_end + 0.15] or [p for _, p in rows[-3:]]
+        sm = [float(p[2]) for p in inside if p[2].replace(".", "").isdigit()]
+        smax = [float(p[3]) for p in inside if p[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(inside),
+                "power_w_max": max((float(p[4]) for p in inside if p[4].replace(".", "").isdigit()), default=None)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(sparse: bool) -> str:
+    files = ["decode.cu", "common.cuh", "internal.h"]
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", f), "rb").read())
+    h.update(b"sparse" if sparse else b"dense")
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(key: str, src_hash: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    try:
+        for line in open(p):
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == key and parts[1] == src_hash:
+                return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Problem:
+    """Device-resident inputs and state of one rank's batch, plus the step function."""
+
+    def __init__(self, w: dict, steps_total: int, seed: int):
+        import torch
+
+        import long_context_decode_swa_b200 as rswa
+        from long_context_decode_swa_b200 import synth
+        self.rswa = rswa
+        self.w = w
+        B, H, D, n = w["B"], w["H"], w["D"], w["n"]
+        self.c = synth.decode_case(B, H, D, w["plen"], w["cap"], n, steps_total, seed=seed, device="cuda",
+                                   wp0=w["wp0"], fill0=n, poison=False)
+        self.dims = rswa.dims_of(self.c.pk, self.c.ring_k)
+        self.ws = rswa.new_workspace(self.dims, rswa.OP_DECODE)
+        self.out = torch.empty((B, H, D), dtype=torch.float32, device="cuda")
+        self.lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
+        self.sparse = w["kind"] == "srswa"
+        if self.sparse:
+            n_dirs = 32
+            pl = synth.plant_router_keys(w["plen"], w["cap"], n_dirs=n_dirs, seed=seed + 1, device="cuda")
+            nb_cap = (w["cap"] + 31) // 32
+            self.kbar = torch.empty((B, nb_cap, 32), dtype=torch.float32, device="cuda")
+            rswa.srswa_index_pool(pl.k_idx, self.c.prefix_len, self.kbar)
+            self.q_idx = pl.q_idx                           # [n_dirs][B][32]
+            self.n_dirs = n_dirs
+            self.blk = torch.empty((B, 16), dtype=torch.int32, device="cuda")
+            self.logp = torch.empty((B, 16), dtype=torch.float32, device="cuda")
+            self.ws_route = rswa.new_workspace(self.dims, rswa.OP_ROUTE)
+            self.ws = rswa.new_workspace(self.dims, rswa.OP_SRSWA_DECODE)
+            del pl
+        torch.cuda.synchronize()
+
+    def step(self, i: int, q=None, k_new=None, v_new=None, ev=None):
+        """Launches one decode step (2 or 3 kernels) on the current stream; returns the launch count."""
+        c, r = self.c, self.rswa
+        q = c.q[i] if q is None else q
+        k_new = c.k_new[i] if k_new is None else k_new
+        v_new = c.v_new[i] if v_new is None else v_new
+        r.rswa_append(c.ring_k, c.ring_v, k_new, v_new, c.wp, c.fill, status=self.ws)
+        if not self.sparse:
+            if ev is not None:
+                ev[0].record()
+            r.rswa_decode(q, c.pk, c.pv, c.prefix_len, c.ring_k, c.ring_v, c.wp, c.fill, self.out, self.ws,
+                          lse=self.lse, scale=c.scale)
+            if ev is not None:
+                ev[1].record()
+            return 2
+        if ev is not None:
+            ev[2].record()
+        r.srswa_route(self.q_idx[i % self.n_dirs], self.kbar, c.prefix_len, self.blk, self.logp, self.ws_route,
+                      prefix_cap=self.w["cap"])
+        if ev is not None:
+            ev[3].record()
+            ev[0].record()
+        r.srswa_decode(q, c.pk, c.pv, c.prefix_len, self.blk, self.logp, c.ring_k, c.ring_v, c.wp, c.fill, self.out,
+                       self.ws, lse=self.lse, scale=c.scale)
+        if ev is not None:
+            ev[1].record()
+        return 3
+
+
+def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
+    import torch
+    K, W = args.steps, args.warmup
+    prob = Problem(w, K + W, seed=1000 * args.config + rank)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            prob.step(K + i)
+    stream.synchronize()
+    # capture the K timed steps, with external event records around the attention (and route) kernels
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(K)]
+    graph = torch.cuda.CUDAGraph()
+    launches = 0
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            launches += prob.step(i, ev=evs[i])
+    graph.replay()                      # untimed replay
+    torch.cuda.synchronize()
+    status = prob.rswa.check_status(prob.ws)
+    if status:
+        raise RuntimeError(f"device status 0x{status:x} during warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record()
+        graph.replay()
+        end.record()
+    end.synchronize()
+    t_wall1 = time.time()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop(t_wall0, t_wall1)
+    ms_total = start.elapsed_time(end)
+    attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    route_ms = [e[2].elapsed_time(e[3]) for e in evs] if prob.sparse else []
+    ms_max = max_over_ranks(world, ms_total)
+    del graph
+
+    # routed rows of the last step (for the SR-SWA byte count)
+    blk_rows = None
+    if prob.sparse:
+        blk = prob.blk.cpu().tolist()
+        lp = prob.logp.cpu().tolist()
+        blk_rows = []
+        for b in range(w["B"]):
+            m = w["plen"][b]
+            blk_rows.append(sum(min(32, m - 32 * c) for c, l in zip(blk[b], lp[b]) if c >= 0 and l > -math.inf))
+    nbytes = algorithmic_bytes(w, blk_rows)
+    attn_avg_s = statistics.mean(attn_ms) / 1e3
+    achieved = nbytes["attn"] / attn_avg_s / 1e9
+    peak, peak_src = measured_peak()
+    key = f"{'srswa' if prob.sparse else 'rswa'}_decode_config{args.config}"
+    traffic = committed_traffic(key, kernel_source_hash(prob.sparse))
+
+    # ---- e2e through the public API: pinned host inputs -> device -> append/decode -> host result ----
+    e2e = run_e2e(prob, K, W)
+    e2e_ms = max_over_ranks(world, e2e["ms"])
+    B, H, D = w["B"], w["H"], w["D"]
+    steps_per_s = world * K / (ms_max / 1e3)
+    res = {
+        "metric": METRIC,
+        "value": steps_per_s,
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms_max / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "storage_dtype": "bf16",
+        "data": "synthetic",
+        "impl": "ours",
+        "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "global_batch": B * world,
+                   "heads": H, "head_dim": D, "ring": w["n"],
+                   "prefix_tokens_mean": statistics.mean(w["plen"]), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (prefix K/V >> 126 MB); no flush" if nbytes["attn"] > 4e8 else
+                         "working set fits in L2; numbers are L2-resident",
+                   "timing": "K steps in one CUDA graph replay, CUDA events"},
+        "qtok_per_s": steps_per_s * B * H,
+        "seq_tok_per_s": steps_per_s * B,
+        "hbm_gbs_step": world * K * (nbytes["attn"] + nbytes["route"]) / (ms_max / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "srswa decode_kernel<true>" if prob.sparse else
+                     "rswa decode_kernel<false>", "achieved": achieved, "peak": peak,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
+                     "fallback 6650 GB/s", "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": nbytes["attn"], "avg_launch_us": attn_avg_s * 1e6},
+        "kernels_us": {"attention": attn_avg_s * 1e6,
+                       **({"route": statistics.mean(route_ms) * 1e3} if route_ms else {})},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "steps/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
+    }
+    return res
+
+
+def run_e2e(prob: Problem, K: int, W: int) -> dict:
+    import torch
+    c = prob.c
+    B, H, D = c.q.shape[1:]
+    pool = min(K, 16)
+    hq = [torch.empty((B, H, D), dtype=torch.bfloat16, pin_memory=True) for _ in range(pool)]
+    hk = [torch.empty((B, H, D), dtype=torch.bfloat16, pin_memory=True) for _ in range(pool)]
+    hv = [torch.empty((B, H, D), dtype=torch.bfloat16, pin_memory=True) for _ in range(pool)]
+    for j in range(pool):
+        hq[j].copy_(c.q[j])
+        hk[j].copy_(c.k_new[j])
+        hv[j].copy_(c.v_new[j])
+    dq = torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda")
+    dk, dv = torch.empty_like(dq), torch.empty_like(dq)
+    hout = torch.empty((B, H, D), dtype=torch.float32, pin_memory=True)
+    hlse = torch.empty((B, H), dtype=torch.float32, pin_memory=True)
+    stream = torch.cuda.Stream()
+
+    def one(j):
+        dq.copy_(hq[j % pool], non_blocking=True)
+        dk.copy_(hk[j % pool], non_blocking=True)
+        dv.copy_(hv[j % pool], non_blocking=True)
+        prob.step(0, q=dq, k_new=dk, v_new=dv)
+        hout.copy_(prob.out, non_blocking=True)
+        hlse.copy_(prob.lse, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for j in range(W):
+            one(j)
+    stream.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record()
+        for j in range(K):
+            one(j)
+        e.record()
+    e.synchronize()
+    h2d = 3 * B * H * D * 2
+    d2h = B * H * D * 4 + B * H * 4
+    return {"ms": s.elapsed_time(e), "h2d": h2d, "d2h": d2h}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arms
+
+def oracle_sample_step(w: dict, sample: int, seed: int):
+    """Inputs for `sample` sequences of the workload, on the host, for the oracle."""
+    from long_context_decode_swa_b200 import synth
+    plen = w["plen"][:sample]
+    cap = max(plen)
+    c = synth.decode_case(sample, w["H"], w["D"], plen, cap, w["n"], 1, seed=seed, wp0=w["wp0"], fill0=w["n"],
+                          poison=False)
+    u = synth.to_u16
+    st = dict(q=u(c.q[0]), k=u(c.k_new[0]), v=u(c.v_new[0]), pk=u(c.pk), pv=u(c.pv), plen=c.prefix_len.numpy(),
+              rk=u(c.ring_k).copy(), rv=u(c.ring_v).copy(), wp=c.wp.numpy().copy(), fill=c.fill.numpy().copy(),
+              scale=c.scale)
+    if w["kind"] == "srswa":
+        pl = synth.plant_router_keys(plen, cap, n_dirs=1, seed=seed + 1)
+        st["k_idx"] = u(pl.k_idx)
+        st["q_idx"] = pl.q_idx[0].numpy()
+    return st
+
+
+def oracle_step(st: dict, w: dict):
+    import oracle
+    oracle.append(st["rk"], st["rv"], st["k"], st["v"], st["wp"], st["fill"])
+    if w["kind"] == "rswa":
+        return oracle.rswa_decode(st["q"], st["pk"], st["pv"], st["plen"], st["rk"], st["rv"], st["wp"], st["fill"],
+                                  st["scale"])
+    kbar = st.get("kbar")
+    if kbar is None:
+        kbar = st["kbar"] = oracle.index_pool(st["k_idx"], st["plen"])   # once per prefix, as on the GPU
+    r = oracle.route(st["q_idx"], kbar, st["plen"])
+    return oracle.srswa_decode(st["q"], st["pk"], st["pv"], st["plen"], r["blk_idx"], r["blk_logp"], st["rk"],
+                               st["rv"], st["wp"], st["fill"], st["scale"])
+
+
+def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
+    import oracle
+    sample = min(w["B"], 2)
+    st = oracle_sample_step(w, sample, seed=77)
+    oracle_step(st, w)                               # warm (and pool the router keys)
+    t0 = time.perf_counter()
+    oracle_step(st, w)
+    one = time.perf_counter() - t0
+    # grow the sample to fill about budget_s of CPU work
+    sample = int(max(1, min(w["B"], sample * budget_s / max(one, 1e-3) / 3)))
+    st = oracle_sample_step(w, sample, seed=78)
+    oracle_step(st, w)
+    reps, t0 = 0, time.perf_counter()
+    while reps < 2 or (time.perf_counter() - t0 < budget_s and reps < 50):
+        oracle_step(st, w)
+        reps += 1
+    dt = (time.perf_counter() - t0) / reps
+    frac = sample / w["B"]
+    return {"value": frac / dt, "unit": "steps/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{sample} of {w['B']} sequences per step (all heads), {reps} steps timed; "
+                      f"steps/s extrapolated by the sample fraction; fp64 C oracle, OpenMP"}
+
+
+def run_reference(args, w: dict) -> dict:
+    """The oracle as the reference arm, on the host cores, K timed steps of a bounded sample."""
+    import oracle
+    sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1}.get(args.config, 1))
+    st = oracle_sample_step(w, sample, seed=99)
+    for _ in range(args.warmup):
+        oracle_step(st, w)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(st, w)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = (sample / w["B"]) / dt
+    cb = {"value": value, "unit": "steps/s", "cores": oracle.get_threads(), "kind": "oracle",
+          "sample": f"{sample} of {w['B']} sequences per step (all heads); steps/s extrapolated by the sample "
+                    f"fraction; fp64 C oracle on the host cores"}
+    return {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": w["B"]},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = workload(args.config)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    world, rank, local = dist_setup(args)
+    try:
+        res = run_ours(args, w, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

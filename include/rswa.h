@@ -1,0 +1,200 @@
+/*
+ * rswa.h -- C ABI of librswa.so: R-SWA / SR-SWA decode attention on B200 (sm_100a).
+ *
+ * Reference Sliding Window Attention (R-SWA): every query attends to a static
+ * reference prefix of m tokens (all page visual tokens plus the prompt, never
+ * evicted) and to a ring buffer holding the last n generated tokens, so the KV
+ * cache holds L_m + min(n, T) tokens after T generated tokens
+ *   ("百度Unlimited OCR" paper summary, lshu.cn/news/33052, §二.1 核心设计逻辑
+ *    and §二.2 数学与KV缓存优势).
+ * SR-SWA, its sparse successor, cuts the prefix into 32-token blocks, scores
+ * each block against the query with a low-dimensional index projection, runs
+ * a 1.5-entmax over the scores, keeps the top-16 blocks and adds log(prob) of
+ * each kept block as a bias inside the attention softmax
+ *   (Unlimited-OCR-2 SR-SWA explainer, nxmr.cn/news/162408, 稀疏路由 steps 1-4).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers into caller-owned memory, 16-byte
+ *   aligned, dense row-major in the layouts given. The library never
+ *   allocates device memory on a call and never keeps a pointer after a call
+ *   returns (kernels may still be running on `stream`).
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call only enqueues work on it and returns; nothing synchronises
+ *   except rswa_check_status.
+ * - bf16 = IEEE bfloat16 bit pattern (2 bytes); f32 = IEEE binary32.
+ * - Host-side validation runs before any launch. On failure the call returns
+ *   a non-zero rswa_status, launches nothing, and rswa_last_error() describes
+ *   the problem. Values that live in device memory (prefix_len, wp, fill,
+ *   blk_idx) are range-checked inside the kernels: an out-of-range value is
+ *   skipped (its rows are not read) and RSWA_DEVICE_* bits are OR-ed into the
+ *   status word of the workspace (or of `status` for rswa_append), which
+ *   rswa_check_status reads back. No kernel traps.
+ * - Outputs are f32. lse is the natural-log log-sum-exp of the scores a query
+ *   attended to (-inf if it attended to nothing; out is then 0).
+ * - Layout: per (sequence, head) every K/V row of head_dim 128 bf16 is 256
+ *   contiguous bytes, and a sequence's rows for one head are contiguous, so a
+ *   32-token block of one head is one 8 KiB run of memory.
+ */
+#ifndef RSWA_H
+#define RSWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RSWA_API __attribute__((visibility("default")))
+#else
+#define RSWA_API
+#endif
+
+typedef enum {
+  RSWA_OK = 0,
+  RSWA_ERR_INVALID = 1,      /* bad argument (null pointer, size, alignment, too-small workspace) */
+  RSWA_ERR_UNSUPPORTED = 2,  /* valid but not built for (head_dim != 128, too many blocks, ...) */
+  RSWA_ERR_CUDA = 3,         /* a CUDA runtime call failed; see rswa_last_error() */
+  RSWA_ERR_DEVICE_CHECK = 5  /* returned by rswa_check_status when a device-side check tripped */
+} rswa_status;
+
+/* Bits of the device status word. */
+#define RSWA_DEVICE_BAD_PREFIX_LEN 0x1 /* prefix_len[b] < 0 or > prefix_cap: sequence skipped        */
+#define RSWA_DEVICE_BAD_RING_STATE 0x2 /* wp[b] not in [0, n) or fill[b] not in [0, n]: ring skipped */
+#define RSWA_DEVICE_BAD_BLOCK_IDX 0x4  /* blk_idx entry >= number of prefix blocks: entry skipped    */
+#define RSWA_DEVICE_WAIT_TIMEOUT 0x8   /* a bounded pipeline wait gave up (the output is not valid)  */
+
+typedef struct {
+  int32_t batch;      /* B: sequences                                                   */
+  int32_t heads;      /* H: attention heads (query heads == KV heads), 1..128            */
+  int32_t head_dim;   /* D: must be 128                                                  */
+  int32_t ring;       /* n: ring slots per (sequence, head), 1..1024 (the pages use 128) */
+  int64_t prefix_cap; /* cap: rows allocated per (sequence, head) in the prefix K/V      */
+} rswa_dims;
+
+/* Operation codes for rswa_workspace_bytes. */
+#define RSWA_OP_DECODE 1        /* rswa_decode                       */
+#define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode (topk = 16 assumed)  */
+#define RSWA_OP_ROUTE 3         /* srswa_route                       */
+
+/* Message of the last failed call on this host thread ("" if none). */
+RSWA_API const char* rswa_last_error(void);
+
+/* Library ABI version (incremented on any signature change). */
+RSWA_API int32_t rswa_version(void);
+
+/*
+ * Bytes of device workspace `op` needs for these dims. The workspace holds a
+ * status word, per-(sequence, head) completion counters and split-KV
+ * partials. It must be zero-filled once before its first use; every call that
+ * completes leaves the counters at zero again, so it can be reused by later
+ * calls on the same stream. Calls that share a workspace must not overlap in
+ * time (use one workspace per stream). Returns 0 for invalid dims.
+ */
+RSWA_API size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op);
+
+/*
+ * Synchronises `stream`, reads the workspace's device status word into
+ * *device_status (may be NULL) and clears it. Returns RSWA_OK if it was zero,
+ * RSWA_ERR_DEVICE_CHECK otherwise, RSWA_ERR_CUDA if the copy failed.
+ * Also accepts the `status` pointer given to rswa_append (ws_bytes >= 4).
+ */
+RSWA_API rswa_status rswa_check_status(void* workspace, size_t ws_bytes, int32_t* device_status, void* stream);
+
+/*
+ * Ring append (one generated token per sequence).
+ * The new token's K and V overwrite ring slot wp[b] of every head of sequence
+ * b, then wp[b] <- (wp[b] + 1) mod n and fill[b] <- min(fill[b] + 1, n);
+ * slot_out[b] (nullable) receives the slot written.
+ *   (SR-SWA explainer, 环形缓冲: the newest token overwrites the oldest slot in
+ *    place and the write pointer advances cyclically; "百度 Unlimited OCR 深度实战"
+ *    tutorial, chenxutan.com/d/4055.html, §3.3.2: a window of at most n K/V.)
+ * ring_k, ring_v : bf16 [B][H][n][D], updated in place.
+ * k_new, v_new   : bf16 [B][H][D].
+ * wp, fill       : int32 [B], updated in place. The ring's valid slots are the
+ *                  fill[b] most recently written: (wp - fill + i) mod n, i < fill.
+ * slot_out       : int32 [B] or NULL.
+ * status         : int32 device word or NULL; RSWA_DEVICE_BAD_RING_STATE is
+ *                  OR-ed in (and the sequence left untouched) if wp[b] is out of range.
+ */
+RSWA_API rswa_status rswa_append(const rswa_dims* dims, void* ring_k, void* ring_v, const void* k_new, const void* v_new,
+                        int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status, void* stream);
+
+/*
+ * R-SWA decode: for every (b, h), one query attends to prefix rows
+ * [0, prefix_len[b]) and to the ring's valid slots (which, after this step's
+ * rswa_append, include the query's own token):
+ *   out[b][h] = softmax(scale * q K^T) V over that key set.
+ *   (paper summary §二.1; tutorial §2.2.1 and §3.3.1.)
+ * Split-KV flash decoding: each CTA streams 32-row K/V tiles through a shared-
+ * memory pipeline filled by bulk async copies, keeps an online softmax, and
+ * the last CTA of a (b, h) merges the partials by log-sum-exp.
+ * q              : bf16 [B][H][D]
+ * pk, pv         : bf16 [B][H][prefix_cap][D]
+ * prefix_len     : int32 [B], each in [0, prefix_cap]
+ * ring_k, ring_v : bf16 [B][H][n][D];  wp, fill : int32 [B] (as after rswa_append)
+ * scale          : softmax scale (1/sqrt(D) in the model)
+ * out            : f32 [B][H][D];  lse : f32 [B][H] or NULL
+ * workspace      : zero-initialised device buffer of rswa_workspace_bytes(dims, RSWA_OP_DECODE) bytes
+ */
+RSWA_API rswa_status rswa_decode(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
+                        const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
+                        const int32_t* fill, float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * SR-SWA block index keys (run once per prefix, not per step): the prefix is
+ * cut into 32-token blocks and a block's index key is the mean of its tokens'
+ * index keys (a partial last block averages its valid tokens; blocks past
+ * the prefix are written as zero).
+ *   (SR-SWA explainer, 稀疏路由 step 1: sparse_block_size 32.)
+ * k_idx : bf16 [B][prefix_cap][32] per-token index keys
+ * kbar  : f32 [B][ceil(prefix_cap / 32)][32]
+ */
+RSWA_API rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, const int32_t* prefix_len, float* kbar,
+                             void* stream);
+
+/*
+ * SR-SWA router, one route per sequence shared by all heads:
+ *   z_c  = idx_scale * <q_idx[b], kbar[b][c]>   for the NB = ceil(prefix_len/32) prefix blocks
+ *   p    = 1.5-entmax(z / 2), solved exactly (sort-based threshold) in fp32
+ *   blk_idx[b] = the topk blocks by z, descending, equal scores to the smaller index;
+ *                -1 past NB when NB < topk
+ *   blk_logp   = ln p of each selected block (-inf where p = 0 or padded)
+ *   (SR-SWA explainer, 稀疏路由 steps 2-4 and 偏置融合; top-16 = sparse_topk_blocks.)
+ * Ring-window tokens are not candidates.
+ * q_idx    : f32 [B][32]
+ * kbar     : f32 [B][ceil(prefix_cap / 32)][32] from srswa_index_pool
+ * topk     : 1..32
+ * blk_idx  : int32 [B][topk];  blk_logp : f32 [B][topk]
+ * probs    : f32 [B][ceil(prefix_cap / 32)] or NULL (zero past NB)
+ * tau      : f32 [B] or NULL: the threshold of the x = z/2 problem
+ * workspace: zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_ROUTE) bytes
+ * Unsupported: ceil(prefix_cap / 32) > 8192.
+ */
+RSWA_API rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,
+                        float idx_scale, int32_t topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * SR-SWA gathered-block decode: for every (b, h) the query reads only the
+ * selected blocks and the ring. A token of selected block c scores
+ * scale * q.k + blk_logp[b][i]; ring tokens score scale * q.k; entries with
+ * blk_idx < 0 or blk_logp = -inf are skipped.
+ *   (SR-SWA explainer, "三者合起来": a fixed local window plus a fixed number of
+ *    remote reference blocks per decoding step.)
+ * Arguments as rswa_decode, plus blk_idx int32 [B][topk], blk_logp f32 [B][topk],
+ * topk in 1..32. workspace: rswa_workspace_bytes(dims, RSWA_OP_SRSWA_DECODE).
+ */
+RSWA_API rswa_status srswa_decode(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
+                         const int32_t* prefix_len, const int32_t* blk_idx, const float* blk_logp, int32_t topk,
+                         const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
+                         float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSWA_H */

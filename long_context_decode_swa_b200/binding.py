@@ -1,0 +1,248 @@
+"""ctypes binding of librswa.so: argument marshalling only.
+
+Each function takes torch CUDA tensors, checks dtype/device/shape/contiguity,
+and passes ``data_ptr()`` values and the CUDA stream handle to the C entry
+point of the same name (declared in ``include/rswa.h``). Every step of the
+computation runs in the library's kernels; there is no CPU or PyTorch
+fallback: if the library is missing, ``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librswa.so")
+
+OP_DECODE = 1
+OP_SRSWA_DECODE = 2
+OP_ROUTE = 3
+
+STATUS_NAMES = {0: "RSWA_OK", 1: "RSWA_ERR_INVALID", 2: "RSWA_ERR_UNSUPPORTED", 3: "RSWA_ERR_CUDA",
+                5: "RSWA_ERR_DEVICE_CHECK"}
+DEVICE_BAD_PREFIX_LEN = 0x1
+DEVICE_BAD_RING_STATE = 0x2
+DEVICE_BAD_BLOCK_IDX = 0x4
+DEVICE_WAIT_TIMEOUT = 0x8
+
+EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
+            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode")
+
+
+class RswaError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} -> {STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("ring", ctypes.c_int32), ("prefix_cap", ctypes.c_int64)]
+
+    def __repr__(self):
+        return (f"Dims(batch={self.batch}, heads={self.heads}, head_dim={self.head_dim}, ring={self.ring}, "
+                f"prefix_cap={self.prefix_cap})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load librswa.so (building it first if the sources are newer). Raises if unavailable."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if path is None:
+            from . import build as _build
+            try:
+                if not _build.up_to_date():
+                    _build.build()
+            except RuntimeError:
+                if not os.path.exists(p):
+                    raise
+        if not os.path.exists(p):
+            raise RuntimeError(f"librswa.so not found at {p}; run python -m long_context_decode_swa_b200.build")
+        lib = ctypes.CDLL(p)
+        P, I32, I64, F32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        DP = ctypes.POINTER(Dims)
+        sig = {
+            "rswa_last_error": ([], ctypes.c_char_p),
+            "rswa_version": ([], I32),
+            "rswa_workspace_bytes": ([DP, I32], SZ),
+            "rswa_check_status": ([P, SZ, P, P], ctypes.c_int),
+            "rswa_append": ([DP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "rswa_decode": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_index_pool": ([DP, P, P, P, P], ctypes.c_int),
+            "srswa_route": ([DP, P, P, P, F32, I32, P, P, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_decode": ([DP, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise RswaError(fn, code, load().rswa_last_error().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _want(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def dims_of(pk: torch.Tensor, ring_k: torch.Tensor) -> Dims:
+    B, H, cap, D = pk.shape
+    return Dims(B, H, D, ring_k.shape[2], cap)
+
+
+def workspace_bytes(dims: Dims, op: int) -> int:
+    n = load().rswa_workspace_bytes(ctypes.byref(dims), op)
+    if n == 0:
+        raise RswaError("rswa_workspace_bytes", 1, load().rswa_last_error().decode())
+    return int(n)
+
+
+def new_workspace(dims: Dims, op: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace tensor (uint8) sized for `op` (see rswa_workspace_bytes)."""
+    return torch.zeros(workspace_bytes(dims, op), dtype=torch.uint8, device=device or "cuda")
+
+
+def check_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise, read and clear the device status word; returns it (0 = clean)."""
+    st = ctypes.c_int32(0)
+    code = load().rswa_check_status(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    ctypes.byref(st), _stream(stream))
+    if code not in (0, 5):
+        _check("rswa_check_status", code)
+    return int(st.value)
+
+
+def rswa_append(ring_k, ring_v, k_new, v_new, wp, fill, slot_out=None, status=None, stream=None):
+    B, H, n, D = ring_k.shape
+    _want(ring_k, "ring_k", torch.bfloat16)
+    _want(ring_v, "ring_v", torch.bfloat16, ring_k.shape)
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    if status is not None:
+        _want(status, "status", status.dtype)
+    dims = Dims(B, H, D, n, 0)
+    _check("rswa_append", load().rswa_append(ctypes.byref(dims), _ptr(ring_k), _ptr(ring_v), _ptr(k_new), _ptr(v_new),
+                                             _ptr(wp), _ptr(fill), _ptr(slot_out), _ptr(status), _stream(stream)))
+
+
+def rswa_decode(q, pk, pv, prefix_len, ring_k, ring_v, wp, fill, out, workspace, lse=None, scale=None, stream=None):
+    B, H, cap, D = pk.shape
+    n = ring_k.shape[2]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("rswa_decode", load().rswa_decode(ctypes.byref(dims), _ptr(q), _ptr(pk), _ptr(pv), _ptr(prefix_len),
+                                             _ptr(ring_k), _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(out),
+                                             _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def srswa_index_pool(k_idx, prefix_len, kbar, heads: int = 1, stream=None):
+    B, cap, DI = k_idx.shape
+    _want(k_idx, "k_idx", torch.bfloat16)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(kbar, "kbar", torch.float32, (B, (cap + 31) // 32, DI))
+    if DI != 32:
+        raise ValueError("index dim must be 32")
+    dims = Dims(B, heads, 128, 1, cap)
+    _check("srswa_index_pool", load().srswa_index_pool(ctypes.byref(dims), _ptr(k_idx), _ptr(prefix_len), _ptr(kbar),
+                                                       _stream(stream)))
+
+
+def srswa_route(q_idx, kbar, prefix_len, blk_idx, blk_logp, workspace, probs=None, tau=None, idx_scale=1.0,
+                prefix_cap: int | None = None, stream=None):
+    B, nb_cap, DI = kbar.shape
+    topk = blk_idx.shape[1]
+    _want(q_idx, "q_idx", torch.float32, (B, DI))
+    _want(kbar, "kbar", torch.float32)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, topk))
+    if probs is not None:
+        _want(probs, "probs", torch.float32, (B, nb_cap))
+    if tau is not None:
+        _want(tau, "tau", torch.float32, (B,))
+    _want(workspace, "workspace", torch.uint8)
+    cap = nb_cap * 32 if prefix_cap is None else int(prefix_cap)
+    if (cap + 31) // 32 != nb_cap:
+        raise ValueError("prefix_cap does not match kbar's block count")
+    dims = Dims(B, 1, 128, 1, cap)
+    _check("srswa_route", load().srswa_route(ctypes.byref(dims), _ptr(q_idx), _ptr(kbar), _ptr(prefix_len),
+                                             float(idx_scale), topk, _ptr(blk_idx), _ptr(blk_logp), _ptr(probs),
+                                             _ptr(tau), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def srswa_decode(q, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, out, workspace, lse=None,
+                 scale=None, stream=None):
+    B, H, cap, D = pk.shape
+    n = ring_k.shape[2]
+    topk = blk_idx.shape[1]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, topk))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_decode", load().srswa_decode(ctypes.byref(dims), _ptr(q), _ptr(pk), _ptr(pv), _ptr(prefix_len),
+                                               _ptr(blk_idx), _ptr(blk_logp), topk, _ptr(ring_k), _ptr(ring_v),
+                                               _ptr(wp), _ptr(fill), scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                                               workspace.numel(), _stream(stream)))

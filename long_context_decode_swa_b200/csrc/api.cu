@@ -1,0 +1,250 @@
+// api.cu -- the exported C ABI of librswa.so (declared in include/rswa.h).
+//
+// Every entry point validates its arguments on the host before launching
+// anything, records a message for rswa_last_error() on failure, and only
+// enqueues work on the caller's stream.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+rswa_status fail(rswa_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+rswa_status ok() {
+  g_last_error[0] = '\0';
+  return RSWA_OK;
+}
+
+rswa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(RSWA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE_PTR(p)                                                                         \
+  do {                                                                                         \
+    if ((p) == nullptr) return fail(RSWA_ERR_INVALID, "%s: %s must not be NULL", fn, #p);     \
+    if (!aligned16(p)) return fail(RSWA_ERR_INVALID, "%s: %s is not 16-byte aligned", fn, #p); \
+  } while (0)
+
+#define REQUIRE_PTR_OR_NULL(p)                                                                 \
+  do {                                                                                         \
+    if ((p) != nullptr && !aligned16(p))                                                       \
+      return fail(RSWA_ERR_INVALID, "%s: %s is not 16-byte aligned", fn, #p);                  \
+  } while (0)
+
+rswa_status check_dims(const char* fn, const rswa_dims* d, bool need_prefix) {
+  if (d == nullptr) return fail(RSWA_ERR_INVALID, "%s: dims must not be NULL", fn);
+  if (d->batch < 1) return fail(RSWA_ERR_INVALID, "%s: batch must be >= 1 (got %d)", fn, d->batch);
+  if (d->heads < 1 || d->heads > 128) return fail(RSWA_ERR_INVALID, "%s: heads must be in [1, 128] (got %d)", fn, d->heads);
+  if (d->head_dim != rswa::kHeadDim)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: head_dim must be 128 (got %d)", fn, d->head_dim);
+  if (d->ring < 1 || d->ring > 1024) return fail(RSWA_ERR_INVALID, "%s: ring must be in [1, 1024] (got %d)", fn, d->ring);
+  if (need_prefix && (d->prefix_cap < 0 || d->prefix_cap > (int64_t)1 << 30))
+    return fail(RSWA_ERR_INVALID, "%s: prefix_cap out of range (got %lld)", fn, (long long)d->prefix_cap);
+  if (d->batch > 65535) return fail(RSWA_ERR_UNSUPPORTED, "%s: batch above 65535", fn);
+  return RSWA_OK;
+}
+
+int32_t* ws_status(void* ws) { return reinterpret_cast<int32_t*>(ws); }
+
+}  // namespace
+
+namespace rswa {
+int device_sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+}  // namespace rswa
+
+extern "C" {
+
+const char* rswa_last_error(void) { return g_last_error; }
+
+int32_t rswa_version(void) { return 1; }
+
+size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
+  const char* fn = "rswa_workspace_bytes";
+  if (check_dims(fn, dims, true) != RSWA_OK) return 0;
+  switch (op) {
+    case RSWA_OP_DECODE:
+      return rswa::plan_decode_workspace(dims->batch, dims->heads, rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring),
+                                         rswa::device_sm_count())
+          .bytes;
+    case RSWA_OP_SRSWA_DECODE:
+      return rswa::plan_decode_workspace(dims->batch, dims->heads, rswa::decode_max_tiles_sparse(rswa::kMaxTopk, dims->ring),
+                                         rswa::device_sm_count())
+          .bytes;
+    case RSWA_OP_ROUTE:
+      return 256;
+    default:
+      fail(RSWA_ERR_INVALID, "%s: unknown op %d", fn, op);
+      return 0;
+  }
+}
+
+rswa_status rswa_check_status(void* workspace, size_t ws_bytes, int32_t* device_status, void* stream) {
+  const char* fn = "rswa_check_status";
+  if (workspace == nullptr || ws_bytes < 4) return fail(RSWA_ERR_INVALID, "%s: workspace must hold the status word", fn);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, workspace, sizeof host, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "rswa_check_status: reading the status word");
+  if (host != 0) {
+    e = cudaMemsetAsync(workspace, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "rswa_check_status: clearing the status word");
+  }
+  if (device_status) *device_status = host;
+  if (host != 0) return fail(RSWA_ERR_DEVICE_CHECK, "%s: device status 0x%x", fn, host);
+  return ok();
+}
+
+rswa_status rswa_append(const rswa_dims* dims, void* ring_k, void* ring_v, const void* k_new, const void* v_new,
+                        int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status, void* stream) {
+  const char* fn = "rswa_append";
+  rswa_status st = check_dims(fn, dims, false);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(ring_k);
+  REQUIRE_PTR(ring_v);
+  REQUIRE_PTR(k_new);
+  REQUIRE_PTR(v_new);
+  if (wp == nullptr || fill == nullptr) return fail(RSWA_ERR_INVALID, "%s: wp and fill must not be NULL", fn);
+  cudaError_t e = rswa::launch_append(dims->batch, dims->heads, dims->ring, static_cast<uint16_t*>(ring_k),
+                                      static_cast<uint16_t*>(ring_v), static_cast<const uint16_t*>(k_new),
+                                      static_cast<const uint16_t*>(v_new), wp, fill, slot_out, status,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rswa_append: launch");
+  return ok();
+}
+
+static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, const void* pk,
+                                 const void* pv, const int32_t* prefix_len, const int32_t* blk_idx,
+                                 const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
+                                 const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(pk);
+  REQUIRE_PTR(pv);
+  REQUIRE_PTR(ring_k);
+  REQUIRE_PTR(ring_v);
+  REQUIRE_PTR(out);
+  REQUIRE_PTR(workspace);
+  if (prefix_len == nullptr || wp == nullptr || fill == nullptr)
+    return fail(RSWA_ERR_INVALID, "%s: prefix_len, wp and fill must not be NULL", fn);
+  if (sparse) {
+    if (blk_idx == nullptr || blk_logp == nullptr)
+      return fail(RSWA_ERR_INVALID, "%s: blk_idx and blk_logp must not be NULL", fn);
+    if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
+  }
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
+  const int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(rswa::kMaxTopk, dims->ring)
+                                   : rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring);
+  const rswa::WorkspacePlan plan =
+      rswa::plan_decode_workspace(dims->batch, dims->heads, max_tiles, rswa::device_sm_count());
+  if (ws_bytes < plan.bytes)
+    return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes,
+                plan.bytes);
+  rswa::DecodeArgs a;
+  a.B = dims->batch;
+  a.H = dims->heads;
+  a.n = dims->ring;
+  a.cap = dims->prefix_cap;
+  a.splits = plan.splits;
+  a.q = static_cast<const uint16_t*>(q);
+  a.pk = static_cast<const uint16_t*>(pk);
+  a.pv = static_cast<const uint16_t*>(pv);
+  a.prefix_len = prefix_len;
+  a.ring_k = static_cast<const uint16_t*>(ring_k);
+  a.ring_v = static_cast<const uint16_t*>(ring_v);
+  a.wp = wp;
+  a.fill = fill;
+  a.qscale = scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = ws_status(workspace);
+  a.counters = reinterpret_cast<int32_t*>(ws + plan.counters_off);
+  a.partials = reinterpret_cast<float*>(ws + plan.partials_off);
+  a.blk_idx = blk_idx;
+  a.blk_logp = blk_logp;
+  a.topk = sparse ? topk : 0;
+  cudaError_t e = rswa::launch_decode(a, sparse, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+rswa_status rswa_decode(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
+                        const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
+                        const int32_t* fill, float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return decode_common("rswa_decode", false, dims, q, pk, pv, prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp,
+                       fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_decode(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
+                         const int32_t* prefix_len, const int32_t* blk_idx, const float* blk_logp, int32_t topk,
+                         const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
+                         float* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("srswa_decode", true, dims, q, pk, pv, prefix_len, blk_idx, blk_logp, topk, ring_k, ring_v, wp,
+                       fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, const int32_t* prefix_len, float* kbar,
+                             void* stream) {
+  const char* fn = "srswa_index_pool";
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(k_idx);
+  REQUIRE_PTR(kbar);
+  if (prefix_len == nullptr) return fail(RSWA_ERR_INVALID, "%s: prefix_len must not be NULL", fn);
+  if (dims->prefix_cap == 0) return ok();
+  cudaError_t e = rswa::launch_index_pool(dims->batch, dims->prefix_cap, static_cast<const uint16_t*>(k_idx),
+                                          prefix_len, kbar, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,
+                        float idx_scale, int32_t topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  const char* fn = "srswa_route";
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(q_idx);
+  REQUIRE_PTR(kbar);
+  REQUIRE_PTR(workspace);
+  REQUIRE_PTR_OR_NULL(probs);
+  if (prefix_len == nullptr || blk_idx == nullptr || blk_logp == nullptr)
+    return fail(RSWA_ERR_INVALID, "%s: prefix_len, blk_idx and blk_logp must not be NULL", fn);
+  if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
+  if (!std::isfinite(idx_scale)) return fail(RSWA_ERR_INVALID, "%s: idx_scale must be finite", fn);
+  if (ws_bytes < 256) return fail(RSWA_ERR_INVALID, "%s: workspace must be at least 256 bytes", fn);
+  const int64_t nb_cap = (dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock;
+  if (nb_cap > rswa::kMaxRouteBlocks)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: %lld prefix blocks exceed the router's limit of %d", fn,
+                (long long)nb_cap, rswa::kMaxRouteBlocks);
+  if (nb_cap == 0) return fail(RSWA_ERR_INVALID, "%s: prefix_cap must be >= 1", fn);
+  cudaError_t e = rswa::launch_route(dims->batch, dims->prefix_cap, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx,
+                                     blk_logp, probs, tau, ws_status(workspace), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,428 @@
+// decode.cu -- split-KV flash decoding for R-SWA and SR-SWA on sm_100a.
+//
+// One CTA owns a contiguous range of 32-row K/V tiles of one (sequence, head).
+// R-SWA tiles are the prefix rows [0, m) ("百度Unlimited OCR" paper summary
+// §二.1: the reference prefix is always visible) followed by the ring's valid
+// slots (at most two contiguous slot ranges). SR-SWA tiles are the routed
+// 32-token blocks, each carrying its log-probability bias (Unlimited-OCR-2
+// SR-SWA explainer, 稀疏路由 step 4, 偏置融合), followed by the ring.
+//
+// Data movement is HBM-bound (about 1 FLOP per byte), so the kernel spends its
+// effort on bytes in flight, not on tensor cores:
+//  * a producer warp streams each tile's K and V rows (8 KiB each, contiguous
+//    thanks to the [B][H][rows][128] layout) into a 6-stage shared-memory ring
+//    with cp.async.bulk, completing on per-stage mbarriers;
+//  * four consumer warps take tiles round-robin. In a warp, lane (g, c) holds
+//    dims 8c..8c+7 and rows 2j+g; the 16 partial dot products of a half-warp
+//    are reduce-scattered in 15 shuffles so each lane ends with one row's
+//    score; online softmax in the exp2 domain; P.V with a shuffle broadcast
+//    of each row's weight;
+//  * the CTA merges its warps, then either writes the output (one split) or a
+//    (max, sum, acc) partial; the last CTA of a (sequence, head) to finish
+//    (atomic counter) merges the partials by log-sum-exp and resets the
+//    counter.
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rswa {
+
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kStages = 6;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kTileBytes = kBlock * kRowBytes;  // 8 KiB
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct DecodeSmem {
+  uint8_t stage[kStages][2][kTileBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  int rows[kStages];
+  float bias[kStages];  // log2 domain
+  float wm[kConsumerWarps];
+  float wl[kConsumerWarps];
+  float wacc[kConsumerWarps][kHeadDim];
+  int abort_flag;
+  int is_last;
+};
+
+// What one CTA needs to enumerate its (sequence, head)'s tiles.
+struct SeqView {
+  const uint16_t* pk;  // prefix rows of this (b, h)
+  const uint16_t* pv;
+  const uint16_t* rk;  // ring rows of this (b, h)
+  const uint16_t* rv;
+  int m;               // valid prefix rows
+  int nb;              // prefix blocks (SR-SWA)
+  int n_first;         // tiles before the ring (prefix tiles, or topk route entries)
+  int a0, len0, len1;  // ring slot ranges [a0, a0+len0) and [0, len1)
+  int n_r0, n_r1;
+  int total;
+  const int32_t* blk;
+  const float* logp;
+};
+
+template <bool kSparse>
+__device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, bool report) {
+  SeqView v;
+  const int64_t bh = (int64_t)b * a.H + h;
+  int m = a.prefix_len[b];
+  if (m < 0 || m > a.cap) {
+    if (report) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
+    m = 0;
+  }
+  int w = a.wp[b], f = a.fill[b];
+  if (w < 0 || w >= a.n || f < 0 || f > a.n) {
+    if (report) set_status(a.status, RSWA_DEVICE_BAD_RING_STATE);
+    w = 0;
+    f = 0;
+  }
+  v.pk = a.pk + bh * a.cap * kHeadDim;
+  v.pv = a.pv + bh * a.cap * kHeadDim;
+  v.rk = a.ring_k + bh * a.n * kHeadDim;
+  v.rv = a.ring_v + bh * a.n * kHeadDim;
+  v.m = m;
+  v.nb = (m + kBlock - 1) / kBlock;
+  // valid slots are (w - f + i) mod n, i < f; a full ring is read as [0, n)
+  int a0 = f == a.n ? 0 : (w - f) % a.n;
+  if (a0 < 0) a0 += a.n;
+  v.a0 = a0;
+  v.len0 = min(f, a.n - a0);
+  v.len1 = f - v.len0;
+  v.n_r0 = (v.len0 + kBlock - 1) / kBlock;
+  v.n_r1 = (v.len1 + kBlock - 1) / kBlock;
+  v.n_first = kSparse ? a.topk : v.nb;
+  v.total = v.n_first + v.n_r0 + v.n_r1;
+  v.blk = kSparse ? a.blk_idx + (int64_t)b * a.topk : nullptr;
+  v.logp = kSparse ? a.blk_logp + (int64_t)b * a.topk : nullptr;
+  return v;
+}
+
+// Tile t of a (b, h): source rows, row count (0 = empty tile) and log2 bias.
+template <bool kSparse>
+__device__ __forceinline__ void tile_at(const SeqView& v, int t, const uint16_t*& k, const uint16_t*& val, int& rows,
+                                        float& bias, int32_t* status) {
+  bias = 0.f;
+  if (t < v.n_first) {
+    int start;
+    if (kSparse) {
+      const int c = v.blk[t];
+      const float lp = v.logp[t];
+      if (c < 0 || !(lp > -INFINITY)) {
+        rows = 0;
+        k = val = v.pk;
+        return;
+      }
+      if (c >= v.nb) {
+        set_status(status, RSWA_DEVICE_BAD_BLOCK_IDX);
+        rows = 0;
+        k = val = v.pk;
+        return;
+      }
+      start = c * kBlock;
+      bias = lp * kLog2e;
+    } else {
+      start = t * kBlock;
+    }
+    rows = min(kBlock, v.m - start);
+    k = v.pk + (int64_t)start * kHeadDim;
+    val = v.pv + (int64_t)start * kHeadDim;
+    return;
+  }
+  t -= v.n_first;
+  int start, len;
+  if (t < v.n_r0) {
+    start = v.a0 + t * kBlock;
+    len = v.len0 - t * kBlock;
+  } else {
+    t -= v.n_r0;
+    start = t * kBlock;
+    len = v.len1 - t * kBlock;
+  }
+  rows = min(kBlock, len);
+  k = v.rk + (int64_t)start * kHeadDim;
+  val = v.rv + (int64_t)start * kHeadDim;
+}
+
+template <bool kSparse>
+__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
+
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = (int64_t)b * a.H + h;
+
+  const SeqView v = make_view<kSparse>(a, b, h, tid == 0 && split == 0 && h == 0);
+  const int per = (v.total + a.splits - 1) / a.splits;
+  const int t_begin = split * per;
+  const int ntiles = max(0, min(per, v.total - t_begin));
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one lane issues the bulk copies ----------------
+    if (lane == 0) {
+      int issued = 0;
+      bool aborted = false;
+      for (int li = 0; li < ntiles; ++li) {
+        const int s = li % kStages;
+        if (li >= kStages && !mbar_wait(&sm.empty[s], ((li / kStages) - 1) & 1)) {
+          aborted = true;
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) {
+          aborted = true;
+          break;
+        }
+        const uint16_t *kp, *vp;
+        int rows;
+        float bias;
+        tile_at<kSparse>(v, t_begin + li, kp, vp, rows, bias, a.status);
+        sm.rows[s] = rows;
+        sm.bias[s] = bias;
+        if (rows > 0) {
+          const uint32_t bytes = (uint32_t)rows * kRowBytes;
+          mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+          bulk_copy_g2s(sm.stage[s][0], kp, bytes, &sm.full[s]);
+          bulk_copy_g2s(sm.stage[s][1], vp, bytes, &sm.full[s]);
+        } else {
+          mbar_arrive(&sm.full[s]);
+        }
+        issued = li + 1;
+      }
+      if (aborted) {
+        sm.abort_flag = 1;
+        set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
+        // let every copy still in flight land before the CTA's shared memory goes away
+        for (int j = max(0, issued - kStages); j < issued; ++j) mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    const int g = lane >> 4, c = lane & 15;
+    float qf[8];
+    {
+      const uint4 w = *reinterpret_cast<const uint4*>(a.q + bh * kHeadDim + c * 8);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qf[2 * e] = bf16lo(ws[e]) * a.qscale;
+        qf[2 * e + 1] = bf16hi(ws[e]) * a.qscale;
+      }
+    }
+    float m_run = -INFINITY, l_lane = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+
+    for (int li = warp; li < ntiles; li += kConsumerWarps) {
+      const int s = li % kStages;
+      // every lane waits (each needs the acquire), then the warp agrees
+      const bool landed = __all_sync(0xffffffffu, mbar_wait(&sm.full[s], (li / kStages) & 1));
+      if (!landed) {
+        if (lane == 0) {
+          sm.abort_flag = 1;
+          set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
+        }
+        break;
+      }
+      const int rows = sm.rows[s];
+      if (rows > 0) {
+        const float bias = sm.bias[s];
+        const uint8_t* kt = sm.stage[s][0];
+        const uint8_t* vt = sm.stage[s][1];
+        float pd[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint4 w = *reinterpret_cast<const uint4*>(kt + (2 * j + g) * kRowBytes + c * 16);
+          float d = qf[0] * bf16lo(w.x);
+          d = fmaf(qf[1], bf16hi(w.x), d);
+          d = fmaf(qf[2], bf16lo(w.y), d);
+          d = fmaf(qf[3], bf16hi(w.y), d);
+          d = fmaf(qf[4], bf16lo(w.z), d);
+          d = fmaf(qf[5], bf16hi(w.z), d);
+          d = fmaf(qf[6], bf16lo(w.w), d);
+          d = fmaf(qf[7], bf16hi(w.w), d);
+          pd[j] = d;
+        }
+        // reduce-scatter the 16 partial dots over the 16 lanes of this half-warp
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const bool up = c & 8;
+          const float send = up ? pd[i] : pd[i + 8];
+          const float keep = up ? pd[i + 8] : pd[i];
+          pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool up = c & 4;
+          const float send = up ? pd[i] : pd[i + 4];
+          const float keep = up ? pd[i + 4] : pd[i];
+          pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const bool up = c & 2;
+          const float send = up ? pd[i] : pd[i + 2];
+          const float keep = up ? pd[i + 2] : pd[i];
+          pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        }
+        {
+          const bool up = c & 1;
+          const float send = up ? pd[0] : pd[1];
+          const float keep = up ? pd[1] : pd[0];
+          pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        }
+        // this lane now holds the score of tile row 2c + g
+        const float sc = (2 * c + g < rows) ? pd[0] + bias : -INFINITY;
+        const float m_new = fmaxf(m_run, warp_max(sc));
+        const float alpha = exp2f(m_run - m_new);
+        const float p = exp2f(sc - m_new);
+        l_lane = fmaf(l_lane, alpha, p);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+        m_run = m_new;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float pj = __shfl_sync(0xffffffffu, p, (g << 4) | j);
+          if (2 * j + g < rows) {
+            const uint4 w = *reinterpret_cast<const uint4*>(vt + (2 * j + g) * kRowBytes + c * 16);
+            acc[0] = fmaf(pj, bf16lo(w.x), acc[0]);
+            acc[1] = fmaf(pj, bf16hi(w.x), acc[1]);
+            acc[2] = fmaf(pj, bf16lo(w.y), acc[2]);
+            acc[3] = fmaf(pj, bf16hi(w.y), acc[3]);
+            acc[4] = fmaf(pj, bf16lo(w.z), acc[4]);
+            acc[5] = fmaf(pj, bf16hi(w.z), acc[5]);
+            acc[6] = fmaf(pj, bf16lo(w.w), acc[6]);
+            acc[7] = fmaf(pj, bf16hi(w.w), acc[7]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+    }
+    // fold the two half-warps (same dims, different rows) and the lanes' sums
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    const float l = warp_sum(l_lane);
+    if (g == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sm.wacc[warp][c * 8 + e] = acc[e];
+    }
+    if (lane == 0) {
+      sm.wm[warp] = m_run;
+      sm.wl[warp] = l;
+    }
+  }
+  __syncthreads();
+
+  // ---------------- merge the consumer warps ----------------
+  float M = -INFINITY, L = 0.f, A = 0.f;
+  if (tid < kHeadDim) {
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w]);
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float f = exp2f(sm.wm[w] - M);
+        L = fmaf(sm.wl[w], f, L);
+        A = fmaf(sm.wacc[w][tid], f, A);
+      }
+    }
+  }
+  if (a.splits == 1) {
+    if (tid < kHeadDim) {
+      a.out[bh * kHeadDim + tid] = L > 0.f ? A / L : 0.f;
+      if (tid == 0 && a.lse) a.lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    return;
+  }
+  float* rec = a.partials + (bh * a.splits + split) * (kHeadDim + 2);
+  if (tid < kHeadDim) {
+    rec[2 + tid] = A;
+    if (tid == 0) {
+      rec[0] = M;
+      rec[1] = L;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.is_last = (atomicAdd(&a.counters[bh], 1) == a.splits - 1);
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+  if (tid < kHeadDim) {
+    const float* recs = a.partials + bh * a.splits * (kHeadDim + 2);
+    float Mg = -INFINITY;
+    for (int s = 0; s < a.splits; ++s) Mg = fmaxf(Mg, __ldcg(recs + s * (kHeadDim + 2)));
+    float Lg = 0.f, Ag = 0.f;
+    if (Mg > -INFINITY) {
+      for (int s = 0; s < a.splits; ++s) {
+        const float* r = recs + s * (kHeadDim + 2);
+        const float f = exp2f(__ldcg(r) - Mg);
+        Lg = fmaf(__ldcg(r + 1), f, Lg);
+        Ag = fmaf(__ldcg(r + 2 + tid), f, Ag);
+      }
+    }
+    a.out[bh * kHeadDim + tid] = Lg > 0.f ? Ag / Lg : 0.f;
+    if (tid == 0) {
+      if (a.lse) a.lse[bh] = Lg > 0.f ? (Mg + log2f(Lg)) * kLn2 : -INFINITY;
+      a.counters[bh] = 0;
+    }
+  }
+}
+
+}  // namespace
+
+int64_t decode_max_tiles_dense(int64_t cap, int n) {
+  return (cap + kBlock - 1) / kBlock + (n + kBlock - 1) / kBlock + 1;
+}
+
+int64_t decode_max_tiles_sparse(int topk, int n) { return topk + (n + kBlock - 1) / kBlock + 1; }
+
+WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_count) {
+  WorkspacePlan p;
+  const int64_t bh = (int64_t)B * H;
+  // Aim for about four waves of two resident CTAs per SM; never split below
+  // two tiles per CTA, and never beyond 64 splits.
+  const int64_t target = (int64_t)sm_count * 2 * 4;
+  int64_t splits = (target + bh - 1) / bh;
+  splits = std::min<int64_t>(splits, std::max<int64_t>(1, max_tiles / 2));
+  splits = std::max<int64_t>(1, std::min<int64_t>(splits, 64));
+  p.splits = (int)splits;
+  p.counters_off = 256;
+  p.partials_off = p.counters_off + ((size_t)bh * 4 + 255) / 256 * 256;
+  p.bytes = p.partials_off + (p.splits > 1 ? (size_t)bh * p.splits * (kHeadDim + 2) * 4 : 0);
+  return p;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, bool sparse, cudaStream_t stream) {
+  const size_t smem = sizeof(DecodeSmem);
+  const dim3 grid(a.splits, a.H, a.B);
+  static unsigned long long done_sparse = 0, done_dense = 0;
+  if (sparse) {
+    cudaError_t e = ensure_smem_limit(decode_kernel<true>, smem, &done_sparse);
+    if (e != cudaSuccess) return e;
+    decode_kernel<true><<<grid, kDecodeThreads, smem, stream>>>(a);
+  } else {
+    cudaError_t e = ensure_smem_limit(decode_kernel<false>, smem, &done_dense);
+    if (e != cudaSuccess) return e;
+    decode_kernel<false><<<grid, kDecodeThreads, smem, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace rswa

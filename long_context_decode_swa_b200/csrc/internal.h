@@ -1,0 +1,55 @@
+// internal.h -- launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace rswa {
+
+struct DecodeArgs {
+  int B, H, n;
+  int64_t cap;
+  int splits;
+  const uint16_t* q;
+  const uint16_t* pk;
+  const uint16_t* pv;
+  const int32_t* prefix_len;
+  const uint16_t* ring_k;
+  const uint16_t* ring_v;
+  const int32_t* wp;
+  const int32_t* fill;
+  float qscale;  // softmax scale * log2(e)
+  float* out;
+  float* lse;
+  float* partials;   // [B*H][splits][D + 2]
+  int32_t* counters; // [B*H]
+  int32_t* status;
+  // SR-SWA only
+  const int32_t* blk_idx;
+  const float* blk_logp;
+  int topk;
+};
+
+// Workspace layout shared by every op: [status: 256 B][counters][partials].
+struct WorkspacePlan {
+  int splits;
+  size_t counters_off, partials_off, bytes;
+};
+
+WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_count);
+int64_t decode_max_tiles_dense(int64_t cap, int n);
+int64_t decode_max_tiles_sparse(int topk, int n);
+int device_sm_count();
+
+cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_v, const uint16_t* k_new,
+                          const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status,
+                          cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, bool sparse, cudaStream_t stream);
+cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const int32_t* prefix_len, float* kbar,
+                              cudaStream_t stream);
+cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
+                         float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
+                         int32_t* status, cudaStream_t stream);
+
+}  // namespace rswa

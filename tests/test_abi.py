@@ -1,0 +1,109 @@
+"""The C-ABI library loads, exports every entry point include/rswa.h declares,
+and rejects bad arguments on the host before launching anything (these calls
+never reach a CUDA launch, so they run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_decode_swa_b200 as rswa
+from long_context_decode_swa_b200.binding import Dims
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INVALID, UNSUPPORTED = 1, 2
+A = ctypes.c_void_p(0x10000)      # 16-byte aligned stand-in pointers: never dereferenced by a
+A2 = ctypes.c_void_p(0x20000)     # call that fails validation
+MIS = ctypes.c_void_p(0x10008)    # misaligned
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "rswa.h"), encoding="utf-8").read()
+    return sorted(set(re.findall(r"RSWA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_api():
+    assert declared_symbols() == sorted(rswa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = rswa.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.rswa_version() == 1
+
+
+def _err():
+    return rswa.load().rswa_last_error().decode()
+
+
+def test_workspace_bytes_rejects_bad_dims():
+    lib = rswa.load()
+    assert lib.rswa_workspace_bytes(ctypes.byref(Dims(4, 16, 64, 128, 100)), 1) == 0
+    assert "head_dim" in _err()
+    assert lib.rswa_workspace_bytes(ctypes.byref(Dims(0, 16, 128, 128, 100)), 1) == 0
+    assert lib.rswa_workspace_bytes(ctypes.byref(Dims(4, 16, 128, 128, 100)), 99) == 0
+    assert lib.rswa_workspace_bytes(ctypes.byref(Dims(4, 16, 128, 128, 100)), 1) >= 256
+
+
+def test_decode_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64)
+    ws = lib.rswa_workspace_bytes(ctypes.byref(d), 1)
+    args = lambda **kw: [ctypes.byref(kw.get("dims", d)), kw.get("q", A), A, A, A, A, A, A, A,
+                         ctypes.c_float(kw.get("scale", 0.088)), kw.get("out", A), None, A,
+                         ctypes.c_size_t(kw.get("ws", ws)), None]
+    assert lib.rswa_decode(*args(q=None)) == INVALID and "q must not be NULL" in _err()
+    assert lib.rswa_decode(*args(q=MIS)) == INVALID and "aligned" in _err()
+    assert lib.rswa_decode(*args(out=None)) == INVALID
+    assert lib.rswa_decode(*args(scale=0.0)) == INVALID and "scale" in _err()
+    assert lib.rswa_decode(*args(scale=float("nan"))) == INVALID
+    assert lib.rswa_decode(*args(ws=ws - 1)) == INVALID and "workspace" in _err()
+    assert lib.rswa_decode(*args(dims=Dims(2, 4, 96, 128, 64))) == UNSUPPORTED
+    assert lib.rswa_decode(*args(dims=Dims(2, 4, 128, 0, 64))) == INVALID
+    assert lib.rswa_decode(*args(dims=Dims(2, 0, 128, 128, 64))) == INVALID
+
+
+def test_srswa_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64)
+    ws = lib.rswa_workspace_bytes(ctypes.byref(d), 2)
+    base = [ctypes.byref(d), A, A, A, A, A, A, 16, A, A, A, A, ctypes.c_float(0.088), A, None, A, ctypes.c_size_t(ws),
+            None]
+    bad_topk = list(base)
+    bad_topk[7] = 0
+    assert lib.srswa_decode(*bad_topk) == INVALID and "topk" in _err()
+    bad_topk[7] = 33
+    assert lib.srswa_decode(*bad_topk) == INVALID
+    no_idx = list(base)
+    no_idx[5] = None
+    assert lib.srswa_decode(*no_idx) == INVALID and "blk_idx" in _err()
+
+
+def test_route_validation():
+    lib = rswa.load()
+    d = Dims(2, 1, 128, 1, 32 * 8193)
+    call = lambda dims, topk=16, probs=None, ws=256: lib.srswa_route(
+        ctypes.byref(dims), A, A, A, ctypes.c_float(1.0), topk, A, A2, probs, None, A, ctypes.c_size_t(ws), None)
+    assert call(d) == UNSUPPORTED and "limit" in _err()
+    d = Dims(2, 1, 128, 1, 1024)
+    assert call(d, topk=0) == INVALID
+    assert call(d, probs=MIS) == INVALID
+    assert call(d, ws=8) == INVALID
+
+
+def test_append_and_pool_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 0)
+    assert lib.rswa_append(ctypes.byref(d), A, A, None, A, A, A, None, None, None) == INVALID
+    assert lib.rswa_append(ctypes.byref(d), A, A, A, A, None, A, None, None, None) == INVALID
+    assert lib.rswa_append(None, A, A, A, A, A, A, None, None, None) == INVALID
+    assert lib.srswa_index_pool(ctypes.byref(Dims(2, 1, 128, 1, 64)), None, A, A, None) == INVALID
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    t = torch.zeros((1, 1, 4, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        rswa.rswa_append(t, t, t[:, :, 0], t[:, :, 0], torch.zeros(1, dtype=torch.int32),
+                         torch.zeros(1, dtype=torch.int32))
