@@ -65,6 +65,7 @@ typedef enum {
 #define RSWA_DEVICE_BAD_RING_STATE 0x2 /* wp[b] not in [0, n) or fill[b] not in [0, n]: ring skipped */
 #define RSWA_DEVICE_BAD_BLOCK_IDX 0x4  /* blk_idx entry >= number of prefix blocks: entry skipped    */
 #define RSWA_DEVICE_WAIT_TIMEOUT 0x8   /* a bounded pipeline wait gave up (the output is not valid)  */
+#define RSWA_DEVICE_PIPELINE 0x10      /* a pipeline stage held an unexpected tile (output not valid) */
 
 typedef struct {
   int32_t batch;      /* B: sequences                                                   */

@@ -16,7 +16,10 @@ import threading
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "librswa.so")
+# RSWA_LIBRARY selects another build of the same library (for example one
+# compiled with different pipeline-depth constants); default: the in-tree build.
+LIB_PATH = os.environ.get("RSWA_LIBRARY") or os.path.join(_PKG, "librswa.so")
+_DEFAULT_LIB = os.path.join(_PKG, "librswa.so")
 
 OP_DECODE = 1
 OP_SRSWA_DECODE = 2
@@ -28,6 +31,7 @@ DEVICE_BAD_PREFIX_LEN = 0x1
 DEVICE_BAD_RING_STATE = 0x2
 DEVICE_BAD_BLOCK_IDX = 0x4
 DEVICE_WAIT_TIMEOUT = 0x8
+DEVICE_PIPELINE = 0x10
 
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
             "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode")
@@ -59,7 +63,7 @@ def load(path: str | None = None):
         if _lib is not None:
             return _lib
         p = path or LIB_PATH
-        if path is None:
+        if path is None and p == _DEFAULT_LIB:
             from . import build as _build
             try:
                 if not _build.up_to_date():

@@ -30,9 +30,21 @@ namespace rswa {
 
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kStages = 6;
+#ifndef RSWA_DECODE_WARPS
+#define RSWA_DECODE_WARPS 2
+#endif
+#ifndef RSWA_DECODE_STAGES_PER_WARP
+#define RSWA_DECODE_STAGES_PER_WARP 2
+#endif
+// Tile li goes to consumer warp li % kConsumerWarps and to stage li % kStages.
+// kStages is a multiple of kConsumerWarps, so every stage has exactly one
+// consumer warp, which meets that stage's uses in order: the parity of each
+// mbarrier wait then names the right phase (a warp can never wait on a stage
+// two phases ahead of the copy in flight).
+constexpr int kConsumerWarps = RSWA_DECODE_WARPS;
+constexpr int kStages = RSWA_DECODE_WARPS * RSWA_DECODE_STAGES_PER_WARP;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+static_assert(kStages % kConsumerWarps == 0, "each stage needs a single consumer warp");
 constexpr int kTileBytes = kBlock * kRowBytes;  // 8 KiB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -42,7 +54,8 @@ struct DecodeSmem {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   int rows[kStages];
-  float bias[kStages];  // log2 domain
+  int tile_id[kStages];  // producer's tile index for the stage's current use
+  float bias[kStages];   // log2 domain
   float wm[kConsumerWarps];
   float wl[kConsumerWarps];
   float wacc[kConsumerWarps][kHeadDim];
@@ -148,8 +161,10 @@ __device__ __forceinline__ void tile_at(const SeqView& v, int t, const uint16_t*
   val = v.rv + (int64_t)start * kHeadDim;
 }
 
+constexpr int kDecodeMinBlocks = (227 * 1024) / (int)sizeof(DecodeSmem) > 0 ? (227 * 1024) / (int)sizeof(DecodeSmem) : 1;
+
 template <bool kSparse>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
 
@@ -193,6 +208,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
         tile_at<kSparse>(v, t_begin + li, kp, vp, rows, bias, a.status);
         sm.rows[s] = rows;
         sm.bias[s] = bias;
+        sm.tile_id[s] = li;
         if (rows > 0) {
           const uint32_t bytes = (uint32_t)rows * kRowBytes;
           mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
@@ -236,6 +252,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
         if (lane == 0) {
           sm.abort_flag = 1;
           set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
+        }
+        break;
+      }
+      if (sm.tile_id[s] != li) {  // protocol check: never compute on another tile's data
+        if (lane == 0) {
+          sm.abort_flag = 1;
+          set_status(a.status, RSWA_DEVICE_PIPELINE);
         }
         break;
       }
@@ -330,33 +353,37 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
   __syncthreads();
 
   // ---------------- merge the consumer warps ----------------
-  float M = -INFINITY, L = 0.f, A = 0.f;
-  if (tid < kHeadDim) {
+  // (the CTA may have fewer threads than head dims: each thread takes dims tid, tid + blockDim, ...)
+  float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w]);
-    if (M > -INFINITY) {
+  for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w]);
+  float fw[kConsumerWarps];
+  float L = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float f = exp2f(sm.wm[w] - M);
-        L = fmaf(sm.wl[w], f, L);
-        A = fmaf(sm.wacc[w][tid], f, A);
-      }
-    }
+  for (int w = 0; w < kConsumerWarps; ++w) {
+    fw[w] = M > -INFINITY ? exp2f(sm.wm[w] - M) : 0.f;
+    L = fmaf(sm.wl[w], fw[w], L);
   }
   if (a.splits == 1) {
-    if (tid < kHeadDim) {
-      a.out[bh * kHeadDim + tid] = L > 0.f ? A / L : 0.f;
-      if (tid == 0 && a.lse) a.lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
+      float A = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
+      a.out[bh * kHeadDim + d] = L > 0.f ? A / L : 0.f;
     }
+    if (tid == 0 && a.lse) a.lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     return;
   }
   float* rec = a.partials + (bh * a.splits + split) * (kHeadDim + 2);
-  if (tid < kHeadDim) {
-    rec[2 + tid] = A;
-    if (tid == 0) {
-      rec[0] = M;
-      rec[1] = L;
-    }
+  for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
+    float A = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
+    rec[2 + d] = A;
+  }
+  if (tid == 0) {
+    rec[0] = M;
+    rec[1] = L;
   }
   __threadfence();
   __syncthreads();
@@ -364,24 +391,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
   __syncthreads();
   if (!sm.is_last) return;
   __threadfence();
-  if (tid < kHeadDim) {
-    const float* recs = a.partials + bh * a.splits * (kHeadDim + 2);
-    float Mg = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) Mg = fmaxf(Mg, __ldcg(recs + s * (kHeadDim + 2)));
-    float Lg = 0.f, Ag = 0.f;
-    if (Mg > -INFINITY) {
+  const float* recs = a.partials + bh * a.splits * (kHeadDim + 2);
+  float Mg = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) Mg = fmaxf(Mg, __ldcg(recs + s * (kHeadDim + 2)));
+  float Lg = 0.f;
+  if (Mg > -INFINITY)
+    for (int s = 0; s < a.splits; ++s) {
+      const float* r = recs + s * (kHeadDim + 2);
+      Lg = fmaf(__ldcg(r + 1), exp2f(__ldcg(r) - Mg), Lg);
+    }
+  for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
+    float Ag = 0.f;
+    if (Mg > -INFINITY)
       for (int s = 0; s < a.splits; ++s) {
         const float* r = recs + s * (kHeadDim + 2);
-        const float f = exp2f(__ldcg(r) - Mg);
-        Lg = fmaf(__ldcg(r + 1), f, Lg);
-        Ag = fmaf(__ldcg(r + 2 + tid), f, Ag);
+        Ag = fmaf(__ldcg(r + 2 + d), exp2f(__ldcg(r) - Mg), Ag);
       }
-    }
-    a.out[bh * kHeadDim + tid] = Lg > 0.f ? Ag / Lg : 0.f;
-    if (tid == 0) {
-      if (a.lse) a.lse[bh] = Lg > 0.f ? (Mg + log2f(Lg)) * kLn2 : -INFINITY;
-      a.counters[bh] = 0;
-    }
+    a.out[bh * kHeadDim + d] = Lg > 0.f ? Ag / Lg : 0.f;
+  }
+  if (tid == 0) {
+    if (a.lse) a.lse[bh] = Lg > 0.f ? (Mg + log2f(Lg)) * kLn2 : -INFINITY;
+    a.counters[bh] = 0;
   }
 }
 
@@ -396,9 +426,9 @@ int64_t decode_max_tiles_sparse(int topk, int n) { return topk + (n + kBlock - 1
 WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_count) {
   WorkspacePlan p;
   const int64_t bh = (int64_t)B * H;
-  // Aim for about four waves of two resident CTAs per SM; never split below
-  // two tiles per CTA, and never beyond 64 splits.
-  const int64_t target = (int64_t)sm_count * 2 * 4;
+  // Aim for about four waves of resident CTAs; never split below two tiles
+  // per CTA, and never beyond 64 splits.
+  const int64_t target = (int64_t)sm_count * kDecodeMinBlocks * 4;
   int64_t splits = (target + bh - 1) / bh;
   splits = std::min<int64_t>(splits, std::max<int64_t>(1, max_tiles / 2));
   splits = std::max<int64_t>(1, std::min<int64_t>(splits, 64));

@@ -38,6 +38,15 @@ def test_decode_small_shapes(cuda_lib, plen, n, wp0, fill0, steps):
     _run(cuda_lib, case, steps, set(range(0, steps, 7)) | {steps - 1}, tag=f"plen={plen} n={n}")
 
 
+def test_decode_long_pipelines(cuda_lib):
+    # 80 x 16 (sequence, head) pairs leave one split per pair, so each CTA streams ~36 tiles
+    # through its stage ring (every stage reused many times), with ragged prefix tails
+    plen = [1000 - 7 * (b % 5) for b in range(80)]
+    case = synth.decode_case(80, 16, 128, plen, 1000, 128, 3, seed=102, device="cuda")
+    sample = np.arange(0, 80, 9)
+    _run(cuda_lib, case, 3, {0, 1, 2}, sample=sample, tag="long pipelines")
+
+
 def test_decode_config1_single_sequence(cuda_lib):
     # batch 1, 16 heads, prefix 256 visual + 32 prompt, full 128-slot ring with wp at slot 37, 64 steps
     m = synth.ocr_prefix_len(1)
