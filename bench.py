@@ -343,7 +343,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     traffic = committed_traffic(key, kernel_source_hash(prob.sparse))
 
     # ---- e2e through the public API: pinned host inputs -> device -> append/decode -> host result ----
-    e2e = run_e2e(prob, K, W)
+    e2e = run_e2e(prob, K, W) if not args.no_e2e else {"ms": float("nan"), "h2d": 0, "d2h": 0}
     e2e_ms = max_over_ranks(world, e2e["ms"])
     B, H, D = w["B"], w["H"], w["D"]
     steps_per_s = world * K / (ms_max / 1e3)
@@ -518,10 +518,18 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (a smaller case, e.g. for an ncu capture)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = workload(args.config)
+    if args.batch is not None:
+        reps = (args.batch + len(w["plen"]) - 1) // len(w["plen"])
+        w["plen"] = (w["plen"] * reps)[:args.batch]
+        w["name"] = w["name"].replace(f"{w['B']} sequences", f"{args.batch} sequences")
+        w["B"] = args.batch
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
