@@ -194,6 +194,34 @@ RSWA_API rswa_status srswa_decode(const rswa_dims* dims, const void* q, const vo
                          const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * rswa_decode for callers that cannot allocate device memory (no
+ * counterpart on the pages; this is an interface convenience).
+ * Some callers cannot call cudaMalloc: code inside an allocator-free serving
+ * loop, plugins that only receive raw pointers from a host engine owning all
+ * allocations, or paths that must not touch a caching allocator. This entry
+ * point computes exactly what rswa_decode computes (same arguments minus the
+ * workspace), taking its scratch (status word, completion counters, split
+ * partials) from a 4 MiB array of static device memory inside the library,
+ * which every GPU that loads the library holds until the process exits. It
+ * calls no cudaMalloc/cudaFree and no allocating library routine.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture on the device.
+ * - Every call shares the one array per device: calls whose work overlaps on
+ *   the GPU (other streams, other threads) race and give wrong results.
+ *   Serialise them, e.g. on one stream.
+ * - Each call first zeroes the status word and completion counters it uses.
+ * - status: int32 device word or NULL; if given, it receives this call's
+ *   RSWA_DEVICE_* bits (copied, not OR-ed).
+ * - Dims whose scratch exceeds 4 MiB are rejected with RSWA_ERR_UNSUPPORTED
+ *   (rswa_workspace_bytes(dims, RSWA_OP_DECODE) gives the size needed).
+ */
+RSWA_API rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
+                                         const int32_t* prefix_len, const void* ring_k, const void* ring_v,
+                                         const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
+                                         int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

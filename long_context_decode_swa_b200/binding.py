@@ -34,7 +34,7 @@ DEVICE_WAIT_TIMEOUT = 0x8
 DEVICE_PIPELINE = 0x10
 
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
-            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode")
+            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc")
 
 
 class RswaError(RuntimeError):
@@ -86,6 +86,7 @@ def load(path: str | None = None):
             "srswa_index_pool": ([DP, P, P, P, P], ctypes.c_int),
             "srswa_route": ([DP, P, P, P, F32, I32, P, P, P, P, P, SZ, P], ctypes.c_int),
             "srswa_decode": ([DP, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "rswa_decode_noalloc": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)

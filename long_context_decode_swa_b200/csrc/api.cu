@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -244,6 +245,88 @@ rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* 
   cudaError_t e = rswa::launch_route(dims->batch, dims->prefix_cap, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx,
                                      blk_logp, probs, tau, ws_status(workspace), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+// ---------------------------------------------------------------------------
+// rswa_decode_noalloc: rswa_decode for callers that cannot allocate device
+// memory. Some callers cannot call cudaMalloc at all: code that runs inside an
+// allocator-free serving loop, plugins handed raw pointers by a host engine
+// that owns every allocation, or code paths that must not touch the caching
+// allocator. For them the split-KV scratch (status word, per-(sequence, head)
+// completion counters and partial results) lives in the file-scope device
+// array below instead of a caller-provided workspace. Every GPU that loads
+// this library holds the array until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. The array's
+// name in host code is only a host-side stand-in, so the address is asked of
+// the runtime once per device, with that device current.
+rswa_status noalloc_scratch(const char* fn, uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(RSWA_ERR_UNSUPPORTED, "%s: device ordinal %d >= %d", fn, dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: cudaGetSymbolAddress of the scratch array");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_addr[dev]);
+  return RSWA_OK;
+}
+
+}  // namespace
+
+rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
+                                const int32_t* prefix_len, const void* ring_k, const void* ring_v,
+                                const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
+                                int32_t* status, void* stream) {
+  const char* fn = "rswa_decode_noalloc";
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(pk);
+  REQUIRE_PTR(pv);
+  REQUIRE_PTR(ring_k);
+  REQUIRE_PTR(ring_v);
+  REQUIRE_PTR(out);
+  REQUIRE_PTR_OR_NULL(status);
+  if (prefix_len == nullptr || wp == nullptr || fill == nullptr)
+    return fail(RSWA_ERR_INVALID, "%s: prefix_len, wp and fill must not be NULL", fn);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
+  const rswa::WorkspacePlan plan = rswa::plan_decode_workspace(
+      dims->batch, dims->heads, rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring), rswa::device_sm_count());
+  if (plan.bytes > kNoAllocScratchBytes)
+    return fail(RSWA_ERR_UNSUPPORTED,
+                "%s: these dims need %zu bytes of scratch, above the %zu-byte static scratch; use rswa_decode "
+                "with a caller-provided workspace",
+                fn, plan.bytes, kNoAllocScratchBytes);
+  uint8_t* scratch = nullptr;
+  st = noalloc_scratch(fn, &scratch);
+  if (st != RSWA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: zero the status word and the
+  // completion counters (everything before the partials) before this call.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, plan.partials_off, s);
+  if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: clearing the scratch counters");
+  st = decode_common(fn, false, dims, q, pk, pv, prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp, fill, scale,
+                     out, lse, scratch, kNoAllocScratchBytes, stream);
+  if (st != RSWA_OK) return st;
+  if (status != nullptr) {
+    e = cudaMemcpyAsync(status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: copying the status word");
+  }
   return ok();
 }
 
