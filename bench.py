@@ -58,6 +58,11 @@ def workload(cfg: int) -> dict:
         return dict(kind="rswa", B=512, H=16, D=128, n=128, plen=[m] * 512, cap=m, wp0=None,
                     name="R-SWA batched decode, 512 sequences, 16 heads, head_dim 128, prefix 2592 "
                          "(10 pages x 256 visual + 32 prompt), full 128-slot ring, wp ~ U[0,128)")
+    if cfg == 3:
+        m = synth.ocr_prefix_len(40)
+        return dict(kind="prefill", B=4, H=16, D=128, n=128, plen=[m] * 4, cap=m, T=4096, wp0=None,
+                    name="R-SWA chunked prefill, 4 sequences, 16 heads, head_dim 128, prefix 10272 (40 pages x 256 "
+                         "visual + 32 prompt), 4096 output-side queries, causal band 128")
     if cfg == 4:
         return dict(kind="srswa", B=64, H=16, D=128, n=128, plen=[32768] * 64, cap=32768, wp0=None,
                     name="SR-SWA decode, 64 sequences, 16 heads, head_dim 128, 32768-token history (1024 blocks "
@@ -69,6 +74,14 @@ def workload(cfg: int) -> dict:
                     name="SR-SWA long-horizon decode, 16 sequences, 16 heads, head_dim 128, ragged histories "
                          "8192-102400 tokens (log-uniform pages x 256), top-16 blocks + 128-slot ring")
     raise SystemExit(f"config {cfg} is not a decode benchmark here")
+
+
+def prefill_flops(w: dict) -> float:
+    """FLOPs the method must do per prefill launch: per (b, h) and query i, q.k and p.v over its
+    visible keys (prefix_len + min(n, i + 1)), 2 x 2 x D FLOPs per key."""
+    T, n, D, H = w["T"], w["n"], w["D"], w["H"]
+    band = sum(min(n, i + 1) for i in range(T))
+    return float(sum(4 * D * (m * T + band) for m in w["plen"]) * H)
 
 
 def algorithmic_bytes(w: dict, blk_rows=None) -> dict:
@@ -282,9 +295,51 @@ class Problem:
         return 3
 
 
+class PrefillProblem:
+    """Device-resident inputs of one rank's prefill chunk; a step is one rswa_prefill launch."""
+
+    def __init__(self, w: dict, seed: int):
+        import torch
+
+        import long_context_decode_swa_b200 as rswa
+        from long_context_decode_swa_b200 import synth
+        self.rswa = rswa
+        self.w = w
+        self.d = synth.prefill_case(w["B"], w["H"], w["D"], w["plen"], w["cap"], w["T"], seed=seed, device="cuda",
+                                    poison=False)
+        B, H, T, D = self.d["q"].shape
+        self.out = torch.empty((B, H, T, D), dtype=torch.float32, device="cuda")
+        self.lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+        self.ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        self.sparse = False
+        torch.cuda.synchronize()
+
+    def step(self, i: int, q=None, k_new=None, v_new=None, ev=None):
+        d = self.d
+        if ev is not None:
+            ev[0].record()
+        self.rswa.rswa_prefill(d["q"] if q is None else q, d["k_out"] if k_new is None else k_new,
+                               d["v_out"] if v_new is None else v_new, d["pk"], d["pv"], d["prefix_len"], self.out,
+                               self.ws, lse=self.lse, scale=d["scale"], ring=self.w["n"])
+        if ev is not None:
+            ev[1].record()
+        return 1
+
+
+def measured_tensor_peak(sustained: bool):
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["bf16_tflops_sustained" if sustained else "bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return (1400.0 if sustained else 1590.0), "fallback"
+
+
 def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     import torch
     K, W = args.steps, args.warmup
+    if w["kind"] == "prefill":
+        return run_prefill(args, w, world, rank, local)
     prob = Problem(w, K + W, seed=1000 * args.config + rank)
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
@@ -384,6 +439,104 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
     }
     return res
+
+
+def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
+    import torch
+    K, W = args.steps, args.warmup
+    prob = PrefillProblem(w, seed=1000 * args.config + rank)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            prob.step(i)
+    stream.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            prob.step(i, ev=evs[i])
+    graph.replay()
+    torch.cuda.synchronize()
+    if prob.rswa.check_status(prob.ws):
+        raise RuntimeError("device status set during warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record()
+        graph.replay()
+        end.record()
+    end.synchronize()
+    t1 = time.time()
+    barrier(world)
+    clk = clocks.stop(t0, t1)
+    ms_total = start.elapsed_time(end)
+    ms_max = max_over_ranks(world, ms_total)
+    kern_s = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    del graph
+    flops = prefill_flops(w)
+    sustained = ms_total > 1000.0
+    peak, src = measured_tensor_peak(sustained)
+    achieved = flops / kern_s / 1e12
+    e2e = run_prefill_e2e(prob, K, W) if not args.no_e2e else {"ms": float("nan"), "h2d": 0, "d2h": 0}
+    e2e_ms = max_over_ranks(world, e2e["ms"])
+    B, H, T = w["B"], w["H"], w["T"]
+    value = world * K / (ms_max / 1e3)
+    return {
+        "metric": METRIC, "value": value, "unit": "prefill chunks/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "heads": H,
+                   "head_dim": w["D"], "ring": w["n"], "chunk": T, "prefix_tokens_mean": statistics.mean(w["plen"]),
+                   "parallelism": f"replicas x{world}", "timing": "K launches in one CUDA graph replay, CUDA events"},
+        "qtok_per_s": value * B * H * T,
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (tcgen05)", "achieved": achieved, "peak": peak,
+                     "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)",
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6},
+        "kernels_us": {"prefill": kern_s * 1e6},
+        "gpu_launches": K,
+        "clocks": clk,
+        "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "prefill chunks/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
+    }
+
+
+def run_prefill_e2e(prob: PrefillProblem, K: int, W: int) -> dict:
+    import torch
+    d = prob.d
+    hq = d["q"].cpu().pin_memory()
+    hk = d["k_out"].cpu().pin_memory()
+    hv = d["v_out"].cpu().pin_memory()
+    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k_out"]), torch.empty_like(d["v_out"])
+    hout = torch.empty(prob.out.shape, dtype=torch.float32, pin_memory=True)
+    hlse = torch.empty(prob.lse.shape, dtype=torch.float32, pin_memory=True)
+    stream = torch.cuda.Stream()
+
+    def one(i):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        prob.step(i, q=dq, k_new=dk, v_new=dv)
+        hout.copy_(prob.out, non_blocking=True)
+        hlse.copy_(prob.lse, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            one(i)
+    stream.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record()
+        for i in range(K):
+            one(i)
+        e.record()
+    e.synchronize()
+    return {"ms": s.elapsed_time(e), "h2d": 3 * hq.numel() * 2, "d2h": hout.numel() * 4 + hlse.numel() * 4}
 
 
 def run_e2e(prob: Problem, K: int, W: int) -> dict:
@@ -515,7 +668,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 4, 5])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")

@@ -79,6 +79,7 @@ typedef struct {
 #define RSWA_OP_DECODE 1        /* rswa_decode                       */
 #define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode (topk = 16 assumed)  */
 #define RSWA_OP_ROUTE 3         /* srswa_route                       */
+#define RSWA_OP_PREFILL 4       /* rswa_prefill                      */
 
 /* Message of the last failed call on this host thread ("" if none). */
 RSWA_API const char* rswa_last_error(void);
@@ -144,6 +145,32 @@ RSWA_API rswa_status rswa_decode(const rswa_dims* dims, const void* q, const voi
                         const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
                         const int32_t* fill, float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
                         void* stream);
+
+/*
+ * R-SWA chunked prefill: for every (b, h) and output-side query i in [0, T),
+ *   out[b][h][i] = softmax(scale q_i K^T) V over the prefix rows [0, prefix_len[b])
+ *                  and the chunk's outputs j with i - n < j <= i
+ * (the most recent n outputs including itself). Positions j < 0 belong to a
+ * previous chunk: they are read from the ring when one is given (position -r
+ * is the r-th most recently written slot, (wp - r) mod n, present if r <= fill).
+ *   (tutorial §3.3.1: reference positions always visible, only the most recent
+ *    n output positions visible; paper summary §二.1.)
+ * Tensor cores: tcgen05.mma with TMEM accumulators, operands staged by TMA.
+ * T              : chunk length, >= 1
+ * q, k_out, v_out: bf16 [B][H][T][D]  (the chunk's queries and its own keys/values)
+ * pk, pv         : bf16 [B][H][prefix_cap][D];  prefix_len : int32 [B]
+ * ring_k, ring_v : bf16 [B][H][n][D], wp, fill : int32 [B]; all four NULL when there is
+ *                  no previous chunk (then write_ring must be 0)
+ * out            : f32 [B][H][T][D];  lse : f32 [B][H][T] or NULL
+ * write_ring     : 1 = afterwards leave ring/wp/fill as if the T outputs had been
+ *                  appended in order with rswa_append (launched after the attention)
+ * workspace      : zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_PREFILL) bytes (status word)
+ * Unsupported: B*H*T or B*H*prefix_cap or B*H*n at or above 2^31 rows.
+ */
+RSWA_API rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,
+                                  const void* pk, const void* pv, const int32_t* prefix_len, void* ring_k, void* ring_v,
+                                  int32_t* wp, int32_t* fill, float scale, float* out, float* lse, int32_t write_ring,
+                                  void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * SR-SWA block index keys (run once per prefix, not per step): the prefix is

@@ -24,6 +24,7 @@ _DEFAULT_LIB = os.path.join(_PKG, "librswa.so")
 OP_DECODE = 1
 OP_SRSWA_DECODE = 2
 OP_ROUTE = 3
+OP_PREFILL = 4
 
 STATUS_NAMES = {0: "RSWA_OK", 1: "RSWA_ERR_INVALID", 2: "RSWA_ERR_UNSUPPORTED", 3: "RSWA_ERR_CUDA",
                 5: "RSWA_ERR_DEVICE_CHECK"}
@@ -34,7 +35,7 @@ DEVICE_WAIT_TIMEOUT = 0x8
 DEVICE_PIPELINE = 0x10
 
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
-            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc")
+            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill")
 
 
 class RswaError(RuntimeError):
@@ -87,6 +88,7 @@ def load(path: str | None = None):
             "srswa_route": ([DP, P, P, P, F32, I32, P, P, P, P, P, SZ, P], ctypes.c_int),
             "srswa_decode": ([DP, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "rswa_decode_noalloc": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, P], ctypes.c_int),
+            "rswa_prefill": ([DP, I32, P, P, P, P, P, P, P, P, P, P, F32, P, P, I32, P, SZ, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -251,3 +253,36 @@ def srswa_decode(q, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, f
                                                _ptr(blk_idx), _ptr(blk_logp), topk, _ptr(ring_k), _ptr(ring_v),
                                                _ptr(wp), _ptr(fill), scale, _ptr(out), _ptr(lse), _ptr(workspace),
                                                workspace.numel(), _stream(stream)))
+
+
+def rswa_prefill(q, k_out, v_out, pk, pv, prefix_len, out, workspace, lse=None, ring_k=None, ring_v=None, wp=None,
+                 fill=None, write_ring=False, scale=None, ring: int | None = None, stream=None):
+    """Chunked R-SWA prefill. q/k_out/v_out bf16 [B][H][T][D]; out f32 [B][H][T][D]."""
+    B, H, T, D = q.shape
+    cap = pk.shape[2]
+    _want(q, "q", torch.bfloat16)
+    _want(k_out, "k_out", torch.bfloat16, q.shape)
+    _want(v_out, "v_out", torch.bfloat16, q.shape)
+    _want(pk, "pk", torch.bfloat16, (B, H, cap, D))
+    _want(pv, "pv", torch.bfloat16, (B, H, cap, D))
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, T, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H, T))
+    _want(workspace, "workspace", torch.uint8)
+    if ring_k is not None:
+        n = ring_k.shape[2]
+        _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+        _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+        _want(wp, "wp", torch.int32, (B,))
+        _want(fill, "fill", torch.int32, (B,))
+    else:
+        if ring is None:
+            raise ValueError("without a ring tensor, pass the window length as ring=n")
+        n = int(ring)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("rswa_prefill", load().rswa_prefill(ctypes.byref(dims), T, _ptr(q), _ptr(k_out), _ptr(v_out), _ptr(pk),
+                                               _ptr(pv), _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp),
+                                               _ptr(fill), scale, _ptr(out), _ptr(lse), 1 if write_ring else 0,
+                                               _ptr(workspace), workspace.numel(), _stream(stream)))

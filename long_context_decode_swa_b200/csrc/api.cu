@@ -90,6 +90,7 @@ size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
                                          rswa::device_sm_count())
           .bytes;
     case RSWA_OP_ROUTE:
+    case RSWA_OP_PREFILL:
       return 256;
     default:
       fail(RSWA_ERR_INVALID, "%s: unknown op %d", fn, op);
@@ -205,6 +206,69 @@ rswa_status srswa_decode(const rswa_dims* dims, const void* q, const void* pk, c
                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
   return decode_common("srswa_decode", true, dims, q, pk, pv, prefix_len, blk_idx, blk_logp, topk, ring_k, ring_v, wp,
                        fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,
+                         const void* pk, const void* pv, const int32_t* prefix_len, void* ring_k, void* ring_v,
+                         int32_t* wp, int32_t* fill, float scale, float* out, float* lse, int32_t write_ring,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  const char* fn = "rswa_prefill";
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  if (T < 1) return fail(RSWA_ERR_INVALID, "%s: T must be >= 1 (got %d)", fn, T);
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k_out);
+  REQUIRE_PTR(v_out);
+  REQUIRE_PTR(out);
+  REQUIRE_PTR(workspace);
+  REQUIRE_PTR_OR_NULL(lse);
+  if (prefix_len == nullptr) return fail(RSWA_ERR_INVALID, "%s: prefix_len must not be NULL", fn);
+  if (dims->prefix_cap > 0) {
+    REQUIRE_PTR(pk);
+    REQUIRE_PTR(pv);
+  }
+  const bool ring = ring_k != nullptr || ring_v != nullptr || wp != nullptr || fill != nullptr;
+  if (ring) {
+    REQUIRE_PTR(ring_k);
+    REQUIRE_PTR(ring_v);
+    if (wp == nullptr || fill == nullptr) return fail(RSWA_ERR_INVALID, "%s: a ring needs wp and fill", fn);
+  } else if (write_ring) {
+    return fail(RSWA_ERR_INVALID, "%s: write_ring needs a ring", fn);
+  }
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
+  if (ws_bytes < 256) return fail(RSWA_ERR_INVALID, "%s: workspace must be at least 256 bytes", fn);
+  const int64_t bh = (int64_t)dims->batch * dims->heads;
+  const int64_t lim = ((int64_t)1 << 31) - 1;
+  if (bh * T >= lim || bh * dims->prefix_cap >= lim || bh * dims->ring >= lim)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: more than 2^31 rows in one operand", fn);
+  rswa::PrefillLaunch L;
+  L.B = dims->batch;
+  L.H = dims->heads;
+  L.n = dims->ring;
+  L.T = T;
+  L.cap = dims->prefix_cap;
+  L.q = q;
+  L.k_out = k_out;
+  L.v_out = v_out;
+  L.pk = pk;
+  L.pv = pv;
+  L.prefix_len = prefix_len;
+  L.ring_k = ring ? ring_k : nullptr;
+  L.ring_v = ring ? ring_v : nullptr;
+  L.wp = wp;
+  L.fill = fill;
+  L.scale = scale;
+  L.out = out;
+  L.lse = lse;
+  L.write_ring = write_ring ? 1 : 0;
+  L.ring_k_w = ring_k;
+  L.ring_v_w = ring_v;
+  L.wp_w = wp;
+  L.fill_w = fill;
+  L.status = ws_status(workspace);
+  cudaError_t e = rswa::launch_prefill(L, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
 }
 
 rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, const int32_t* prefix_len, float* kbar,

@@ -52,4 +52,31 @@ cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kb
                          float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
                          int32_t* status, cudaStream_t stream);
 
+struct PrefillLaunch {
+  int B, H, n, T;
+  int64_t cap;
+  const void* q;
+  const void* k_out;
+  const void* v_out;
+  const void* pk;
+  const void* pv;
+  const int32_t* prefix_len;
+  const void* ring_k;  // NULL: no previous chunk
+  const void* ring_v;
+  const int32_t* wp;
+  const int32_t* fill;
+  float scale;
+  float* out;
+  float* lse;
+  int write_ring;
+  void* ring_k_w;      // same buffers as ring_k/ring_v/wp/fill, written when write_ring
+  void* ring_v_w;
+  int32_t* wp_w;
+  int32_t* fill_w;
+  int32_t* status;
+};
+
+size_t prefill_smem_bytes();
+cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t stream);
+
 }  // namespace rswa

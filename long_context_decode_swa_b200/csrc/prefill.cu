@@ -1,0 +1,653 @@
+// prefill.cu -- chunked R-SWA prefill on sm_100a tensor cores (tcgen05 + TMEM).
+//
+// Output-side query i of a chunk attends to every reference-prefix token and to
+// the output tokens j with i - n < j <= i ("百度 Unlimited OCR 深度实战" tutorial
+// §3.3.1: reference positions always visible, only the most recent n output
+// positions visible). Positions j < 0 belong to a previous chunk and are read
+// from the ring (the r-th most recent slot is (wp - r) mod n, present when
+// r <= fill).
+//
+// This is the path's one dense contraction, so it runs on the 5th-generation
+// tensor cores. One CTA owns 128 query rows of one (sequence, head):
+//   warp 0, lane 0 : TMA producer of Q and of the K tiles (128 keys x 128 dims)
+//   warp 2, lane 0 : TMA producer of the V tiles
+//   warp 1         : allocates TMEM; lane 0 issues tcgen05.mma (S = Q K^T into
+//                    one of two TMEM S buffers, O += P V into the TMEM O
+//                    accumulator) and tcgen05.commit; the warp zeroes V rows of
+//                    keys that no query may see (so 0 * garbage never reaches O)
+//   warps 4-7      : softmax; thread r owns query row r = TMEM lane r. It loads
+//                    its S row (tcgen05.ld), masks, keeps the running max and sum
+//                    in the exp2 domain, writes its bf16 P row into a 128B-
+//                    swizzled shared-memory tile (the MMA's A operand), and at
+//                    the end normalises its O row and stores it.
+// The running max is only moved when it grows by more than 2^8 (log2 units);
+// the exponentials are then bounded by 256 and the final O / l is the same
+// quotient, so this lazy rescale is exact, and the O read-modify-write through
+// TMEM happens only on those rare steps.
+// Operands: Q, K in K-major SW128 layout (TMA SWIZZLE_128B, boxes of 64 dims x
+// 128 rows); V as the MN-major B operand of O += P V (dims contiguous); P
+// K-major SW128 written by the softmax threads with the same XOR swizzle.
+// Every mbarrier wait is bounded; on expiry the kernel flags
+// RSWA_DEVICE_WAIT_TIMEOUT, drains what it issued and frees its TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rswa {
+
+namespace {
+
+constexpr int kTileRows = 128;                 // query rows per CTA, keys per KV tile
+constexpr int kRegionBytes = kTileRows * 128;  // one 64-column SW128 region of a 128-row tile
+constexpr int kTileBytes = 2 * kRegionBytes;   // 128 x 128 bf16
+constexpr int kPrefillThreads = 256;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr uint32_t kTmemCols = 512;            // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t kColO = 256;
+constexpr float kLazyRescaleLog2 = 8.f;
+constexpr float kLog2eP = 1.4426950408889634f;
+constexpr float kLn2P = 0.6931471805599453f;
+
+struct PrefillCtx {
+  int m, n, fill, wp, T, i0;
+  int np, nr, no, jt0, total;
+  int has_ring;
+};
+
+struct __align__(1024) PrefillSmem {
+  uint8_t q[kTileBytes];
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
+  uint8_t p[2][kTileBytes];
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], s_empty[2], p_full[2];
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  PrefillCtx ctx;
+};
+
+// ---- tcgen05 / TMA wrappers -------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and stride
+// byte offsets (16-byte units), version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;   // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;   // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of kind::f16: f32 accumulate, bf16 A and B, M = N = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16_m128_n128(uint32_t b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+// ---- tile enumeration shared by every role --------------------------------------
+// kind 0: prefix rows [start, start+128); kind 1: ring slots [start, start+128);
+// kind 2: output rows [start, start+128) of this chunk.
+__device__ __forceinline__ void tile_kind(const PrefillCtx& c, int t, int& kind, int& start) {
+  if (t < c.np) {
+    kind = 0;
+    start = t * kTileRows;
+  } else if (t < c.np + c.nr) {
+    kind = 1;
+    start = (t - c.np) * kTileRows;
+  } else {
+    kind = 2;
+    start = (c.jt0 + t - c.np - c.nr) * kTileRows;
+  }
+}
+
+// Age of ring slot s: 1 for the most recently written slot.
+__device__ __forceinline__ int ring_age(const PrefillCtx& c, int s) {
+  int a = (c.wp - 1 - s) % c.n;
+  if (a < 0) a += c.n;
+  return a + 1;
+}
+
+// Can any query of the chunk see key row `row` of tile (kind, start)?
+__device__ __forceinline__ bool key_exists(const PrefillCtx& c, int kind, int start, int row) {
+  const int x = start + row;
+  if (kind == 0) return x < c.m;
+  if (kind == 1) return x < c.n && ring_age(c, x) <= c.fill;
+  return x < c.T;
+}
+
+// Is key row `row` of tile (kind, start) visible to query position i?
+__device__ __forceinline__ bool key_visible(const PrefillCtx& c, int kind, int start, int row, int i) {
+  const int x = start + row;
+  if (kind == 0) return x < c.m;
+  if (kind == 1) {
+    if (x >= c.n) return false;
+    const int age = ring_age(c, x);
+    return age <= c.fill && age < c.n - i;
+  }
+  return x < c.T && x <= i && x > i - c.n;
+}
+
+struct PrefillArgs {
+  int B, H, n, T;
+  int64_t cap;
+  const int32_t* prefix_len;
+  const int32_t* wp;
+  const int32_t* fill;
+  int has_ring;
+  float qk_scale_log2;
+  float* out;
+  float* lse;
+  int32_t* status;
+};
+
+__device__ __forceinline__ bool wait_or_abort(PrefillSmem& sm, uint64_t* bar, uint32_t parity, int32_t* status) {
+  if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) return false;
+  if (mbar_wait(bar, parity)) return true;
+  sm.abort_flag = 1;
+  set_status(status, RSWA_DEVICE_WAIT_TIMEOUT);
+  return false;
+}
+
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_ko, const __grid_constant__ CUtensorMap tm_vo,
+                   const __grid_constant__ CUtensorMap tm_pk, const __grid_constant__ CUtensorMap tm_pv,
+                   const __grid_constant__ CUtensorMap tm_rk, const __grid_constant__ CUtensorMap tm_rv) {
+  extern __shared__ uint8_t smem_raw[];
+  PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = (int64_t)b * a.H + h;
+
+  __shared__ int s_skip;
+  if (tid == 0) {
+    // a CTA of this launch already gave up on a wait: skip the work (the output is flagged invalid)
+    s_skip = a.status != nullptr && (*reinterpret_cast<volatile int32_t*>(a.status) & RSWA_DEVICE_WAIT_TIMEOUT);
+  }
+  __syncthreads();
+  if (s_skip) return;
+
+  if (tid == 0) {
+    PrefillCtx c;
+    int m = a.prefix_len[b];
+    if (m < 0 || m > a.cap) {
+      if (qt == 0 && h == 0) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
+      m = 0;
+    }
+    c.m = m;
+    c.n = a.n;
+    c.T = a.T;
+    c.i0 = qt * kTileRows;
+    c.wp = 0;
+    c.fill = 0;
+    c.has_ring = 0;
+    if (a.has_ring) {
+      const int w = a.wp[b], f = a.fill[b];
+      if (w < 0 || w >= a.n || f < 0 || f > a.n) {
+        if (qt == 0 && h == 0) set_status(a.status, RSWA_DEVICE_BAD_RING_STATE);
+      } else {
+        c.wp = w;
+        c.fill = f;
+        c.has_ring = f > 0 && c.i0 <= a.n - 2;  // some query of the tile can still see a ring slot
+      }
+    }
+    c.np = (m + kTileRows - 1) / kTileRows;
+    c.nr = c.has_ring ? (a.n + kTileRows - 1) / kTileRows : 0;
+    const int jlo = c.i0 - a.n + 1;
+    c.jt0 = jlo > 0 ? jlo / kTileRows : 0;
+    c.no = qt - c.jt0 + 1;
+    c.total = c.np + c.nr + c.no;
+    sm.ctx = c;
+    sm.abort_flag = 0;
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_empty[s], 128);
+      mbar_init(&sm.p_full[s], 128);
+    }
+    mbar_init(&sm.o_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {  // TMEM allocation: one warp, result written to shared memory
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sm.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const PrefillCtx c = sm.ctx;
+  const uint32_t tmem = sm.tmem_base;
+  const int total = c.total;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer: Q and K tiles ----------------
+    const int qrow = (int)(bh * a.T) + c.i0;
+    mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+    tma_load_2d(sm.q, &tm_q, 0, qrow, &sm.q_full);
+    tma_load_2d(sm.q + kRegionBytes, &tm_q, 64, qrow, &sm.q_full);
+    int issued = 0;
+    for (int t = 0; t < total; ++t) {
+      const int s = t & 1;
+      if (t >= 2 && !wait_or_abort(sm, &sm.k_empty[s], ((t >> 1) - 1) & 1, a.status)) break;
+      int kind, start;
+      tile_kind(c, t, kind, start);
+      const CUtensorMap* map = kind == 0 ? &tm_pk : (kind == 1 ? &tm_rk : &tm_ko);
+      const int row = kind == 0 ? (int)(bh * a.cap) + start : (kind == 1 ? (int)(bh * a.n) + start : (int)(bh * a.T) + start);
+      mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
+      tma_load_2d(sm.k[s], map, 0, row, &sm.k_full[s]);
+      tma_load_2d(sm.k[s] + kRegionBytes, map, 64, row, &sm.k_full[s]);
+      issued = t + 1;
+    }
+    if (sm.abort_flag) {  // let the copies in flight land before shared memory is released
+      mbar_wait(&sm.q_full, 0);
+      for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait(&sm.k_full[t & 1], (t >> 1) & 1);
+    }
+  } else if (warp == 2 && lane == 0) {
+    // ---------------- producer: V tiles ----------------
+    int issued = 0;
+    for (int t = 0; t < total; ++t) {
+      const int s = t & 1;
+      if (t >= 2 && !wait_or_abort(sm, &sm.v_empty[s], ((t >> 1) - 1) & 1, a.status)) break;
+      int kind, start;
+      tile_kind(c, t, kind, start);
+      const CUtensorMap* map = kind == 0 ? &tm_pv : (kind == 1 ? &tm_rv : &tm_vo);
+      const int row = kind == 0 ? (int)(bh * a.cap) + start : (kind == 1 ? (int)(bh * a.n) + start : (int)(bh * a.T) + start);
+      mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
+      tma_load_2d(sm.v[s], map, 0, row, &sm.v_full[s]);
+      tma_load_2d(sm.v[s] + kRegionBytes, map, 64, row, &sm.v_full[s]);
+      issued = t + 1;
+    }
+    if (sm.abort_flag)
+      for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait(&sm.v_full[t & 1], (t >> 1) & 1);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (lane 0) + V-row zeroing (whole warp) ----------------
+    constexpr uint32_t kIdescQK = idesc_bf16_m128_n128(0);
+    constexpr uint32_t kIdescPV = idesc_bf16_m128_n128(1);
+    const uint32_t q_addr = smem_addr(sm.q);
+    bool ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.q_full, 0, a.status));
+    auto issue_s = [&](int t) {  // S[t&1] = Q K_t^T
+      const uint32_t k_addr = smem_addr(sm.k[t & 1]);
+      const uint32_t d = tmem + (uint32_t)(t & 1) * 128u;
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kRegionBytes + (uint32_t)(kk & 3) * 32u;
+          tc_mma_f16(d, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK,
+                     kk > 0);
+        }
+        tc_commit(&sm.s_full[t & 1]);
+        tc_commit(&sm.k_empty[t & 1]);
+      }
+      __syncwarp();
+    };
+    if (ok && total > 0) {
+      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.k_full[0], 0, a.status));
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+    }
+    for (int t = 0; ok && t < total; ++t) {
+      if (t + 1 < total) {
+        const int u = t + 1, bs = u & 1;
+        ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.k_full[bs], (u >> 1) & 1, a.status));
+        if (ok && u >= 2) ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.s_empty[bs], ((u >> 1) - 1) & 1, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(u);
+      }
+      const int s = t & 1;
+      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.p_full[s], (t >> 1) & 1, a.status));
+      if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.v_full[s], (t >> 1) & 1, a.status));
+      if (!ok) break;
+      // zero V rows of keys no query can see (their P is 0; their bytes may be anything)
+      int kind, start;
+      tile_kind(c, t, kind, start);
+      bool zeroed = false;
+      for (int r = lane; r < kTileRows; r += 32) {
+        if (!key_exists(c, kind, start, r)) {
+          uint4* row0 = reinterpret_cast<uint4*>(sm.v[s] + r * 128);
+          uint4* row1 = reinterpret_cast<uint4*>(sm.v[s] + kRegionBytes + r * 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            row0[e] = make_uint4(0, 0, 0, 0);
+            row1[e] = make_uint4(0, 0, 0, 0);
+          }
+          zeroed = true;
+        }
+      }
+      if (__any_sync(0xffffffffu, zeroed)) fence_async_smem();
+      __syncwarp();
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t p_addr = smem_addr(sm.p[s]);
+        const uint32_t v_addr = smem_addr(sm.v[s]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a_off = (uint32_t)(kk >> 2) * kRegionBytes + (uint32_t)(kk & 3) * 32u;
+          const uint32_t b_off = (uint32_t)kk * 16u * 128u;  // 16 keys = two 8-row groups
+          tc_mma_f16(tmem + kColO, smem_desc_sw128(p_addr + a_off, 16, 1024),
+                     smem_desc_sw128(v_addr + b_off, kRegionBytes, 1024), kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&sm.v_empty[s]);
+        tc_commit(&sm.o_done);
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {  // make sure every MMA this thread issued has finished before TMEM goes away
+      tc_commit(&sm.o_done);
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ---------------- softmax: thread r owns query row r ----------------
+    const int r = tid - kSoftmaxWarp0 * 32;
+    const int i = c.i0 + r;
+    const uint32_t lane_base = (uint32_t)((warp - kSoftmaxWarp0) * 32) << 16;
+    // l normalises O with the same bf16-rounded weights the MMA used; lu (unrounded) gives lse
+    float m_used = -INFINITY, l = 0.f, lu = 0.f;
+    bool ok = true;
+    for (int t = 0; t < total; ++t) {
+      const int s = t & 1;
+      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.s_full[s], (t >> 1) & 1, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      float x[128];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)s * 128u + (uint32_t)ch * 32u, rr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[ch * 32 + e] = __uint_as_float(rr[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.s_empty[s]);
+      int kind, start;
+      tile_kind(c, t, kind, start);
+      float tmax = -INFINITY;
+      if (kind == 1) {
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          x[e] = key_visible(c, kind, start, e, i) ? x[e] * a.qk_scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, x[e]);
+        }
+      } else {
+        // visible columns form one interval (lo, hi]: prefix rows below m; outputs with i - n < j <= i, j < T
+        const int hi = kind == 0 ? min(127, c.m - start - 1) : min(127, min(i, c.T - 1) - start);
+        const int lo = kind == 0 ? -1 : max(-1, i - c.n - start);
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          x[e] = (e > lo && e <= hi) ? x[e] * a.qk_scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, x[e]);
+        }
+      }
+      const bool rescale = tmax > m_used + kLazyRescaleLog2;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = exp2f(m_used - tmax);  // 0 while nothing has been seen
+        l *= alpha;
+        lu *= alpha;
+        m_used = tmax;
+      }
+      uint32_t pk[64];
+      float lsum = 0.f, lusum = 0.f;
+      const float m_sub = m_used == -INFINITY ? 0.f : m_used;  // a row with nothing visible yet: exp2(-inf) = 0
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float p0 = exp2f(x[2 * e] - m_sub);
+        const float p1 = exp2f(x[2 * e + 1] - m_sub);
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
+        lsum += __low2float(pb) + __high2float(pb);
+        lusum += p0 + p1;
+      }
+      l += lsum;
+      lu += lusum;
+      if (t >= 1) {
+        // O and the P buffer are touched below: PV of the previous tile must be complete
+        ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.o_done, (t - 1) & 1, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t rr[32];
+            const uint32_t ta = tmem + lane_base + kColO + (uint32_t)ch * 32u;
+            tmem_ld32(ta, rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st32(ta, rr);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row -> 128B-swizzled K-major tile: 16-byte chunk c of row r sits at chunk (c ^ (r & 7))
+      uint8_t* prow0 = sm.p[s] + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const int region = ch >> 3, cc = ch & 7;
+        uint4 val = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(prow0 + region * kRegionBytes + ((cc ^ (r & 7)) << 4)) = val;
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[s]);
+    }
+    if (ok && total > 0) {
+      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.o_done, (total - 1) & 1, a.status));
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* orow = a.out + (bh * a.T + i) * kHeadDim;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + kColO + (uint32_t)ch * 32u, rr);
+        tmem_wait_ld();
+        if (i < c.T) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(orow + ch * 32 + e) =
+                make_float4(__uint_as_float(rr[e]) * inv, __uint_as_float(rr[e + 1]) * inv,
+                            __uint_as_float(rr[e + 2]) * inv, __uint_as_float(rr[e + 3]) * inv);
+        }
+      }
+      if (i < c.T && a.lse) a.lse[bh * a.T + i] = lu > 0.f ? (m_used + log2f(lu)) * kLn2P : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    if (sm.abort_flag && lane == 0) mbar_wait(&sm.o_done, 0);  // bounded; MMAs drain before TMEM is freed
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ---- writes the chunk's last min(T, n) output K/V rows into the ring ----------
+__global__ void ring_from_outputs_kernel(int H, int n, int T, const uint16_t* __restrict__ k_out,
+                                         const uint16_t* __restrict__ v_out, uint16_t* __restrict__ ring_k,
+                                         uint16_t* __restrict__ ring_v, int32_t* wp, int32_t* fill, int32_t* status) {
+  __shared__ int s_wp;
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) {
+    const int w = wp[b], f = fill[b];
+    const bool ok = w >= 0 && w < n && f >= 0 && f <= n;
+    if (!ok) set_status(status, RSWA_DEVICE_BAD_RING_STATE);
+    s_wp = ok ? w : -1;
+  }
+  __syncthreads();
+  const int w = s_wp;
+  if (w < 0) return;
+  const int keep = min(T, n);
+  constexpr int kVec = kHeadDim / 8;
+  const int work = keep * H * kVec * 2;
+  for (int idx = threadIdx.x; idx < work; idx += blockDim.x) {
+    const int which = idx / (keep * H * kVec);
+    const int rem = idx - which * keep * H * kVec;
+    const int k = rem / (H * kVec);
+    const int hh = (rem / kVec) % H;
+    const int e = rem % kVec;
+    const int tok = T - keep + k;                           // output position
+    const int slot = (int)(((int64_t)w + tok) % n);         // the slot the tok-th append would write
+    const int64_t bh = (int64_t)b * H + hh;
+    const uint4* src = reinterpret_cast<const uint4*>((which ? v_out : k_out) + (bh * T + tok) * kHeadDim) + e;
+    uint4* dst = reinterpret_cast<uint4*>((which ? ring_v : ring_k) + (bh * n + slot) * kHeadDim) + e;
+    *dst = *src;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    wp[b] = (int)(((int64_t)w + T) % n);
+    const int64_t nf = (int64_t)fill[b] + T;
+    fill[b] = (int)(nf < n ? nf : n);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// A [rows][128] bf16 matrix as a 2D tensor map with 64 x 128 boxes and 128B swizzle.
+cudaError_t make_rows_map(CUtensorMap* map, const void* base, int64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kTileRows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t prefill_smem_bytes() { return sizeof(PrefillSmem) + 1024; }
+
+cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t stream) {
+  CUtensorMap tq, tko, tvo, tpk, tpv, trk, trv;
+  const int64_t bh = (int64_t)L.B * L.H;
+  cudaError_t e;
+  if ((e = make_rows_map(&tq, L.q, bh * L.T)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&tko, L.k_out, bh * L.T)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&tvo, L.v_out, bh * L.T)) != cudaSuccess) return e;
+  const int64_t prows = bh * L.cap > 0 ? bh * L.cap : 1;
+  if ((e = make_rows_map(&tpk, L.cap > 0 ? L.pk : L.q, L.cap > 0 ? prows : bh * L.T)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&tpv, L.cap > 0 ? L.pv : L.q, L.cap > 0 ? prows : bh * L.T)) != cudaSuccess) return e;
+  const bool ring = L.ring_k != nullptr;
+  if ((e = make_rows_map(&trk, ring ? L.ring_k : L.q, ring ? bh * L.n : bh * L.T)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&trv, ring ? L.ring_v : L.q, ring ? bh * L.n : bh * L.T)) != cudaSuccess) return e;
+  PrefillArgs a;
+  a.B = L.B;
+  a.H = L.H;
+  a.n = L.n;
+  a.T = L.T;
+  a.cap = L.cap;
+  a.prefix_len = L.prefix_len;
+  a.wp = L.wp;
+  a.fill = L.fill;
+  a.has_ring = ring ? 1 : 0;
+  a.qk_scale_log2 = L.scale * kLog2eP;
+  a.out = L.out;
+  a.lse = L.lse;
+  a.status = L.status;
+  const size_t smem = prefill_smem_bytes();
+  static unsigned long long done = 0;
+  if ((e = ensure_smem_limit(prefill_kernel, smem, &done)) != cudaSuccess) return e;
+  const dim3 grid((L.T + kTileRows - 1) / kTileRows, L.H, L.B);
+  prefill_kernel<<<grid, kPrefillThreads, smem, stream>>>(a, tq, tko, tvo, tpk, tpv, trk, trv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (L.write_ring) {
+    ring_from_outputs_kernel<<<L.B, 256, 0, stream>>>(L.H, L.n, L.T, static_cast<const uint16_t*>(L.k_out),
+                                                      static_cast<const uint16_t*>(L.v_out),
+                                                      static_cast<uint16_t*>(L.ring_k_w),
+                                                      static_cast<uint16_t*>(L.ring_v_w), L.wp_w, L.fill_w, L.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace rswa
