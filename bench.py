@@ -674,6 +674,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (a smaller case, e.g. for an ncu capture)")
+    ap.add_argument("--prefix", type=int, default=None,
+                    help="override every sequence's prefix length (and the capacity) of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -683,6 +685,10 @@ def main():
         w["plen"] = (w["plen"] * reps)[:args.batch]
         w["name"] = w["name"].replace(f"{w['B']} sequences", f"{args.batch} sequences")
         w["B"] = args.batch
+    if args.prefix is not None:
+        w["plen"] = [args.prefix] * w["B"]
+        w["cap"] = args.prefix
+        w["name"] += f" [prefix overridden: {args.prefix}]"
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
