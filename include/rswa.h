@@ -77,7 +77,7 @@ typedef struct {
 
 /* Operation codes for rswa_workspace_bytes. */
 #define RSWA_OP_DECODE 1        /* rswa_decode                       */
-#define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode (topk = 16 assumed)  */
+#define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode (any topk in 1..32)  */
 #define RSWA_OP_ROUTE 3         /* srswa_route                       */
 #define RSWA_OP_PREFILL 4       /* rswa_prefill                      */
 
@@ -199,7 +199,10 @@ RSWA_API rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, 
  * blk_idx  : int32 [B][topk];  blk_logp : f32 [B][topk]
  * probs    : f32 [B][ceil(prefix_cap / 32)] or NULL (zero past NB)
  * tau      : f32 [B] or NULL: the threshold of the x = z/2 problem
- * workspace: zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_ROUTE) bytes
+ * workspace: zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_ROUTE) bytes (status word,
+ *            per-sequence counters, chunk top lists and the block scores)
+ * The scores are computed by ceil(NB / 512) CTAs per sequence; the last one to finish
+ * merges their sorted top-32 lists and solves the threshold.
  * Unsupported: ceil(prefix_cap / 32) > 8192.
  */
 RSWA_API rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,
@@ -241,8 +244,10 @@ RSWA_API rswa_status srswa_decode(const rswa_dims* dims, const void* q, const vo
  * - Each call first zeroes the status word and completion counters it uses.
  * - status: int32 device word or NULL; if given, it receives this call's
  *   RSWA_DEVICE_* bits (copied, not OR-ed).
- * - Dims whose scratch exceeds 4 MiB are rejected with RSWA_ERR_UNSUPPORTED
- *   (rswa_workspace_bytes(dims, RSWA_OP_DECODE) gives the size needed).
+ * - The split-KV work is planned to fit the 4 MiB (it may use fewer splits
+ *   than rswa_decode would); dims that do not fit even with one split (more
+ *   than about a million (sequence, head) pairs) are rejected with
+ *   RSWA_ERR_UNSUPPORTED.
  */
 RSWA_API rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
                                          const int32_t* prefix_len, const void* ring_k, const void* ring_v,

@@ -6,9 +6,9 @@ seeded synthetic-input generators. There is no CPU fallback.
 """
 from .binding import (  # noqa: F401
     EXPORTED, LIB_PATH, OP_DECODE, OP_PREFILL, OP_ROUTE, OP_SRSWA_DECODE, Dims, RswaError, check_status, dims_of,
-    load, new_workspace, rswa_append, rswa_decode, rswa_prefill, srswa_decode, srswa_index_pool, srswa_route,
+    load, new_workspace, route_workspace, rswa_append, rswa_decode, rswa_prefill, srswa_decode, srswa_index_pool, srswa_route,
     workspace_bytes,
 )
 
 __all__ = ["load", "Dims", "RswaError", "rswa_append", "rswa_decode", "rswa_prefill", "srswa_index_pool", "srswa_route",
-           "srswa_decode", "workspace_bytes", "new_workspace", "check_status", "dims_of"]
+           "srswa_decode", "workspace_bytes", "new_workspace", "route_workspace", "check_status", "dims_of"]

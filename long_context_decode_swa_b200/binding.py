@@ -144,6 +144,11 @@ def new_workspace(dims: Dims, op: int, device=None) -> torch.Tensor:
     return torch.zeros(workspace_bytes(dims, op), dtype=torch.uint8, device=device or "cuda")
 
 
+def route_workspace(batch: int, prefix_cap: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace for srswa_route over `batch` sequences of capacity `prefix_cap`."""
+    return new_workspace(Dims(batch, 1, 128, 1, prefix_cap), OP_ROUTE, device)
+
+
 def check_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise, read and clear the device status word; returns it (0 = clean)."""
     st = ctypes.c_int32(0)

@@ -85,11 +85,20 @@ size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
       return rswa::plan_decode_workspace(dims->batch, dims->heads, rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring),
                                          rswa::device_sm_count())
           .bytes;
-    case RSWA_OP_SRSWA_DECODE:
-      return rswa::plan_decode_workspace(dims->batch, dims->heads, rswa::decode_max_tiles_sparse(rswa::kMaxTopk, dims->ring),
-                                         rswa::device_sm_count())
-          .bytes;
+    case RSWA_OP_SRSWA_DECODE: {
+      // the plan depends on topk: size for the largest plan over every allowed topk
+      size_t most = 0;
+      for (int k = 1; k <= rswa::kMaxTopk; ++k) {
+        const size_t b = rswa::plan_decode_workspace(dims->batch, dims->heads,
+                                                     rswa::decode_max_tiles_sparse(k, dims->ring),
+                                                     rswa::device_sm_count())
+                             .bytes;
+        most = b > most ? b : most;
+      }
+      return most;
+    }
     case RSWA_OP_ROUTE:
+      return rswa::plan_route_workspace(dims->batch, dims->prefix_cap).bytes;
     case RSWA_OP_PREFILL:
       return 256;
     default:
@@ -134,11 +143,12 @@ rswa_status rswa_append(const rswa_dims* dims, void* ring_k, void* ring_v, const
   return ok();
 }
 
+// plan_budget > 0: plan the split-KV work to fit a workspace of that many bytes.
 static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, const void* pk,
                                  const void* pv, const int32_t* prefix_len, const int32_t* blk_idx,
                                  const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                                  const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
-                                 void* workspace, size_t ws_bytes, void* stream) {
+                                 void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0) {
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q);
@@ -156,10 +166,10 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
     if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
   }
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
-  const int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(rswa::kMaxTopk, dims->ring)
+  const int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(topk, dims->ring)
                                    : rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring);
   const rswa::WorkspacePlan plan =
-      rswa::plan_decode_workspace(dims->batch, dims->heads, max_tiles, rswa::device_sm_count());
+      rswa::plan_decode_workspace(dims->batch, dims->heads, max_tiles, rswa::device_sm_count(), plan_budget);
   if (ws_bytes < plan.bytes)
     return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes,
                 plan.bytes);
@@ -169,6 +179,9 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.n = dims->ring;
   a.cap = dims->prefix_cap;
   a.splits = plan.splits;
+  a.tiles_per_item = plan.tiles_per_item;
+  if (plan.items > INT32_MAX) return fail(RSWA_ERR_UNSUPPORTED, "%s: too many work items", fn);
+  a.items = (int)plan.items;
   a.q = static_cast<const uint16_t*>(q);
   a.pk = static_cast<const uint16_t*>(pk);
   a.pv = static_cast<const uint16_t*>(pv);
@@ -187,7 +200,7 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.blk_idx = blk_idx;
   a.blk_logp = blk_logp;
   a.topk = sparse ? topk : 0;
-  cudaError_t e = rswa::launch_decode(a, sparse, static_cast<cudaStream_t>(stream));
+  cudaError_t e = rswa::launch_decode(a, plan.grid, sparse, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
 }
@@ -300,14 +313,16 @@ rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* 
     return fail(RSWA_ERR_INVALID, "%s: prefix_len, blk_idx and blk_logp must not be NULL", fn);
   if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
   if (!std::isfinite(idx_scale)) return fail(RSWA_ERR_INVALID, "%s: idx_scale must be finite", fn);
-  if (ws_bytes < 256) return fail(RSWA_ERR_INVALID, "%s: workspace must be at least 256 bytes", fn);
   const int64_t nb_cap = (dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock;
   if (nb_cap > rswa::kMaxRouteBlocks)
     return fail(RSWA_ERR_UNSUPPORTED, "%s: %lld prefix blocks exceed the router's limit of %d", fn,
                 (long long)nb_cap, rswa::kMaxRouteBlocks);
   if (nb_cap == 0) return fail(RSWA_ERR_INVALID, "%s: prefix_cap must be >= 1", fn);
+  const size_t need = rswa::plan_route_workspace(dims->batch, dims->prefix_cap).bytes;
+  if (ws_bytes < need)
+    return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes, need);
   cudaError_t e = rswa::launch_route(dims->batch, dims->prefix_cap, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx,
-                                     blk_logp, probs, tau, ws_status(workspace), static_cast<cudaStream_t>(stream));
+                                     blk_logp, probs, tau, workspace, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
 }
@@ -369,8 +384,9 @@ rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void
   if (prefix_len == nullptr || wp == nullptr || fill == nullptr)
     return fail(RSWA_ERR_INVALID, "%s: prefix_len, wp and fill must not be NULL", fn);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
-  const rswa::WorkspacePlan plan = rswa::plan_decode_workspace(
-      dims->batch, dims->heads, rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring), rswa::device_sm_count());
+  const rswa::WorkspacePlan plan =
+      rswa::plan_decode_workspace(dims->batch, dims->heads, rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring),
+                                  rswa::device_sm_count(), kNoAllocScratchBytes);
   if (plan.bytes > kNoAllocScratchBytes)
     return fail(RSWA_ERR_UNSUPPORTED,
                 "%s: these dims need %zu bytes of scratch, above the %zu-byte static scratch; use rswa_decode "
@@ -385,7 +401,7 @@ rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void
   cudaError_t e = cudaMemsetAsync(scratch, 0, plan.partials_off, s);
   if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: clearing the scratch counters");
   st = decode_common(fn, false, dims, q, pk, pv, prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp, fill, scale,
-                     out, lse, scratch, kNoAllocScratchBytes, stream);
+                     out, lse, scratch, kNoAllocScratchBytes, stream, kNoAllocScratchBytes);
   if (st != RSWA_OK) return st;
   if (status != nullptr) {
     e = cudaMemcpyAsync(status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);

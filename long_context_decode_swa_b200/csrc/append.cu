@@ -4,8 +4,8 @@
 // head, the pointer advances cyclically and the valid count saturates at n
 // (Unlimited-OCR-2 SR-SWA explainer, 环形缓冲; "百度 Unlimited OCR 深度实战"
 // tutorial §3.3.2). One CTA per sequence copies its H x 256 B of K and of V
-// with 16-byte loads/stores; thread 0 alone reads and advances wp/fill, after
-// a CTA barrier, so no other thread of the launch touches them.
+// with 16-byte loads/stores; thread 0 alone reads and advances wp/fill, so no
+// other thread of the launch touches them.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(int H, int n, ui
                                                                 int32_t* fill, int32_t* slot_out, int32_t* status) {
   __shared__ int s_slot;
   const int b = blockIdx.x;
+  griddep_wait();  // the previous kernel may still be reading the slot this one overwrites
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     const int w = wp[b], f = fill[b];
     const bool ok = w >= 0 && w < n && f >= 0 && f <= n;
@@ -54,8 +56,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(int H, int n, ui
 cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_v, const uint16_t* k_new,
                           const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status,
                           cudaStream_t stream) {
-  append_kernel<<<B, kAppendThreads, 0, stream>>>(H, n, ring_k, ring_v, k_new, v_new, wp, fill, slot_out, status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  fill_launch_config(cfg, attr, dim3(B), dim3(kAppendThreads), 0, stream);
+  return cudaLaunchKernelEx(&cfg, append_kernel, H, n, ring_k, ring_v, k_new, v_new, wp, fill, slot_out, status);
 }
 
 }  // namespace rswa

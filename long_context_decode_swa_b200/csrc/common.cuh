@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_runtime.h>
 
 #include "rswa.h"
@@ -122,6 +123,36 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ void set_status(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
+}
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start while the previous kernel in the
+// stream is still running. griddep_wait() blocks until that kernel has
+// completed and its writes are visible (it returns at once for a normal
+// launch), so every kernel here calls it before touching memory;
+// griddep_launch_dependents() lets the next kernel begin its prologue.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+inline bool pdl_enabled() {
+  static const int on = [] {
+    const char* e = getenv("RSWA_PDL");
+    return (e != nullptr && e[0] == '0') ? 0 : 1;
+  }();
+  return on != 0;
+}
+
+// Launch configuration with programmatic dependent launch (unless RSWA_PDL=0).
+inline void fill_launch_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, dim3 grid, dim3 block,
+                               size_t smem, cudaStream_t stream) {
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
 }
 
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device) so

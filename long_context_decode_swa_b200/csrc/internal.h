@@ -20,6 +20,8 @@ struct DecodeArgs {
   const int32_t* wp;
   const int32_t* fill;
   float qscale;  // softmax scale * log2(e)
+  int tiles_per_item;  // P: tiles of one (sequence, head, split) item (padded with empty tiles)
+  int items;           // B * H * splits
   float* out;
   float* lse;
   float* partials;   // [B*H][splits][D + 2]
@@ -33,11 +35,13 @@ struct DecodeArgs {
 
 // Workspace layout shared by every op: [status: 256 B][counters][partials].
 struct WorkspacePlan {
-  int splits;
+  int splits, tiles_per_item, grid;
+  int64_t items;
   size_t counters_off, partials_off, bytes;
 };
 
-WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_count);
+// max_bytes > 0 restricts the split count to plans whose workspace fits that many bytes.
+WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_count, size_t max_bytes = 0);
 int64_t decode_max_tiles_dense(int64_t cap, int n);
 int64_t decode_max_tiles_sparse(int topk, int n);
 int device_sm_count();
@@ -45,12 +49,19 @@ int device_sm_count();
 cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_v, const uint16_t* k_new,
                           const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status,
                           cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, bool sparse, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream);
 cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const int32_t* prefix_len, float* kbar,
                               cudaStream_t stream);
+// Router workspace: [status: 256 B][counters: int32 per sequence][chunk maxima]
+// [chunk top-32 lists: (z, block) pairs][block scores z: f32 per block].
+struct RouteWorkspace {
+  int nb_cap, chunks_cap;
+  size_t counters_off, cmax_off, cand_off, zbuf_off, bytes;
+};
+RouteWorkspace plan_route_workspace(int B, int64_t cap);
 cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
                          float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                         int32_t* status, cudaStream_t stream);
+                         void* workspace, cudaStream_t stream);
 
 struct PrefillLaunch {
   int B, H, n, T;

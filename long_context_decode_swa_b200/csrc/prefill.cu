@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int64_t bh = (int64_t)b * a.H + h;
 
   __shared__ int s_skip;
+  griddep_wait();
+  griddep_launch_dependents();
   if (tid == 0) {
     // a CTA of this launch already gave up on a wait: skip the work (the output is flagged invalid)
     s_skip = a.status != nullptr && (*reinterpret_cast<volatile int32_t*>(a.status) & RSWA_DEVICE_WAIT_TIMEOUT);
@@ -540,6 +542,7 @@ __global__ void ring_from_outputs_kernel(int H, int n, int T, const uint16_t* __
                                          uint16_t* __restrict__ ring_v, int32_t* wp, int32_t* fill, int32_t* status) {
   __shared__ int s_wp;
   const int b = blockIdx.x;
+  griddep_wait();
   if (threadIdx.x == 0) {
     const int w = wp[b], f = fill[b];
     const bool ok = w >= 0 && w < n && f >= 0 && f <= n;
@@ -638,8 +641,10 @@ cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t stream) {
   static unsigned long long done = 0;
   if ((e = ensure_smem_limit(prefill_kernel, smem, &done)) != cudaSuccess) return e;
   const dim3 grid((L.T + kTileRows - 1) / kTileRows, L.H, L.B);
-  prefill_kernel<<<grid, kPrefillThreads, smem, stream>>>(a, tq, tko, tvo, tpk, tpv, trk, trv);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  fill_launch_config(cfg, attr, grid, dim3(kPrefillThreads), smem, stream);
+  if ((e = cudaLaunchKernelEx(&cfg, prefill_kernel, a, tq, tko, tvo, tpk, tpv, trk, trv)) != cudaSuccess) return e;
   if (L.write_ring) {
     ring_from_outputs_kernel<<<L.B, 256, 0, stream>>>(L.H, L.n, L.T, static_cast<const uint16_t*>(L.k_out),
                                                       static_cast<const uint16_t*>(L.v_out),

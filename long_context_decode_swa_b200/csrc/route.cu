@@ -30,7 +30,6 @@ namespace {
 constexpr int kPoolWarps = 8;
 constexpr int kRouteThreads = 512;
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kScoreUnroll = 8;
 
 // Index keys: one warp per 32-token block; lane (tg, dq) sums tokens tg, tg+8, ...
 // over dims 8dq..8dq+7, then the eight token groups are folded with shuffles.
@@ -40,6 +39,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32) index_pool_kernel(int64_t cap
                                                                      float* __restrict__ kbar) {
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();
   const int c = blockIdx.x * kPoolWarps + warp;
   if (c >= nb_cap) return;
   int64_t m = prefix_len[b];
@@ -80,123 +80,202 @@ __device__ __forceinline__ bool ranks_before(float za, int ia, float zb, int ib)
   return za > zb || (za == zb && ia < ib);
 }
 
-__device__ __forceinline__ void warp_best(float& z, int& i) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float oz = __shfl_xor_sync(0xffffffffu, z, off);
-    const int oi = __shfl_xor_sync(0xffffffffu, i, off);
-    if (ranks_before(oz, oi, z, i)) {
-      z = oz;
-      i = oi;
-    }
+constexpr int kNone = 0x7fffffff;
+constexpr int kList = 32;  // sorted candidates kept per warp / per chunk (>= the largest topk)
+
+// Compare-exchange with the lane `j` apart: the lane whose bit j equals `keep_better_bit`
+// keeps the better of the pair, its partner the worse.
+__device__ __forceinline__ void cmp_xchg(float& z, int& i, int j, bool keep_better) {
+  const float oz = __shfl_xor_sync(0xffffffffu, z, j);
+  const int oi = __shfl_xor_sync(0xffffffffu, i, j);
+  const bool other_better = ranks_before(oz, oi, z, i);
+  if (other_better == keep_better) {
+    z = oz;
+    i = oi;
   }
 }
 
-constexpr int kNone = 0x7fffffff;
+// Bitonic sort of one (z, i) pair per lane; afterwards lane 0 holds the best.
+__device__ __forceinline__ void warp_sort(float& z, int& i, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) cmp_xchg(z, i, j, ((lane & j) == 0) == ((lane & k) == 0));
+}
 
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(int64_t cap, int nb_cap, const float* __restrict__ q_idx,
-                                                              const float* __restrict__ kbar,
-                                                              const int32_t* __restrict__ prefix_len, float idx_scale,
-                                                              int topk, int32_t* __restrict__ blk_idx,
-                                                              float* __restrict__ blk_logp, float* __restrict__ probs,
-                                                              float* __restrict__ tau_out, int32_t* status) {
+// Top 32 of two sorted lists: lane l holds A[l] and B[31 - l] (a bitonic pair); keep the
+// better, then merge the resulting bitonic sequence across the warp.
+__device__ __forceinline__ void warp_merge(float& z, int& i, float bz, int bi, int lane) {
+  if (ranks_before(bz, bi, z, i)) {
+    z = bz;
+    i = bi;
+  }
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) cmp_xchg(z, i, j, (lane & j) == 0);
+}
+
+struct RouteArgs {
+  int64_t cap;
+  int nb_cap, chunks_cap, topk;
+  float idx_scale;
+  const float* q_idx;
+  const float* kbar;
+  const int32_t* prefix_len;
+  int32_t* blk_idx;
+  float* blk_logp;
+  float* probs;
+  float* tau;
+  int32_t* status;
+  int32_t* counters;  // [B]
+  float* cmax;        // [B][chunks_cap]
+  float2* cand;       // [B][chunks_cap][kList]: (z, block index as int bits)
+  float* zbuf;        // [B][nb_cap]
+};
+
+// Merges `n` sorted lists of kList held in (lz, li) shared arrays into lists[0]; every
+// warp of the CTA must call it (it synchronises the CTA).
+__device__ void merge_lists(float (*lz)[kList], int (*li)[kList], int n, int warp, int lane) {
+  for (int width = 1; width < n; width <<= 1) {
+    const int pairs = (n + 2 * width - 1) / (2 * width);
+    if (warp < pairs) {
+      const int a = 2 * width * warp, bidx = a + width;
+      float z = lz[a][lane];
+      int i = li[a][lane];
+      float bz = -INFINITY;
+      int bi = kNone;
+      if (bidx < n) {
+        bz = lz[bidx][kList - 1 - lane];
+        bi = li[bidx][kList - 1 - lane];
+      }
+      __syncwarp();
+      warp_merge(z, i, bz, bi, lane);
+      lz[a][lane] = z;
+      li[a][lane] = i;
+    }
+    __syncthreads();
+  }
+}
+
+// One CTA scores kRouteThreads blocks of one sequence (grid = chunks x B), keeps their
+// sorted top-kList, and the last CTA of the sequence merges the chunk lists and solves
+// the 1.5-entmax threshold exactly.
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  float* z = reinterpret_cast<float*>(smem_raw);  // [nb_cap] block scores
-  float* cy = z + nb_cap;                         // [nb_cap] candidates: y = z/2 - max(z/2)
-  int* ci = reinterpret_cast<int*>(cy + nb_cap);  // [nb_cap] candidates: block index
-  float* sy = reinterpret_cast<float*>(ci + nb_cap);  // [nb_cap] candidates sorted by rank
+  __shared__ float lz[kRouteWarps][kList];
+  __shared__ int li[kRouteWarps][kList];
   __shared__ float red[kRouteWarps];
-  __shared__ float s_xmax;
-  __shared__ int s_count;
+  __shared__ int s_last, s_count;
   __shared__ unsigned long long s_best;  // (support size << 32) | bits(tau_y)
-  __shared__ float wz[kRouteWarps][kMaxTopk];
-  __shared__ int wi[kRouteWarps][kMaxTopk];
 
-  const int b = blockIdx.x;
+  const int chunk = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int64_t m64 = prefix_len[b];
-  if (m64 < 0 || m64 > cap) {
-    if (tid == 0) set_status(status, RSWA_DEVICE_BAD_PREFIX_LEN);
+  griddep_wait();
+  griddep_launch_dependents();
+  int64_t m64 = a.prefix_len[b];
+  if (m64 < 0 || m64 > a.cap) {
+    if (tid == 0 && chunk == 0) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
     m64 = 0;
   }
   const int NB = (int)((m64 + kBlock - 1) / kBlock);
+  const int chunks = (NB + kRouteThreads - 1) / kRouteThreads;
   if (NB == 0) {
-    if (tid < topk) {
-      blk_idx[(int64_t)b * topk + tid] = -1;
-      blk_logp[(int64_t)b * topk + tid] = -INFINITY;
+    if (chunk == 0) {
+      if (tid < a.topk) {
+        a.blk_idx[(int64_t)b * a.topk + tid] = -1;
+        a.blk_logp[(int64_t)b * a.topk + tid] = -INFINITY;
+      }
+      if (a.probs)
+        for (int c = tid; c < a.nb_cap; c += kRouteThreads) a.probs[(int64_t)b * a.nb_cap + c] = 0.f;
+      if (a.tau && tid == 0) a.tau[b] = NAN;
     }
-    if (probs)
-      for (int c = tid; c < nb_cap; c += kRouteThreads) probs[(int64_t)b * nb_cap + c] = 0.f;
-    if (tau_out && tid == 0) tau_out[b] = NAN;
     return;
   }
+  if (chunk >= chunks) return;
 
-  // ---- 1. block scores z_c = idx_scale * <q_idx, kbar_c>: 8 lanes per block ----
-  const int sub = lane >> 3, dq = lane & 7;
-  const float4 q4 = reinterpret_cast<const float4*>(q_idx + (int64_t)b * kIndexDim)[dq];
-  const float* kb = kbar + (int64_t)b * nb_cap * kIndexDim;
-  float lmax = -INFINITY;
-  for (int c0 = warp * 4 * kScoreUnroll; c0 < NB; c0 += kRouteWarps * 4 * kScoreUnroll) {
-    float4 k4[kScoreUnroll];
+  // ---- score one block per thread ----
+  const int c = chunk * kRouteThreads + tid;
+  float z = -INFINITY;
+  int ci = kNone;
+  if (c < NB) {
+    const float4* q4 = reinterpret_cast<const float4*>(a.q_idx + (int64_t)b * kIndexDim);
+    const float4* k4 = reinterpret_cast<const float4*>(a.kbar + ((int64_t)b * a.nb_cap + c) * kIndexDim);
+    float4 kv[8];
 #pragma unroll
-    for (int u = 0; u < kScoreUnroll; ++u) {
-      const int c = c0 + u * 4 + sub;
-      k4[u] = c < NB ? reinterpret_cast<const float4*>(kb + (int64_t)c * kIndexDim)[dq]
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int u = 0; u < 8; ++u) kv[u] = k4[u];
+    float d = 0.f;
 #pragma unroll
-    for (int u = 0; u < kScoreUnroll; ++u) {
-      const int c = c0 + u * 4 + sub;
-      float d = q4.x * k4[u].x;
-      d = fmaf(q4.y, k4[u].y, d);
-      d = fmaf(q4.z, k4[u].z, d);
-      d = fmaf(q4.w, k4[u].w, d);
-      d += __shfl_xor_sync(0xffffffffu, d, 1);
-      d += __shfl_xor_sync(0xffffffffu, d, 2);
-      d += __shfl_xor_sync(0xffffffffu, d, 4);
-      if (c < NB) {
-        const float zc = idx_scale * d;
-        if (dq == 0) z[c] = zc;
-        lmax = fmaxf(lmax, zc);
-      }
+    for (int u = 0; u < 8; ++u) {
+      const float4 qv = q4[u];
+      d = fmaf(qv.x, kv[u].x, d);
+      d = fmaf(qv.y, kv[u].y, d);
+      d = fmaf(qv.z, kv[u].z, d);
+      d = fmaf(qv.w, kv[u].w, d);
     }
+    z = a.idx_scale * d;
+    ci = c;
+    a.zbuf[(int64_t)b * a.nb_cap + c] = z;
   }
-  lmax = warp_max(lmax);
-  if (lane == 0) red[warp] = lmax;
+  const float wmax = warp_max(z);
+  if (lane == 0) red[warp] = wmax;
+  warp_sort(z, ci, lane);
+  lz[warp][lane] = z;
+  li[warp][lane] = ci;
   __syncthreads();
+  merge_lists(lz, li, kRouteWarps, warp, lane);
+  float2* my_list = a.cand + ((int64_t)b * a.chunks_cap + chunk) * kList;
+  if (warp == 0) my_list[lane] = make_float2(lz[0][lane], __int_as_float(li[0][lane]));
   if (tid == 0) {
     float mx = red[0];
     for (int w = 1; w < kRouteWarps; ++w) mx = fmaxf(mx, red[w]);
-    s_xmax = 0.5f * mx;
+    a.cmax[(int64_t)b * a.chunks_cap + chunk] = mx;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&a.counters[b], 1) == chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // ---- last CTA of the sequence: merge the chunk lists ----
+  if (warp < chunks) {
+    const float2 e = __ldcg(a.cand + ((int64_t)b * a.chunks_cap + warp) * kList + lane);
+    lz[warp][lane] = e.x;
+    li[warp][lane] = __float_as_int(e.y);
+  }
+  if (tid == 0) {
+    float mx = -INFINITY;
+    for (int k = 0; k < chunks; ++k) mx = fmaxf(mx, __ldcg(a.cmax + (int64_t)b * a.chunks_cap + k));
+    red[0] = 0.5f * mx;
     s_count = 0;
     s_best = 0ull;
   }
   __syncthreads();
-  const float xmax = s_xmax;
+  merge_lists(lz, li, chunks, warp, lane);
+  const float xmax = red[0];
 
-  // ---- 2. gather the candidates x_c > max x - 1 ----
-  for (int c = tid; c < NB; c += kRouteThreads) {
-    const float y = fmaf(z[c], 0.5f, -xmax);
+  // ---- 1.5-entmax over all NB blocks: candidates x > max x - 1, ranked, prefix sums ----
+  float* cy = reinterpret_cast<float*>(smem_raw);  // [NB] shifted candidates y = x - max x
+  int* cix = reinterpret_cast<int*>(cy + a.nb_cap);
+  float* sy = reinterpret_cast<float*>(cix + a.nb_cap);
+  const float* zb = a.zbuf + (int64_t)b * a.nb_cap;
+  for (int k = tid; k < NB; k += kRouteThreads) {
+    const float y = fmaf(__ldcg(zb + k), 0.5f, -xmax);
     if (y > -1.f) {
-      const int k = atomicAdd(&s_count, 1);
-      cy[k] = y;
-      ci[k] = c;
+      const int slot = atomicAdd(&s_count, 1);
+      cy[slot] = y;
+      cix[slot] = k;
     }
   }
   __syncthreads();
   const int K = s_count;
-
-  // ---- 3. rank the candidates (descending y, ties to the smaller block) ----
   for (int i = tid; i < K; i += kRouteThreads) {
     const float yi = cy[i];
-    const int ii = ci[i];
+    const int ii = cix[i];
     int r = 0;
-    for (int j = 0; j < K; ++j) r += ranks_before(cy[j], ci[j], yi, ii) ? 1 : 0;
+    for (int j = 0; j < K; ++j) r += ranks_before(cy[j], cix[j], yi, ii) ? 1 : 0;
     sy[r] = yi;
   }
   __syncthreads();
-
-  // ---- 4. sort-based threshold: prefix sums in rank order ----
   for (int r = tid; r < K; r += kRouteThreads) {
     float s1 = 0.f, s2 = 0.f;
     for (int j = 0; j <= r; ++j) {
@@ -215,75 +294,31 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int64_t cap, int n
   }
   __syncthreads();
   const float tau_y = __uint_as_float((unsigned)(s_best & 0xffffffffull));
-  if (tau_out && tid == 0) tau_out[b] = tau_y + xmax;
-  if (probs) {
-    for (int c = tid; c < nb_cap; c += kRouteThreads) {
-      float p = 0.f;
-      if (c < NB) {
-        const float r = fmaf(z[c], 0.5f, -xmax) - tau_y;
-        p = r > 0.f ? r * r : 0.f;
+  if (a.tau && tid == 0) a.tau[b] = tau_y + xmax;
+  if (a.probs) {
+    for (int k = tid; k < a.nb_cap; k += kRouteThreads) {
+      float pr = 0.f;
+      if (k < NB) {
+        const float r = fmaf(__ldcg(zb + k), 0.5f, -xmax) - tau_y;
+        pr = r > 0.f ? r * r : 0.f;
       }
-      probs[(int64_t)b * nb_cap + c] = p;
+      a.probs[(int64_t)b * a.nb_cap + k] = pr;
     }
   }
-
-  // ---- 5. top-k: each warp selects from its slice, warp 0 merges ----
-  {
-    const int chunk = (NB + kRouteWarps - 1) / kRouteWarps;
-    const int lo = warp * chunk, hi = min(NB, lo + chunk);
-    float pz = INFINITY;
-    int pi = -1;
-    for (int r = 0; r < topk; ++r) {
-      float bz = -INFINITY;
-      int bi = kNone;
-      for (int c = lo + lane; c < hi; c += 32) {
-        const float zc = z[c];
-        if (ranks_before(pz, pi, zc, c) && ranks_before(zc, c, bz, bi)) {
-          bz = zc;
-          bi = c;
-        }
-      }
-      warp_best(bz, bi);
-      if (lane == 0) {
-        wz[warp][r] = bz;
-        wi[warp][r] = bi;
-      }
-      pz = bz;
-      pi = bi;
+  if (warp == 0 && lane < a.topk) {
+    const int64_t o = (int64_t)b * a.topk + lane;
+    const int bi = li[0][lane];
+    if (bi == kNone) {
+      a.blk_idx[o] = -1;
+      a.blk_logp[o] = -INFINITY;
+    } else {
+      const float d = fmaf(lz[0][lane], 0.5f, -xmax) - tau_y;
+      const float pr = d > 0.f ? d * d : 0.f;
+      a.blk_idx[o] = bi;
+      a.blk_logp[o] = pr > 0.f ? logf(pr) : -INFINITY;
     }
   }
-  __syncthreads();
-  if (warp == 0) {
-    float pz = INFINITY;
-    int pi = -1;
-    for (int r = 0; r < topk; ++r) {
-      float bz = -INFINITY;
-      int bi = kNone;
-      for (int e = lane; e < kRouteWarps * topk; e += 32) {
-        const float zc = wz[e / topk][e % topk];
-        const int c = wi[e / topk][e % topk];
-        if (c != kNone && ranks_before(pz, pi, zc, c) && ranks_before(zc, c, bz, bi)) {
-          bz = zc;
-          bi = c;
-        }
-      }
-      warp_best(bz, bi);
-      if (lane == 0) {
-        const int64_t o = (int64_t)b * topk + r;
-        if (bi == kNone) {
-          blk_idx[o] = -1;
-          blk_logp[o] = -INFINITY;
-        } else {
-          const float d = fmaf(z[bi], 0.5f, -xmax) - tau_y;
-          const float p = d > 0.f ? d * d : 0.f;
-          blk_idx[o] = bi;
-          blk_logp[o] = p > 0.f ? logf(p) : -INFINITY;
-        }
-      }
-      pz = bz;
-      pi = bi;
-    }
-  }
+  if (tid == 0) a.counters[b] = 0;
 }
 
 }  // namespace
@@ -296,18 +331,54 @@ cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const i
   return cudaGetLastError();
 }
 
+RouteWorkspace plan_route_workspace(int B, int64_t cap) {
+  RouteWorkspace w;
+  w.nb_cap = (int)((cap + kBlock - 1) / kBlock);
+  w.chunks_cap = (w.nb_cap + kRouteThreads - 1) / kRouteThreads;
+  size_t off = 256;  // status word
+  w.counters_off = off;
+  off += ((size_t)B * 4 + 255) / 256 * 256;
+  w.cmax_off = off;
+  off += ((size_t)B * w.chunks_cap * 4 + 255) / 256 * 256;
+  w.cand_off = off;
+  off += (size_t)B * w.chunks_cap * kList * 8;
+  w.zbuf_off = off;
+  off += (size_t)B * w.nb_cap * 4;
+  w.bytes = off;
+  return w;
+}
+
 cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
                          float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                         int32_t* status, cudaStream_t stream) {
-  const int nb_cap = (int)((cap + kBlock - 1) / kBlock);
-  const size_t smem = (size_t)nb_cap * 16;
+                         void* workspace, cudaStream_t stream) {
+  const RouteWorkspace w = plan_route_workspace(B, cap);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  RouteArgs a;
+  a.cap = cap;
+  a.nb_cap = w.nb_cap;
+  a.chunks_cap = w.chunks_cap;
+  a.topk = topk;
+  a.idx_scale = idx_scale;
+  a.q_idx = q_idx;
+  a.kbar = kbar;
+  a.prefix_len = prefix_len;
+  a.blk_idx = blk_idx;
+  a.blk_logp = blk_logp;
+  a.probs = probs;
+  a.tau = tau;
+  a.status = reinterpret_cast<int32_t*>(ws);
+  a.counters = reinterpret_cast<int32_t*>(ws + w.counters_off);
+  a.cmax = reinterpret_cast<float*>(ws + w.cmax_off);
+  a.cand = reinterpret_cast<float2*>(ws + w.cand_off);
+  a.zbuf = reinterpret_cast<float*>(ws + w.zbuf_off);
+  const size_t smem = (size_t)w.nb_cap * 12;
   static unsigned long long done = 0;
-  // one-time raise to the largest size the router supports
-  cudaError_t e = ensure_smem_limit(route_kernel, (size_t)kMaxRouteBlocks * 16, &done);
+  cudaError_t e = ensure_smem_limit(route_kernel, (size_t)kMaxRouteBlocks * 12, &done);
   if (e != cudaSuccess) return e;
-  route_kernel<<<B, kRouteThreads, smem, stream>>>(cap, nb_cap, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx,
-                                                   blk_logp, probs, tau, status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  fill_launch_config(cfg, attr, dim3(w.chunks_cap, B), dim3(kRouteThreads), smem, stream);
+  return cudaLaunchKernelEx(&cfg, route_kernel, a);
 }
 
 }  // namespace rswa

@@ -25,8 +25,9 @@ def _route_gpu(rswa, q_idx, kbar, plen_t, cap, topk=16):
     logp = torch.empty((B, topk), dtype=torch.float32, device="cuda")
     probs = torch.empty((B, nb_cap), dtype=torch.float32, device="cuda")
     tau = torch.empty((B,), dtype=torch.float32, device="cuda")
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = rswa.route_workspace(B, cap)
     rswa.srswa_route(q_idx, kbar, plen_t, blk, logp, ws, probs=probs, tau=tau, prefix_cap=cap)
+    rswa.srswa_route(q_idx, kbar, plen_t, blk, logp, ws, probs=probs, tau=tau, prefix_cap=cap)  # reuse: counters reset
     assert rswa.check_status(ws) == 0
     return to_np(blk), to_np(logp), to_np(probs), to_np(tau)
 
@@ -144,7 +145,7 @@ def _chain(rswa, plen, cap, B, steps, sample, seed):
     rswa.srswa_index_pool(pl.k_idx, plen_t, kbar)
     blk = torch.empty((B, 16), dtype=torch.int32, device="cuda")
     logp = torch.empty((B, 16), dtype=torch.float32, device="cuda")
-    ws_r = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws_r = rswa.route_workspace(B, cap)
     r = DecodeRunner(rswa, c, sample)
     for s in range(steps):
         rswa.srswa_route(pl.q_idx[s], kbar, plen_t, blk, logp, ws_r, prefix_cap=cap)

@@ -5,8 +5,9 @@ that only receive raw pointers from an engine that owns every allocation).
 rswa_decode_noalloc takes its split-KV scratch from static device memory in
 the library instead of a caller workspace. These tests call it through the C
 ABI and check it against rswa_decode (same tolerance as the other decode
-parity tests) on two calls in a row, once with several split-KV partials per
-(sequence, head) and once with one split. The file is named to be collected
+parity tests) on two calls in a row: with several split-KV partials per
+(sequence, head), with a split count capped by the scratch size, and with one
+split. The file is named to be collected
 last; it passes alone in a fresh process and after the other tests.
 """
 import ctypes
@@ -38,7 +39,8 @@ def _noalloc(lib, c, ring_k, ring_v, wp, fill, out, lse, status):
 @pytest.mark.gpu
 @pytest.mark.parametrize("B,H,plen,cap", [
     (2, 16, [1000, 613], 1000),     # few (sequence, head) pairs: many split-KV partials in the scratch
-    (112, 16, [700] * 112, 700),    # enough pairs for one split: counters only
+    (112, 16, [700] * 112, 700),    # the scratch budget caps the split count below rswa_decode's choice
+    (512, 16, [700] * 512, 700),    # enough pairs for one split: counters only
 ])
 def test_noalloc_matches_rswa_decode_twice(cuda_lib, B, H, plen, cap):
     rswa = cuda_lib
@@ -68,7 +70,7 @@ def test_noalloc_matches_rswa_decode_twice(cuda_lib, B, H, plen, cap):
 @pytest.mark.gpu
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_lib):
     lib = cuda_lib.load()
-    # 65535 x 128 (sequence, head) completion counters alone need 32 MiB > 4 MiB
+    # 65535 x 128 (sequence, head) completion counters alone need 32 MiB > 4 MiB, even with one split
     dims = Dims(65535, 128, 128, 128, 64)
     x = torch.zeros(16, dtype=torch.uint8, device="cuda")
     p = _p(x)
