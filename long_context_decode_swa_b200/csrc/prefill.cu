@@ -8,25 +8,30 @@
 // r <= fill).
 //
 // This is the path's one dense contraction, so it runs on the 5th-generation
-// tensor cores. One CTA owns 128 query rows of one (sequence, head):
-//   warp 0, lane 0 : TMA producer of Q and of the K tiles (128 keys x 128 dims)
-//   warp 2, lane 0 : TMA producer of the V tiles
-//   warp 1         : allocates TMEM; lane 0 issues tcgen05.mma (S = Q K^T into
-//                    one of two TMEM S buffers, O += P V into the TMEM O
-//                    accumulator) and tcgen05.commit; the warp zeroes V rows of
-//                    keys that no query may see (so 0 * garbage never reaches O)
-//   warps 4-7      : softmax; thread r owns query row r = TMEM lane r. It loads
-//                    its S row (tcgen05.ld), masks, keeps the running max and sum
-//                    in the exp2 domain, writes its bf16 P row into a 128B-
-//                    swizzled shared-memory tile (the MMA's A operand), and at
-//                    the end normalises its O row and stores it.
-// The running max is only moved when it grows by more than 2^8 (log2 units);
-// the exponentials are then bounded by 256 and the final O / l is the same
-// quotient, so this lazy rescale is exact, and the O read-modify-write through
-// TMEM happens only on those rare steps.
-// Operands: Q, K in K-major SW128 layout (TMA SWIZZLE_128B, boxes of 64 dims x
-// 128 rows); V as the MN-major B operand of O += P V (dims contiguous); P
-// K-major SW128 written by the softmax threads with the same XOR swizzle.
+// tensor cores. One CTA owns two 128-row query tiles (A and B) of one
+// (sequence, head) and walks the key tiles (128 keys each) both need:
+//   warp 0, lane 0  : TMA producer of Q (both tiles) and of the K tiles (3 stages)
+//   warp 2, lane 0  : TMA producer of the V tiles (2 stages)
+//   warp 1          : allocates TMEM; lane 0 issues tcgen05.mma; the warp zeroes
+//                     the V rows of keys no query may see (their P is 0, their
+//                     bytes may be anything, and 0 * NaN would reach O)
+//   warps 4-7 / 8-11: softmax of tile A / tile B; thread r owns query row r, i.e.
+//                     TMEM lane r of its tile's S, P and O.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// P (bf16, two per 32-bit column) is written over the first 64 columns of its
+// tile's S once those scores have been read, and the P.V product takes its A
+// operand straight from TMEM. The MMA thread issues, per key tile t,
+//   PV_A(t), S_A(t+1), PV_B(t), S_B(t+1)
+// so while one tile's softmax runs the tensor core works on the other tile.
+// Tensor-core operations of one thread execute in issue order, so S_A(t+1) may
+// overwrite P_A(t) right after PV_A(t) is issued, and a softmax that sees S_X(t)
+// complete also knows PV_X(t-1) has completed (the commit covers every earlier
+// operation): the O rescale it may then do needs no further wait.
+// The running max only moves when it grows by more than 2^8 (log2 units); the
+// exponentials stay below 256 and the final O / l is the same quotient, so this
+// lazy rescale is exact and the O read-modify-write through TMEM is rare.
+// (query tile, key tile) pairs in which every score is masked are skipped by the
+// MMA thread and the softmax alike.
 // Every mbarrier wait is bounded; on expiry the kernel flags
 // RSWA_DEVICE_WAIT_TIMEOUT, drains what it issued and frees its TMEM.
 #include <cuda.h>
@@ -41,32 +46,34 @@ namespace rswa {
 
 namespace {
 
-constexpr int kTileRows = 128;                 // query rows per CTA, keys per KV tile
+constexpr int kTileRows = 128;                 // query rows per tile, keys per key tile
+constexpr int kQTiles = 2;                     // query tiles per CTA
 constexpr int kRegionBytes = kTileRows * 128;  // one 64-column SW128 region of a 128-row tile
 constexpr int kTileBytes = 2 * kRegionBytes;   // 128 x 128 bf16
-constexpr int kPrefillThreads = 256;
-constexpr int kSoftmaxWarp0 = 4;
-constexpr uint32_t kTmemCols = 512;            // S0 [0,128), S1 [128,256), O [256,384)
-constexpr uint32_t kColO = 256;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kPrefillThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;               // warps 4-7: tile A, 8-11: tile B
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;                // O_A at 256, O_B at 384
 constexpr float kLazyRescaleLog2 = 8.f;
 constexpr float kLog2eP = 1.4426950408889634f;
 constexpr float kLn2P = 0.6931471805599453f;
 
 struct PrefillCtx {
-  int m, n, fill, wp, T, i0;
-  int np, nr, no, jt0, total;
+  int m, n, fill, wp, T, i0;  // i0: first query row of the CTA (tile A)
+  int np, nr, jt0, jt1, total;
   int has_ring;
 };
 
 struct __align__(1024) PrefillSmem {
-  uint8_t q[kTileBytes];
-  uint8_t k[2][kTileBytes];
-  uint8_t v[2][kTileBytes];
-  uint8_t p[2][kTileBytes];
+  uint8_t q[kQTiles][kTileBytes];
+  uint8_t k[kKStages][kTileBytes];
+  uint8_t v[kVStages][kTileBytes];
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], s_empty[2], p_full[2];
-  uint64_t o_done;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
   uint32_t tmem_base;
   int abort_flag;
   PrefillCtx ctx;
@@ -90,13 +97,25 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
+// D[tmem] (+)= A[smem desc] * B[smem desc]
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -122,10 +141,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 2^x on the MUFU unit (the hardware's approximate base-2 exponential, flush-to-zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and stride
 // byte offsets (16-byte units), version 1, 128-byte swizzle.
@@ -144,7 +179,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m128_n128(uint32_t b_mn_major)
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-// ---- tile enumeration shared by every role --------------------------------------
+// ---- key-tile enumeration shared by every role -----------------------------------
 // kind 0: prefix rows [start, start+128); kind 1: ring slots [start, start+128);
 // kind 2: output rows [start, start+128) of this chunk.
 __device__ __forceinline__ void tile_kind(const PrefillCtx& c, int t, int& kind, int& start) {
@@ -187,6 +222,19 @@ __device__ __forceinline__ bool key_visible(const PrefillCtx& c, int kind, int s
   return x < c.T && x <= i && x > i - c.n;
 }
 
+// Does query tile X see anything of key tile t?
+__device__ __forceinline__ bool tile_visible(const PrefillCtx& c, int X, int t) {
+  const int ilo = c.i0 + X * kTileRows;
+  if (ilo >= c.T) return false;
+  const int ihi = min(ilo + kTileRows - 1, c.T - 1);
+  int kind, start;
+  tile_kind(c, t, kind, start);
+  if (kind == 0) return true;
+  if (kind == 1) return ilo <= c.n - 2;
+  const int jhi = min(start + kTileRows - 1, c.T - 1);
+  return start <= ihi && jhi >= ilo - c.n + 1;
+}
+
 struct PrefillArgs {
   int B, H, n, T;
   int64_t cap;
@@ -206,6 +254,22 @@ __device__ __forceinline__ bool wait_or_abort(PrefillSmem& sm, uint64_t* bar, ui
   sm.abort_flag = 1;
   set_status(status, RSWA_DEVICE_WAIT_TIMEOUT);
   return false;
+}
+
+// Masked, scaled scores of one 32-column chunk of a tile (log2 domain).
+__device__ __forceinline__ void mask_chunk(const PrefillCtx& c, int kind, int start, int i, int col0, float scale,
+                                           const uint32_t (&r)[32], float (&x)[32]) {
+  if (kind == 1) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      x[e] = key_visible(c, kind, start, col0 + e, i) ? __uint_as_float(r[e]) * scale : -INFINITY;
+  } else {
+    // visible columns form one interval (lo, hi]: prefix rows below m; outputs i - n < j <= i, j < T
+    const int hi = (kind == 0 ? min(127, c.m - start - 1) : min(127, min(i, c.T - 1) - start)) - col0;
+    const int lo = (kind == 0 ? -1 : max(-1, i - c.n - start)) - col0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = (e > lo && e <= hi) ? __uint_as_float(r[e]) * scale : -INFINITY;
+  }
 }
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -240,7 +304,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     c.m = m;
     c.n = a.n;
     c.T = a.T;
-    c.i0 = qt * kTileRows;
+    c.i0 = qt * kQTiles * kTileRows;
     c.wp = 0;
     c.fill = 0;
     c.has_ring = 0;
@@ -251,28 +315,32 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       } else {
         c.wp = w;
         c.fill = f;
-        c.has_ring = f > 0 && c.i0 <= a.n - 2;  // some query of the tile can still see a ring slot
+        c.has_ring = f > 0 && c.i0 <= a.n - 2;  // some query of the CTA can still see a ring slot
       }
     }
     c.np = (m + kTileRows - 1) / kTileRows;
     c.nr = c.has_ring ? (a.n + kTileRows - 1) / kTileRows : 0;
     const int jlo = c.i0 - a.n + 1;
     c.jt0 = jlo > 0 ? jlo / kTileRows : 0;
-    c.no = qt - c.jt0 + 1;
-    c.total = c.np + c.nr + c.no;
+    const int last_row = min(c.i0 + kQTiles * kTileRows - 1, a.T - 1);
+    c.jt1 = last_row / kTileRows;
+    c.total = c.np + c.nr + (c.jt1 - c.jt0 + 1);
     sm.ctx = c;
     sm.abort_flag = 0;
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], 128);
-      mbar_init(&sm.p_full[s], 128);
     }
-    mbar_init(&sm.o_done, 1);
+    for (int x = 0; x < kQTiles; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], 128);
+      mbar_init(&sm.o_done[x], 1);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {  // TMEM allocation: one warp, result written to shared memory
@@ -289,19 +357,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int total = c.total;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- producer: Q and K tiles ----------------
+    // ---------------- producer: Q (both tiles) and K tiles ----------------
     const int qrow = (int)(bh * a.T) + c.i0;
-    mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-    tma_load_2d(sm.q, &tm_q, 0, qrow, &sm.q_full);
-    tma_load_2d(sm.q + kRegionBytes, &tm_q, 64, qrow, &sm.q_full);
+    mbar_arrive_expect_tx(&sm.q_full, kQTiles * kTileBytes);
+    for (int x = 0; x < kQTiles; ++x) {
+      tma_load_2d(sm.q[x], &tm_q, 0, qrow + x * kTileRows, &sm.q_full);
+      tma_load_2d(sm.q[x] + kRegionBytes, &tm_q, 64, qrow + x * kTileRows, &sm.q_full);
+    }
     int issued = 0;
     for (int t = 0; t < total; ++t) {
-      const int s = t & 1;
-      if (t >= 2 && !wait_or_abort(sm, &sm.k_empty[s], ((t >> 1) - 1) & 1, a.status)) break;
+      const int s = t % kKStages;
+      if (t >= kKStages && !wait_or_abort(sm, &sm.k_empty[s], ((t / kKStages) - 1) & 1, a.status)) break;
       int kind, start;
       tile_kind(c, t, kind, start);
       const CUtensorMap* map = kind == 0 ? &tm_pk : (kind == 1 ? &tm_rk : &tm_ko);
-      const int row = kind == 0 ? (int)(bh * a.cap) + start : (kind == 1 ? (int)(bh * a.n) + start : (int)(bh * a.T) + start);
+      const int row =
+          kind == 0 ? (int)(bh * a.cap) + start : (kind == 1 ? (int)(bh * a.n) + start : (int)(bh * a.T) + start);
       mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
       tma_load_2d(sm.k[s], map, 0, row, &sm.k_full[s]);
       tma_load_2d(sm.k[s] + kRegionBytes, map, 64, row, &sm.k_full[s]);
@@ -309,74 +380,72 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     if (sm.abort_flag) {  // let the copies in flight land before shared memory is released
       mbar_wait(&sm.q_full, 0);
-      for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait(&sm.k_full[t & 1], (t >> 1) & 1);
+      for (int t = max(0, issued - kKStages); t < issued; ++t)
+        mbar_wait(&sm.k_full[t % kKStages], (t / kKStages) & 1);
     }
   } else if (warp == 2 && lane == 0) {
     // ---------------- producer: V tiles ----------------
     int issued = 0;
     for (int t = 0; t < total; ++t) {
-      const int s = t & 1;
-      if (t >= 2 && !wait_or_abort(sm, &sm.v_empty[s], ((t >> 1) - 1) & 1, a.status)) break;
+      const int s = t % kVStages;
+      if (t >= kVStages && !wait_or_abort(sm, &sm.v_empty[s], ((t / kVStages) - 1) & 1, a.status)) break;
       int kind, start;
       tile_kind(c, t, kind, start);
       const CUtensorMap* map = kind == 0 ? &tm_pv : (kind == 1 ? &tm_rv : &tm_vo);
-      const int row = kind == 0 ? (int)(bh * a.cap) + start : (kind == 1 ? (int)(bh * a.n) + start : (int)(bh * a.T) + start);
+      const int row =
+          kind == 0 ? (int)(bh * a.cap) + start : (kind == 1 ? (int)(bh * a.n) + start : (int)(bh * a.T) + start);
       mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
       tma_load_2d(sm.v[s], map, 0, row, &sm.v_full[s]);
       tma_load_2d(sm.v[s] + kRegionBytes, map, 64, row, &sm.v_full[s]);
       issued = t + 1;
     }
     if (sm.abort_flag)
-      for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait(&sm.v_full[t & 1], (t >> 1) & 1);
+      for (int t = max(0, issued - kVStages); t < issued; ++t)
+        mbar_wait(&sm.v_full[t % kVStages], (t / kVStages) & 1);
   } else if (warp == 1) {
     // ---------------- MMA issuer (lane 0) + V-row zeroing (whole warp) ----------------
     constexpr uint32_t kIdescQK = idesc_bf16_m128_n128(0);
     constexpr uint32_t kIdescPV = idesc_bf16_m128_n128(1);
-    const uint32_t q_addr = smem_addr(sm.q);
+    int n_s[kQTiles] = {0, 0};   // S issued per query tile
+    int n_pv[kQTiles] = {0, 0};  // P.V issued per query tile
     bool ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.q_full, 0, a.status));
-    auto issue_s = [&](int t) {  // S[t&1] = Q K_t^T
-      const uint32_t k_addr = smem_addr(sm.k[t & 1]);
-      const uint32_t d = tmem + (uint32_t)(t & 1) * 128u;
+    auto issue_s = [&](int x, int t) {  // S_x = Q_x K_t^T
+      const uint32_t q_addr = smem_addr(sm.q[x]);
+      const uint32_t k_addr = smem_addr(sm.k[t % kKStages]);
       if (lane == 0) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (uint32_t)(kk >> 2) * kRegionBytes + (uint32_t)(kk & 3) * 32u;
-          tc_mma_f16(d, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK,
-                     kk > 0);
+          tc_mma_ss(tmem + (uint32_t)x * 128u, smem_desc_sw128(q_addr + off, 16, 1024),
+                    smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0);
         }
-        tc_commit(&sm.s_full[t & 1]);
-        tc_commit(&sm.k_empty[t & 1]);
+        tc_commit(&sm.s_full[x]);
       }
       __syncwarp();
+      ++n_s[x];
     };
-    if (ok && total > 0) {
+    // key tile 0: S for both query tiles
+    if (ok) {
       ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.k_full[0], 0, a.status));
       if (ok) {
         tc_fence_after();
-        issue_s(0);
+        for (int x = 0; x < kQTiles; ++x)
+          if (tile_visible(c, x, 0)) issue_s(x, 0);
+        if (lane == 0) tc_commit(&sm.k_empty[0]);
+        __syncwarp();
       }
     }
     for (int t = 0; ok && t < total; ++t) {
-      if (t + 1 < total) {
-        const int u = t + 1, bs = u & 1;
-        ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.k_full[bs], (u >> 1) & 1, a.status));
-        if (ok && u >= 2) ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.s_empty[bs], ((u >> 1) - 1) & 1, a.status));
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(u);
-      }
-      const int s = t & 1;
-      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.p_full[s], (t >> 1) & 1, a.status));
-      if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.v_full[s], (t >> 1) & 1, a.status));
+      const int vs = t % kVStages;
+      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.v_full[vs], (t / kVStages) & 1, a.status));
       if (!ok) break;
-      // zero V rows of keys no query can see (their P is 0; their bytes may be anything)
       int kind, start;
       tile_kind(c, t, kind, start);
       bool zeroed = false;
       for (int r = lane; r < kTileRows; r += 32) {
         if (!key_exists(c, kind, start, r)) {
-          uint4* row0 = reinterpret_cast<uint4*>(sm.v[s] + r * 128);
-          uint4* row1 = reinterpret_cast<uint4*>(sm.v[s] + kRegionBytes + r * 128);
+          uint4* row0 = reinterpret_cast<uint4*>(sm.v[vs] + r * 128);
+          uint4* row1 = reinterpret_cast<uint4*>(sm.v[vs] + kRegionBytes + r * 128);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             row0[e] = make_uint4(0, 0, 0, 0);
@@ -387,132 +456,141 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       if (__any_sync(0xffffffffu, zeroed)) fence_async_smem();
       __syncwarp();
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t p_addr = smem_addr(sm.p[s]);
-        const uint32_t v_addr = smem_addr(sm.v[s]);
+      const bool next = t + 1 < total;
+      bool k_next_ready = false;
+      for (int x = 0; ok && x < kQTiles; ++x) {
+        if (tile_visible(c, x, t)) {
+          ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.p_full[x], n_pv[x] & 1, a.status));
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t v_addr = smem_addr(sm.v[vs]);
+            const uint32_t p_tmem = tmem + (uint32_t)x * 128u;
+            const uint32_t o_tmem = tmem + kColO + (uint32_t)x * 128u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a_off = (uint32_t)(kk >> 2) * kRegionBytes + (uint32_t)(kk & 3) * 32u;
-          const uint32_t b_off = (uint32_t)kk * 16u * 128u;  // 16 keys = two 8-row groups
-          tc_mma_f16(tmem + kColO, smem_desc_sw128(p_addr + a_off, 16, 1024),
-                     smem_desc_sw128(v_addr + b_off, kRegionBytes, 1024), kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)  // 16 keys per step: 8 packed TMEM columns of P, two 8-row groups of V
+              tc_mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u, smem_desc_sw128(v_addr + (uint32_t)kk * 2048u, kRegionBytes, 1024),
+                        kIdescPV, (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&sm.o_done[x]);
+          }
+          __syncwarp();
+          ++n_pv[x];
         }
-        tc_commit(&sm.v_empty[s]);
-        tc_commit(&sm.o_done);
+        if (next && tile_visible(c, x, t + 1)) {
+          if (!k_next_ready) {
+            ok = __all_sync(0xffffffffu,
+                            wait_or_abort(sm, &sm.k_full[(t + 1) % kKStages], ((t + 1) / kKStages) & 1, a.status));
+            if (!ok) break;
+            tc_fence_after();
+            k_next_ready = true;
+          }
+          issue_s(x, t + 1);
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(&sm.v_empty[vs]);
+      if (next) {
+        if (!k_next_ready) {  // no query tile needed it: still let the copy land before freeing the stage
+          ok = __all_sync(0xffffffffu,
+                          wait_or_abort(sm, &sm.k_full[(t + 1) % kKStages], ((t + 1) / kKStages) & 1, a.status));
+          if (!ok) break;
+        }
+        if (lane == 0) tc_commit(&sm.k_empty[(t + 1) % kKStages]);
       }
       __syncwarp();
     }
-    if (!ok && lane == 0) {  // make sure every MMA this thread issued has finished before TMEM goes away
-      tc_commit(&sm.o_done);
-    }
+    if (!ok && lane == 0) tc_commit(&sm.o_done[0]);  // drain: the barrier fires once every issued MMA is done
   } else if (warp >= kSoftmaxWarp0) {
-    // ---------------- softmax: thread r owns query row r ----------------
-    const int r = tid - kSoftmaxWarp0 * 32;
-    const int i = c.i0 + r;
-    const uint32_t lane_base = (uint32_t)((warp - kSoftmaxWarp0) * 32) << 16;
+    // ---------------- softmax: warps 4-7 own tile A, 8-11 tile B; thread r owns row r ----------------
+    const int x = (warp - kSoftmaxWarp0) / 4;
+    const int r = tid - (kSoftmaxWarp0 + 4 * x) * 32;
+    const int i = c.i0 + x * kTileRows + r;
+    const uint32_t lane_base = (uint32_t)(((warp - kSoftmaxWarp0) & 3) * 32) << 16;
+    const uint32_t s_cols = tmem + lane_base + (uint32_t)x * 128u;
+    const uint32_t o_cols = tmem + lane_base + kColO + (uint32_t)x * 128u;
     // l normalises O with the same bf16-rounded weights the MMA used; lu (unrounded) gives lse
     float m_used = -INFINITY, l = 0.f, lu = 0.f;
+    int j = 0;  // visible key tiles seen so far
     bool ok = true;
     for (int t = 0; t < total; ++t) {
-      const int s = t & 1;
-      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.s_full[s], (t >> 1) & 1, a.status));
+      if (!tile_visible(c, x, t)) continue;
+      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.s_full[x], j & 1, a.status));
       if (!ok) break;
       tc_fence_after();
-      float x[128];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)s * 128u + (uint32_t)ch * 32u, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[ch * 32 + e] = __uint_as_float(rr[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(&sm.s_empty[s]);
       int kind, start;
       tile_kind(c, t, kind, start);
+      // pass 1: the tile's row maximum
       float tmax = -INFINITY;
-      if (kind == 1) {
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t rr[32];
+        float xv[32];
+        tmem_ld32(s_cols + (uint32_t)ch * 32u, rr);
+        tmem_wait_ld();
+        mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          x[e] = key_visible(c, kind, start, e, i) ? x[e] * a.qk_scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, x[e]);
-        }
-      } else {
-        // visible columns form one interval (lo, hi]: prefix rows below m; outputs with i - n < j <= i, j < T
-        const int hi = kind == 0 ? min(127, c.m - start - 1) : min(127, min(i, c.T - 1) - start);
-        const int lo = kind == 0 ? -1 : max(-1, i - c.n - start);
-#pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          x[e] = (e > lo && e <= hi) ? x[e] * a.qk_scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, x[e]);
-        }
+        for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, xv[e]);
       }
       const bool rescale = tmax > m_used + kLazyRescaleLog2;
       float alpha = 1.f;
       if (rescale) {
-        alpha = exp2f(m_used - tmax);  // 0 while nothing has been seen
+        alpha = ex2(m_used - tmax);  // 0 while nothing has been seen
         l *= alpha;
         lu *= alpha;
         m_used = tmax;
       }
-      uint32_t pk[64];
-      float lsum = 0.f, lusum = 0.f;
-      const float m_sub = m_used == -INFINITY ? 0.f : m_used;  // a row with nothing visible yet: exp2(-inf) = 0
+      // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp rescales its O rows
+      // together, lanes that keep their max with alpha = 1. PV of the previous visible tile is
+      // complete (see the header).
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t rr[32];
+          tmem_ld32(o_cols + (uint32_t)ch * 32u, rr);
+          tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const float p0 = exp2f(x[2 * e] - m_sub);
-        const float p1 = exp2f(x[2 * e + 1] - m_sub);
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
-        lsum += __low2float(pb) + __high2float(pb);
-        lusum += p0 + p1;
+          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+          tmem_st32(o_cols + (uint32_t)ch * 32u, rr);
+        }
+      }
+      const float m_sub = m_used == -INFINITY ? 0.f : m_used;  // a row with nothing visible yet: exp2(-inf) = 0
+      // pass 2: P = 2^(s - m) as bf16 pairs, written over the first 64 columns of this tile's S
+      float lsum = 0.f, lusum = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t rr[32];
+        float xv[32];
+        tmem_ld32(s_cols + (uint32_t)ch * 32u, rr);
+        tmem_wait_ld();
+        mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(xv[2 * e] - m_sub);
+          const float p1 = ex2(xv[2 * e + 1] - m_sub);
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
+          lsum += __low2float(pb) + __high2float(pb);
+          lusum += p0 + p1;
+        }
+        tmem_st16(s_cols + (uint32_t)ch * 16u, pk);
       }
       l += lsum;
       lu += lusum;
-      if (t >= 1) {
-        // O and the P buffer are touched below: PV of the previous tile must be complete
-        ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.o_done, (t - 1) & 1, a.status));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t rr[32];
-            const uint32_t ta = tmem + lane_base + kColO + (uint32_t)ch * 32u;
-            tmem_ld32(ta, rr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st32(ta, rr);
-          }
-          tmem_wait_st();
-        }
-      }
-      // P row -> 128B-swizzled K-major tile: 16-byte chunk c of row r sits at chunk (c ^ (r & 7))
-      uint8_t* prow0 = sm.p[s] + r * 128;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int region = ch >> 3, cc = ch & 7;
-        uint4 val = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(prow0 + region * kRegionBytes + ((cc ^ (r & 7)) << 4)) = val;
-      }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[s]);
+      mbar_arrive(&sm.p_full[x]);
+      ++j;
     }
-    if (ok && total > 0) {
-      ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.o_done, (total - 1) & 1, a.status));
-    }
-    if (ok) {
+    if (ok && j > 0) ok = __all_sync(0xffffffffu, wait_or_abort(sm, &sm.o_done[x], (j - 1) & 1, a.status));
+    if (ok && j > 0) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float* orow = a.out + (bh * a.T + i) * kHeadDim;
-#pragma unroll
+#pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + kColO + (uint32_t)ch * 32u, rr);
+        tmem_ld32(o_cols + (uint32_t)ch * 32u, rr);
         tmem_wait_ld();
         if (i < c.T) {
 #pragma unroll
@@ -530,7 +608,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    if (sm.abort_flag && lane == 0) mbar_wait(&sm.o_done, 0);  // bounded; MMAs drain before TMEM is freed
+    if (sm.abort_flag && lane == 0) mbar_wait(&sm.o_done[0], 0);  // bounded; MMAs drain before TMEM is freed
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
@@ -640,7 +718,7 @@ cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t stream) {
   const size_t smem = prefill_smem_bytes();
   static unsigned long long done = 0;
   if ((e = ensure_smem_limit(prefill_kernel, smem, &done)) != cudaSuccess) return e;
-  const dim3 grid((L.T + kTileRows - 1) / kTileRows, L.H, L.B);
+  const dim3 grid((L.T + kQTiles * kTileRows - 1) / (kQTiles * kTileRows), L.H, L.B);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   fill_launch_config(cfg, attr, grid, dim3(kPrefillThreads), smem, stream);
