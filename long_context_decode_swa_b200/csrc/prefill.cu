@@ -508,7 +508,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t lane_base = (uint32_t)(((warp - kSoftmaxWarp0) & 3) * 32) << 16;
     const uint32_t s_cols = tmem + lane_base + (uint32_t)x * 128u;
     const uint32_t o_cols = tmem + lane_base + kColO + (uint32_t)x * 128u;
-    // l normalises O with the same bf16-rounded weights the MMA used; lu (unrounded) gives lse
+    // l normalises O with the same bf16-rounded weights the MMA used (a peaked softmax
+    // would otherwise carry the rounding of its dominant weight into O's scale);
+    // lu, the sum of the unrounded exponentials, gives lse
     float m_used = -INFINITY, l = 0.f, lu = 0.f;
     int j = 0;  // visible key tiles seen so far
     bool ok = true;
@@ -519,18 +521,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_fence_after();
       int kind, start;
       tile_kind(c, t, kind, start);
-      // pass 1: the tile's row maximum
+      // a prefix tile that lies wholly inside the prefix is visible to every row: no mask
+      const bool full = kind == 0 && start + kTileRows <= c.m;
+      // pass 1: the tile's row maximum (on raw scores for a full tile: the scale is positive)
       float tmax = -INFINITY;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t rr[32];
-        float xv[32];
         tmem_ld32(s_cols + (uint32_t)ch * 32u, rr);
         tmem_wait_ld();
-        mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
+        if (full) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, xv[e]);
+          for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(rr[e]));
+        } else {
+          float xv[32];
+          mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, xv[e]);
+        }
       }
+      if (full) tmax *= a.qk_scale_log2;
       const bool rescale = tmax > m_used + kLazyRescaleLog2;
       float alpha = 1.f;
       if (rescale) {
@@ -559,19 +569,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t rr[32];
-        float xv[32];
         tmem_ld32(s_cols + (uint32_t)ch * 32u, rr);
         tmem_wait_ld();
-        mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
         uint32_t pk[16];
+        if (full) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(xv[2 * e] - m_sub);
-          const float p1 = ex2(xv[2 * e + 1] - m_sub);
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
-          lsum += __low2float(pb) + __high2float(pb);
-          lusum += p0 + p1;
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(rr[2 * e]), a.qk_scale_log2, -m_sub));
+            const float p1 = ex2(fmaf(__uint_as_float(rr[2 * e + 1]), a.qk_scale_log2, -m_sub));
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
+            lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+            lusum += p0 + p1;
+          }
+        } else {
+          float xv[32];
+          mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(xv[2 * e] - m_sub);
+            const float p1 = ex2(xv[2 * e + 1] - m_sub);
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
+            lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+            lusum += p0 + p1;
+          }
         }
         tmem_st16(s_cols + (uint32_t)ch * 16u, pk);
       }
