@@ -199,10 +199,10 @@ RSWA_API rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, 
  * blk_idx  : int32 [B][topk];  blk_logp : f32 [B][topk]
  * probs    : f32 [B][ceil(prefix_cap / 32)] or NULL (zero past NB)
  * tau      : f32 [B] or NULL: the threshold of the x = z/2 problem
- * workspace: zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_ROUTE) bytes (status word,
- *            per-sequence counters, chunk top lists and the block scores)
- * The scores are computed by ceil(NB / 512) CTAs per sequence; the last one to finish
- * merges their sorted top-32 lists and solves the threshold.
+ * workspace: zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_ROUTE) bytes (status word)
+ * One thread-block cluster of ceil(ceil(prefix_cap / 32) / 1024) CTAs per sequence scores
+ * the blocks; the CTAs hand their sorted top-32 lists and candidates to the first CTA
+ * through distributed shared memory, which merges them and solves the threshold.
  * Unsupported: ceil(prefix_cap / 32) > 8192.
  */
 RSWA_API rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,

@@ -98,7 +98,6 @@ size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
       return most;
     }
     case RSWA_OP_ROUTE:
-      return rswa::plan_route_workspace(dims->batch, dims->prefix_cap).bytes;
     case RSWA_OP_PREFILL:
       return 256;
     default:
@@ -318,11 +317,9 @@ rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* 
     return fail(RSWA_ERR_UNSUPPORTED, "%s: %lld prefix blocks exceed the router's limit of %d", fn,
                 (long long)nb_cap, rswa::kMaxRouteBlocks);
   if (nb_cap == 0) return fail(RSWA_ERR_INVALID, "%s: prefix_cap must be >= 1", fn);
-  const size_t need = rswa::plan_route_workspace(dims->batch, dims->prefix_cap).bytes;
-  if (ws_bytes < need)
-    return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes, need);
+  if (ws_bytes < 256) return fail(RSWA_ERR_INVALID, "%s: workspace must be at least 256 bytes", fn);
   cudaError_t e = rswa::launch_route(dims->batch, dims->prefix_cap, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx,
-                                     blk_logp, probs, tau, workspace, static_cast<cudaStream_t>(stream));
+                                     blk_logp, probs, tau, ws_status(workspace), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
 }

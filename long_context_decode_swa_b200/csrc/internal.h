@@ -52,16 +52,11 @@ cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_
 cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream);
 cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const int32_t* prefix_len, float* kbar,
                               cudaStream_t stream);
-// Router workspace: [status: 256 B][counters: int32 per sequence][chunk maxima]
-// [chunk top-32 lists: (z, block) pairs][block scores z: f32 per block].
-struct RouteWorkspace {
-  int nb_cap, chunks_cap;
-  size_t counters_off, cmax_off, cand_off, zbuf_off, bytes;
-};
-RouteWorkspace plan_route_workspace(int B, int64_t cap);
+// CTAs per sequence of the router (its thread-block cluster size).
+int route_cluster_size(int64_t cap);
 cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
                          float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                         void* workspace, cudaStream_t stream);
+                         int32_t* status, cudaStream_t stream);
 
 struct PrefillLaunch {
   int B, H, n, T;

@@ -18,6 +18,8 @@
 //     tau_k = S1/k - sqrt(delta_k);
 //   * the support size is the largest k with delta_k >= 0 and tau_k < y_(k).
 // Shifting by max x keeps the fp32 sums small (shift invariance of entmax).
+#include <cooperative_groups.h>
+
 #include <cmath>
 
 #include "common.cuh"
@@ -81,6 +83,7 @@ __device__ __forceinline__ bool ranks_before(float za, int ia, float zb, int ib)
 }
 
 constexpr int kNone = 0x7fffffff;
+constexpr int kMaxClusterCtas = 8;  // portable cluster size: up to 8 x 1024 = 8192 blocks
 constexpr int kList = 32;  // sorted candidates kept per warp / per chunk (>= the largest topk)
 
 // Compare-exchange with the lane `j` apart: the lane whose bit j equals `keep_better_bit`
@@ -116,7 +119,7 @@ __device__ __forceinline__ void warp_merge(float& z, int& i, float bz, int bi, i
 
 struct RouteArgs {
   int64_t cap;
-  int nb_cap, chunks_cap, topk;
+  int nb_cap, csize, topk;  // csize: CTAs per sequence (the cluster size)
   float idx_scale;
   const float* q_idx;
   const float* kbar;
@@ -126,10 +129,6 @@ struct RouteArgs {
   float* probs;
   float* tau;
   int32_t* status;
-  int32_t* counters;  // [B]
-  float* cmax;        // [B][chunks_cap]
-  float2* cand;       // [B][chunks_cap][kList]: (z, block index as int bits)
-  float* zbuf;        // [B][nb_cap]
 };
 
 // Merges `n` sorted lists of kList held in (lz, li) shared arrays into lists[0]; every
@@ -156,30 +155,47 @@ __device__ void merge_lists(float (*lz)[kList], int (*li)[kList], int n, int war
   }
 }
 
-// One CTA scores kRouteThreads blocks of one sequence (grid = chunks x B), keeps their
-// sorted top-kList, and the last CTA of the sequence merges the chunk lists and solves
-// the 1.5-entmax threshold exactly.
+// One thread-block cluster per sequence (grid = csize x B, cluster = csize x 1).
+// CTA r scores blocks [1024 r, 1024 r + 1024) (two per thread), keeps their sorted
+// top-32 and the candidates z > (its own max) - 2, and stores list, maximum and
+// candidates into CTA 0's shared memory over DSMEM (the global candidates
+// z > max z - 2 are among them: every CTA's max is at most the global one).
+// After one cluster barrier CTA 0 merges the lists and solves the threshold.
+// With probs requested, CTA 0 sends tau back and every CTA writes its blocks' p.
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ float lz[kRouteWarps][kList];
   __shared__ int li[kRouteWarps][kList];
+  __shared__ float cl_z[kMaxClusterCtas][kList];  // on CTA 0: every CTA's sorted list
+  __shared__ int cl_i[kMaxClusterCtas][kList];
+  __shared__ float cl_max[kMaxClusterCtas];
+  __shared__ int cl_cnt[kMaxClusterCtas];
   __shared__ float red[kRouteWarps];
-  __shared__ int s_last, s_count;
+  __shared__ int s_cnt;
   __shared__ unsigned long long s_best;  // (support size << 32) | bits(tau_y)
+  __shared__ float s_tau_y, s_xmax;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
 
-  const int chunk = blockIdx.x, b = blockIdx.y;
+  const int rank = (int)cluster.block_rank(), b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int region = kRouteThreads * 2;  // blocks per CTA
+  float* cand_z = reinterpret_cast<float*>(smem_raw);  // [csize * region] on CTA 0
+  int* cand_i = reinterpret_cast<int*>(cand_z + a.csize * region);
+  float* cy = reinterpret_cast<float*>(cand_i + a.csize * region);  // compacted global candidates
+  int* ci = reinterpret_cast<int*>(cy + a.csize * region);
+  float* sy = cand_z;  // rank-ordered candidates (reuses cand_z once compacted)
+
   griddep_wait();
   griddep_launch_dependents();
   int64_t m64 = a.prefix_len[b];
   if (m64 < 0 || m64 > a.cap) {
-    if (tid == 0 && chunk == 0) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
+    if (tid == 0 && rank == 0) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
     m64 = 0;
   }
   const int NB = (int)((m64 + kBlock - 1) / kBlock);
-  const int chunks = (NB + kRouteThreads - 1) / kRouteThreads;
-  if (NB == 0) {
-    if (chunk == 0) {
+  if (NB == 0) {  // uniform over the cluster: no barrier is reached
+    if (rank == 0) {
       if (tid < a.topk) {
         a.blk_idx[(int64_t)b * a.topk + tid] = -1;
         a.blk_logp[(int64_t)b * a.topk + tid] = -INFINITY;
@@ -190,89 +206,133 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     }
     return;
   }
-  if (chunk >= chunks) return;
 
-  // ---- score one block per thread ----
-  const int c = chunk * kRouteThreads + tid;
-  float z = -INFINITY;
-  int ci = kNone;
-  if (c < NB) {
+  // ---- score two blocks per thread ----
+  float z[2];
+  int cidx[2];
+  {
     const float4* q4 = reinterpret_cast<const float4*>(a.q_idx + (int64_t)b * kIndexDim);
-    const float4* k4 = reinterpret_cast<const float4*>(a.kbar + ((int64_t)b * a.nb_cap + c) * kIndexDim);
-    float4 kv[8];
+    float4 qv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) kv[u] = k4[u];
-    float d = 0.f;
+    for (int u = 0; u < 8; ++u) qv[u] = q4[u];
+    float4 kv[2][8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 qv = q4[u];
-      d = fmaf(qv.x, kv[u].x, d);
-      d = fmaf(qv.y, kv[u].y, d);
-      d = fmaf(qv.z, kv[u].z, d);
-      d = fmaf(qv.w, kv[u].w, d);
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int c = rank * region + s2 * kRouteThreads + tid;
+      cidx[s2] = c < NB ? c : kNone;
+      if (c < NB) {
+        const float4* k4 = reinterpret_cast<const float4*>(a.kbar + ((int64_t)b * a.nb_cap + c) * kIndexDim);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) kv[s2][u] = k4[u];
+      }
     }
-    z = a.idx_scale * d;
-    ci = c;
-    a.zbuf[(int64_t)b * a.nb_cap + c] = z;
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      float d = 0.f;
+      if (cidx[s2] != kNone) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          d = fmaf(qv[u].x, kv[s2][u].x, d);
+          d = fmaf(qv[u].y, kv[s2][u].y, d);
+          d = fmaf(qv[u].z, kv[s2][u].z, d);
+          d = fmaf(qv[u].w, kv[s2][u].w, d);
+        }
+      }
+      z[s2] = cidx[s2] != kNone ? a.idx_scale * d : -INFINITY;
+    }
   }
-  const float wmax = warp_max(z);
+  // ---- this CTA's maximum and sorted top-32 ----
+  const float wmax = warp_max(fmaxf(z[0], z[1]));
   if (lane == 0) red[warp] = wmax;
-  warp_sort(z, ci, lane);
-  lz[warp][lane] = z;
-  li[warp][lane] = ci;
+  float za = z[0], zb = z[1];
+  int ia = cidx[0], ib = cidx[1];
+  warp_sort(za, ia, lane);
+  warp_sort(zb, ib, lane);
+  {  // merge the two sorted columns: lane l pairs A[l] with B[31 - l]
+    const float rz = __shfl_sync(0xffffffffu, zb, 31 - lane);
+    const int ri = __shfl_sync(0xffffffffu, ib, 31 - lane);
+    warp_merge(za, ia, rz, ri, lane);
+  }
+  lz[warp][lane] = za;
+  li[warp][lane] = ia;
+  if (tid == 0) s_cnt = 0;
   __syncthreads();
+  float lmax = red[0];
+#pragma unroll
+  for (int w = 1; w < kRouteWarps; ++w) lmax = fmaxf(lmax, red[w]);
   merge_lists(lz, li, kRouteWarps, warp, lane);
-  float2* my_list = a.cand + ((int64_t)b * a.chunks_cap + chunk) * kList;
-  if (warp == 0) my_list[lane] = make_float2(lz[0][lane], __int_as_float(li[0][lane]));
-  if (tid == 0) {
-    float mx = red[0];
-    for (int w = 1; w < kRouteWarps; ++w) mx = fmaxf(mx, red[w]);
-    a.cmax[(int64_t)b * a.chunks_cap + chunk] = mx;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&a.counters[b], 1) == chunks - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
 
-  // ---- last CTA of the sequence: merge the chunk lists ----
-  if (warp < chunks) {
-    const float2 e = __ldcg(a.cand + ((int64_t)b * a.chunks_cap + warp) * kList + lane);
-    lz[warp][lane] = e.x;
-    li[warp][lane] = __float_as_int(e.y);
+  // ---- publish list, maximum and candidates to CTA 0 ----
+  float* r_cand_z = cluster.map_shared_rank(cand_z, 0);
+  int* r_cand_i = cluster.map_shared_rank(cand_i, 0);
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+    if (cidx[s2] != kNone && z[s2] > lmax - 2.f) {
+      const int k = atomicAdd(&s_cnt, 1);
+      r_cand_z[rank * region + k] = z[s2];
+      r_cand_i[rank * region + k] = cidx[s2];
+    }
+  }
+  if (warp == 0) {
+    cluster.map_shared_rank(&cl_z[0][0], 0)[rank * kList + lane] = lz[0][lane];
+    cluster.map_shared_rank(&cl_i[0][0], 0)[rank * kList + lane] = li[0][lane];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    cluster.map_shared_rank(cl_max, 0)[rank] = lmax;
+    cluster.map_shared_rank(cl_cnt, 0)[rank] = s_cnt;
+  }
+  cluster.sync();
+
+  if (rank != 0) {
+    if (a.probs == nullptr) return;
+    cluster.sync();  // CTA 0 sends tau
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int c = rank * region + s2 * kRouteThreads + tid;
+      if (c < a.nb_cap) {
+        float pr = 0.f;
+        if (c < NB) {
+          const float r = fmaf(z[s2], 0.5f, -s_xmax) - s_tau_y;
+          pr = r > 0.f ? r * r : 0.f;
+        }
+        a.probs[(int64_t)b * a.nb_cap + c] = pr;
+      }
+    }
+    return;
+  }
+
+  // ---- CTA 0: merge the lists, gather the global candidates, exact threshold ----
+  float zmax = cl_max[0];
+  for (int r = 1; r < a.csize; ++r) zmax = fmaxf(zmax, cl_max[r]);
+  const float xmax = 0.5f * zmax;
+  if (warp < a.csize) {
+    lz[warp][lane] = cl_z[warp][lane];
+    li[warp][lane] = cl_i[warp][lane];
   }
   if (tid == 0) {
-    float mx = -INFINITY;
-    for (int k = 0; k < chunks; ++k) mx = fmaxf(mx, __ldcg(a.cmax + (int64_t)b * a.chunks_cap + k));
-    red[0] = 0.5f * mx;
-    s_count = 0;
+    s_cnt = 0;
     s_best = 0ull;
   }
   __syncthreads();
-  merge_lists(lz, li, chunks, warp, lane);
-  const float xmax = red[0];
-
-  // ---- 1.5-entmax over all NB blocks: candidates x > max x - 1, ranked, prefix sums ----
-  float* cy = reinterpret_cast<float*>(smem_raw);  // [NB] shifted candidates y = x - max x
-  int* cix = reinterpret_cast<int*>(cy + a.nb_cap);
-  float* sy = reinterpret_cast<float*>(cix + a.nb_cap);
-  const float* zb = a.zbuf + (int64_t)b * a.nb_cap;
-  for (int k = tid; k < NB; k += kRouteThreads) {
-    const float y = fmaf(__ldcg(zb + k), 0.5f, -xmax);
-    if (y > -1.f) {
-      const int slot = atomicAdd(&s_count, 1);
-      cy[slot] = y;
-      cix[slot] = k;
+  merge_lists(lz, li, a.csize, warp, lane);
+  for (int r = 0; r < a.csize; ++r) {
+    const int cnt = cl_cnt[r];
+    for (int k = tid; k < cnt; k += kRouteThreads) {
+      const float y = fmaf(cand_z[r * region + k], 0.5f, -xmax);
+      if (y > -1.f) {
+        const int slot = atomicAdd(&s_cnt, 1);
+        cy[slot] = y;
+        ci[slot] = cand_i[r * region + k];
+      }
     }
   }
   __syncthreads();
-  const int K = s_count;
+  const int K = s_cnt;
   for (int i = tid; i < K; i += kRouteThreads) {
     const float yi = cy[i];
-    const int ii = cix[i];
+    const int ii = ci[i];
     int r = 0;
-    for (int j = 0; j < K; ++j) r += ranks_before(cy[j], cix[j], yi, ii) ? 1 : 0;
+    for (int j = 0; j < K; ++j) r += ranks_before(cy[j], ci[j], yi, ii) ? 1 : 0;
     sy[r] = yi;
   }
   __syncthreads();
@@ -295,16 +355,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   __syncthreads();
   const float tau_y = __uint_as_float((unsigned)(s_best & 0xffffffffull));
   if (a.tau && tid == 0) a.tau[b] = tau_y + xmax;
-  if (a.probs) {
-    for (int k = tid; k < a.nb_cap; k += kRouteThreads) {
-      float pr = 0.f;
-      if (k < NB) {
-        const float r = fmaf(__ldcg(zb + k), 0.5f, -xmax) - tau_y;
-        pr = r > 0.f ? r * r : 0.f;
-      }
-      a.probs[(int64_t)b * a.nb_cap + k] = pr;
-    }
-  }
   if (warp == 0 && lane < a.topk) {
     const int64_t o = (int64_t)b * a.topk + lane;
     const int bi = li[0][lane];
@@ -318,7 +368,24 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       a.blk_logp[o] = pr > 0.f ? logf(pr) : -INFINITY;
     }
   }
-  if (tid == 0) a.counters[b] = 0;
+  if (a.probs != nullptr) {
+    if (tid < a.csize) {
+      cluster.map_shared_rank(&s_tau_y, tid)[0] = tau_y;
+      cluster.map_shared_rank(&s_xmax, tid)[0] = xmax;
+    }
+    cluster.sync();
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int c = s2 * kRouteThreads + tid;
+      if (c < a.nb_cap) {
+        float pr = 0.f;
+        if (c < NB) {
+          const float r = fmaf(z[s2], 0.5f, -xmax) - tau_y;
+          pr = r > 0.f ? r * r : 0.f;
+        }
+        a.probs[(int64_t)b * a.nb_cap + c] = pr;
+      }
+    }
+  }
 }
 
 }  // namespace
@@ -331,32 +398,19 @@ cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const i
   return cudaGetLastError();
 }
 
-RouteWorkspace plan_route_workspace(int B, int64_t cap) {
-  RouteWorkspace w;
-  w.nb_cap = (int)((cap + kBlock - 1) / kBlock);
-  w.chunks_cap = (w.nb_cap + kRouteThreads - 1) / kRouteThreads;
-  size_t off = 256;  // status word
-  w.counters_off = off;
-  off += ((size_t)B * 4 + 255) / 256 * 256;
-  w.cmax_off = off;
-  off += ((size_t)B * w.chunks_cap * 4 + 255) / 256 * 256;
-  w.cand_off = off;
-  off += (size_t)B * w.chunks_cap * kList * 8;
-  w.zbuf_off = off;
-  off += (size_t)B * w.nb_cap * 4;
-  w.bytes = off;
-  return w;
+int route_cluster_size(int64_t cap) {
+  const int nb_cap = (int)((cap + kBlock - 1) / kBlock);
+  const int per = kRouteThreads * 2;
+  return (nb_cap + per - 1) / per;
 }
 
 cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
                          float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                         void* workspace, cudaStream_t stream) {
-  const RouteWorkspace w = plan_route_workspace(B, cap);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+                         int32_t* status, cudaStream_t stream) {
   RouteArgs a;
   a.cap = cap;
-  a.nb_cap = w.nb_cap;
-  a.chunks_cap = w.chunks_cap;
+  a.nb_cap = (int)((cap + kBlock - 1) / kBlock);
+  a.csize = route_cluster_size(cap);
   a.topk = topk;
   a.idx_scale = idx_scale;
   a.q_idx = q_idx;
@@ -366,18 +420,19 @@ cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kb
   a.blk_logp = blk_logp;
   a.probs = probs;
   a.tau = tau;
-  a.status = reinterpret_cast<int32_t*>(ws);
-  a.counters = reinterpret_cast<int32_t*>(ws + w.counters_off);
-  a.cmax = reinterpret_cast<float*>(ws + w.cmax_off);
-  a.cand = reinterpret_cast<float2*>(ws + w.cand_off);
-  a.zbuf = reinterpret_cast<float*>(ws + w.zbuf_off);
-  const size_t smem = (size_t)w.nb_cap * 12;
+  a.status = status;
+  const size_t smem = (size_t)a.csize * kRouteThreads * 2 * 16;
   static unsigned long long done = 0;
-  cudaError_t e = ensure_smem_limit(route_kernel, (size_t)kMaxRouteBlocks * 12, &done);
+  cudaError_t e = ensure_smem_limit(route_kernel, (size_t)kMaxClusterCtas * kRouteThreads * 2 * 16, &done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  fill_launch_config(cfg, attr, dim3(w.chunks_cap, B), dim3(kRouteThreads), smem, stream);
+  cudaLaunchAttribute attr[2];
+  fill_launch_config(cfg, attr, dim3(a.csize, B), dim3(kRouteThreads), smem, stream);
+  attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+  attr[cfg.numAttrs].val.clusterDim.x = a.csize;
+  attr[cfg.numAttrs].val.clusterDim.y = 1;
+  attr[cfg.numAttrs].val.clusterDim.z = 1;
+  cfg.numAttrs += 1;
   return cudaLaunchKernelEx(&cfg, route_kernel, a);
 }
 
