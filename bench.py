@@ -200,35 +200,27 @@ def committed_traffic(key: str, src_hash: str):
 
 def dist_setup(args):
     import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from long_context_decode_swa_b200 import replicas
+    world, rank, local = replicas.env_rank()
     if world != args.gpus and "WORLD_SIZE" in os.environ:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         raise SystemExit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
     torch.cuda.set_device(local)
     if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        replicas.init("nccl", timeout_s=120.0, device=torch.device("cuda", local))
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from long_context_decode_swa_b200 import replicas
+    replicas.barrier()
 
 
 def max_over_ranks(world, x: float) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from long_context_decode_swa_b200 import replicas
+    return replicas.max_over_ranks(x, device="cuda")
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -705,9 +697,8 @@ def main():
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        from long_context_decode_swa_b200 import replicas
+        replicas.shutdown()
 
 
 if __name__ == "__main__":
