@@ -11,12 +11,15 @@
 //
 // The path is HBM-bound (about 1 FLOP per byte), so the kernel spends its
 // effort on bytes in flight, not on tensor cores:
-//  * the grid is one wave of resident CTAs; each walks its items in turn and a
-//    producer warp keeps a 4-stage shared-memory ring filled with cp.async.bulk
-//    copies (8 KiB of K and 8 KiB of V per stage) across item boundaries, so
-//    the copy pipeline never drains between items;
-//  * two consumer warps take the tiles round-robin; stage s always belongs to
-//    warp s mod 2, so each warp meets its stages' mbarrier phases in order.
+//  * the grid is one wave of resident CTAs (two per SM); each walks its items
+//    in turn and a producer warp keeps a 6-stage shared-memory ring filled
+//    with cp.async.bulk copies (8 KiB of K and 8 KiB of V per stage) across
+//    item boundaries, so the copy pipeline never drains between items;
+//  * six consumer warps take the tiles round-robin, one stage each (a sweep of
+//    2-8 consumer warps and 1-3 stages per warp put this shape first for the
+//    batched, 32K-history and ragged long-horizon workloads alike); stage s
+//    always belongs to warp s mod 6, so each warp meets its stages' mbarrier
+//    phases in order.
 //    In a warp, lane (g, c) holds dims 8c..8c+7 and rows 2j+g; the 16 partial
 //    dot products of a half-warp are reduce-scattered in 15 shuffles, the
 //    online softmax runs in the exp2 domain, and P.V broadcasts each row's
@@ -36,10 +39,10 @@ namespace rswa {
 namespace {
 
 #ifndef RSWA_DECODE_WARPS
-#define RSWA_DECODE_WARPS 2
+#define RSWA_DECODE_WARPS 6
 #endif
 #ifndef RSWA_DECODE_STAGES_PER_WARP
-#define RSWA_DECODE_STAGES_PER_WARP 2
+#define RSWA_DECODE_STAGES_PER_WARP 1
 #endif
 // Local tile li goes to consumer warp li % kConsumerWarps and to stage
 // li % kStages. kStages is a multiple of kConsumerWarps, so every stage has
