@@ -13,10 +13,13 @@ head_dim 128, a 10-page prefix (2560 visual + 32 prompt tokens) and a full
 
 The K timed steps are captured in one CUDA graph and replayed once (after W
 eager warm-up steps and one untimed replay); CUDA events with external
-record nodes bracket every attention-kernel launch inside the graph, so the
-kernel's average duration is measured on its own stream inside the timed
-region. Inputs (the prefix K/V) are larger than L2, so no flush is needed
-between steps. Under torchrun every rank runs its own batch (weak scaling,
+record nodes bracket the attention (and route) kernel launches of every 8th
+step inside the graph, so the kernels' average durations are measured on
+their own stream inside the timed region (an event node adds several
+microseconds to the step it sits in, so bracketing every step would slow the
+step being timed; the sampled steps' extra time stays in the step time).
+Inputs (the prefix K/V) are larger than L2, so no flush is needed between
+steps. Under torchrun every rank runs its own batch (weak scaling,
 no data-path collective); the timing is the max over ranks.
 
 --impl reference runs the CPU oracle (test infrastructure, fp64) on a bounded
@@ -42,6 +45,7 @@ if ROOT not in sys.path:
 
 METRIC = "decode attn steps/s & achieved HBM GB/s (fraction of peak) on 1 B200"
 FALLBACK_HBM_GBS = 6650.0
+EVENT_EVERY = 8  # kernel durations are bracketed with CUDA events in every 8th timed step
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -102,6 +106,22 @@ def algorithmic_bytes(w: dict, blk_rows=None) -> dict:
     attn = sum((r + n) * 512 + per_q for r in rows) * H
     route = sum(((m + 31) // 32) * 128 + 128 + 16 * 8 for m in w["plen"])
     return dict(attn=attn, route=route)
+
+
+def l2_note(w: dict, nbytes: dict) -> str:
+    """How the timed steps relate to the 126 MB L2 (no flush is issued between steps)."""
+    B, H, n = w["B"], w["H"], w["n"]
+    kv_store = sum(w["plen"]) * H * 512
+    ring = B * H * n * 512
+    if w["kind"] == "rswa":
+        if nbytes["attn"] > 4e8:
+            return f"inputs larger than L2 (each step reads {nbytes['attn'] / 1e9:.2f} GB of K/V); no flush"
+        return "working set fits in L2; numbers are L2-resident"
+    gathered = nbytes["attn"] - ring
+    return (f"no flush: routed prefix blocks change every step (32 planted query directions, cycled; "
+            f"{gathered / 1e6:.0f} MB gathered per step out of a {kv_store / 1e9:.1f} GB K/V store, a direction "
+            f"recurs after 32 steps); the {ring / 1e6:.0f} MB ring is re-read every step, as in decode, and may "
+            f"hit L2")
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -174,12 +194,13 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash(sparse: bool) -> str:
-    files = ["decode.cu", "common.cuh", "internal.h"]
+def kernel_source_hash(kind: str) -> str:
+    """Hash of the sources the measured kernel is built from (kind: dense, sparse or prefill)."""
+    files = ["prefill.cu" if kind == "prefill" else "decode.cu", "common.cuh", "internal.h"]
     h = hashlib.sha256()
     for f in files:
         h.update(open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", f), "rb").read())
-    h.update(b"sparse" if sparse else b"dense")
+    h.update(kind.encode())
     return h.hexdigest()[:16]
 
 
@@ -339,13 +360,16 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
         for i in range(W):
             prob.step(K + i)
     stream.synchronize()
-    # capture the K timed steps, with external event records around the attention (and route) kernels
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(K)]
+    # capture the K timed steps; external event records bracket the attention (and route) kernels of
+    # every EVENT_EVERY-th step (an event node costs several microseconds of step time, so bracketing
+    # every step would slow the step it measures)
+    sampled = list(range(0, K, EVENT_EVERY))
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in sampled]
     graph = torch.cuda.CUDAGraph()
     launches = 0
     with torch.cuda.graph(graph, stream=stream):
         for i in range(K):
-            launches += prob.step(i, ev=evs[i])
+            launches += prob.step(i, ev=evs[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
     graph.replay()                      # untimed replay
     torch.cuda.synchronize()
     status = prob.rswa.check_status(prob.ws)
@@ -387,7 +411,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     achieved = nbytes["attn"] / attn_avg_s / 1e9
     peak, peak_src = measured_peak()
     key = f"{'srswa' if prob.sparse else 'rswa'}_decode_config{args.config}"
-    traffic = committed_traffic(key, kernel_source_hash(prob.sparse))
+    traffic = committed_traffic(key, kernel_source_hash("sparse" if prob.sparse else "dense"))
 
     # ---- e2e through the public API: pinned host inputs -> device -> append/decode -> host result ----
     e2e = run_e2e(prob, K, W) if not args.no_e2e else {"ms": float("nan"), "h2d": 0, "d2h": 0}
@@ -412,9 +436,9 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
         "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "global_batch": B * world,
                    "heads": H, "head_dim": D, "ring": w["n"],
                    "prefix_tokens_mean": statistics.mean(w["plen"]), "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (prefix K/V >> 126 MB); no flush" if nbytes["attn"] > 4e8 else
-                         "working set fits in L2; numbers are L2-resident",
-                   "timing": "K steps in one CUDA graph replay, CUDA events"},
+                   "l2": l2_note(w, nbytes),
+                   "timing": "K steps in one CUDA graph replay, CUDA events; kernel durations from "
+                             f"event brackets in every {EVENT_EVERY}th step"},
         "qtok_per_s": steps_per_s * B * H,
         "seq_tok_per_s": steps_per_s * B,
         "hbm_gbs_step": world * K * (nbytes["attn"] + nbytes["route"]) / (ms_max / 1e3) / 1e9,
@@ -442,11 +466,12 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
         for i in range(W):
             prob.step(i)
     stream.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    sampled = list(range(0, K, EVENT_EVERY))
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in sampled]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(K):
-            prob.step(i, ev=evs[i])
+            prob.step(i, ev=evs[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
     graph.replay()
     torch.cuda.synchronize()
     if prob.rswa.check_status(prob.ws):
@@ -484,11 +509,13 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
         "dtype": "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
         "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "heads": H,
                    "head_dim": w["D"], "ring": w["n"], "chunk": T, "prefix_tokens_mean": statistics.mean(w["plen"]),
-                   "parallelism": f"replicas x{world}", "timing": "K launches in one CUDA graph replay, CUDA events"},
+                   "parallelism": f"replicas x{world}", "timing": "K launches in one CUDA graph replay, CUDA events; kernel durations from "
+                             f"event brackets in every {EVENT_EVERY}th step"},
         "qtok_per_s": value * B * H * T,
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel (tcgen05)", "achieved": achieved, "peak": peak,
                      "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)",
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": committed_traffic(f"rswa_prefill_config{args.config}", kernel_source_hash("prefill")),
                      "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6},
         "kernels_us": {"prefill": kern_s * 1e6},
         "gpu_launches": K,

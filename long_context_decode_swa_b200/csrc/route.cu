@@ -171,8 +171,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   __shared__ float cl_max[kMaxClusterCtas];
   __shared__ int cl_cnt[kMaxClusterCtas];
   __shared__ float red[kRouteWarps];
+  __shared__ int red_i[kRouteWarps];
   __shared__ int s_cnt;
-  __shared__ unsigned long long s_best;  // (support size << 32) | bits(tau_y)
   __shared__ float s_tau_y, s_xmax;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -189,6 +189,62 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   griddep_wait();
   griddep_launch_dependents();
   int64_t m64 = a.prefix_len[b];
+  // ---- score: warp w covers blocks [64 w, 64 w + 64) of the CTA's region ----
+  // The keys are read coalesced, four blocks (512 B) per warp load: octet o = lane / 8
+  // reads block 4i + o of the warp's range, lane j = lane % 8 its dims 4j..4j+3. The
+  // 16 partial dots of a lane are then reduce-scattered over the octet (xor 4, 2, 1),
+  // leaving lane j with the full dots of groups 2j and 2j + 1, i.e. of blocks
+  // 8j + o and 8j + 4 + o. The loads depend only on the capacity, so they are in
+  // flight while prefix_len is still being read.
+  float dot[2];
+  int cpos[2];
+  {
+    const int o = lane >> 3, j = lane & 7;
+    const int wbase = rank * region + warp * 64;
+    const float4 qv = reinterpret_cast<const float4*>(a.q_idx + (int64_t)b * kIndexDim)[j];
+    const float4* k4 = reinterpret_cast<const float4*>(a.kbar + (int64_t)b * a.nb_cap * kIndexDim);
+    float4 kv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = wbase + 4 * i + o;
+      kv[i] = c < a.nb_cap ? k4[(int64_t)c * 8 + j] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    asm volatile("" ::: "memory");  // all 16 loads are issued before the first use
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float d = qv.x * kv[i].x;
+      d = fmaf(qv.y, kv[i].y, d);
+      d = fmaf(qv.z, kv[i].z, d);
+      v[i] = fmaf(qv.w, kv[i].w, d);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool up = j & 4;
+      const float send = up ? v[i] : v[i + 8];
+      const float keep = up ? v[i + 8] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool up = j & 2;
+      const float send = up ? v[i] : v[i + 4];
+      const float keep = up ? v[i + 4] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const bool up = j & 1;
+      const float send = up ? v[i] : v[i + 2];
+      const float keep = up ? v[i + 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      cpos[s2] = wbase + 4 * (2 * j + s2) + o;
+      dot[s2] = v[s2];
+    }
+  }
   if (m64 < 0 || m64 > a.cap) {
     if (tid == 0 && rank == 0) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
     m64 = 0;
@@ -207,39 +263,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     return;
   }
 
-  // ---- score two blocks per thread ----
   float z[2];
   int cidx[2];
-  {
-    const float4* q4 = reinterpret_cast<const float4*>(a.q_idx + (int64_t)b * kIndexDim);
-    float4 qv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) qv[u] = q4[u];
-    float4 kv[2][8];
-#pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-      const int c = rank * region + s2 * kRouteThreads + tid;
-      cidx[s2] = c < NB ? c : kNone;
-      if (c < NB) {
-        const float4* k4 = reinterpret_cast<const float4*>(a.kbar + ((int64_t)b * a.nb_cap + c) * kIndexDim);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) kv[s2][u] = k4[u];
-      }
-    }
-#pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-      float d = 0.f;
-      if (cidx[s2] != kNone) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          d = fmaf(qv[u].x, kv[s2][u].x, d);
-          d = fmaf(qv[u].y, kv[s2][u].y, d);
-          d = fmaf(qv[u].z, kv[s2][u].z, d);
-          d = fmaf(qv[u].w, kv[s2][u].w, d);
-        }
-      }
-      z[s2] = cidx[s2] != kNone ? a.idx_scale * d : -INFINITY;
-    }
+  for (int s2 = 0; s2 < 2; ++s2) {
+    cidx[s2] = cpos[s2] < NB ? cpos[s2] : kNone;
+    z[s2] = cpos[s2] < NB ? a.idx_scale * dot[s2] : -INFINITY;
   }
   // ---- this CTA's maximum and sorted top-32 ----
   const float wmax = warp_max(fmaxf(z[0], z[1]));
@@ -282,13 +311,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     cluster.map_shared_rank(cl_max, 0)[rank] = lmax;
     cluster.map_shared_rank(cl_cnt, 0)[rank] = s_cnt;
   }
-  cluster.sync();
+  if (a.csize > 1)  // uniform over the cluster
+    cluster.sync();
+  else
+    __syncthreads();
 
   if (rank != 0) {
     if (a.probs == nullptr) return;
     cluster.sync();  // CTA 0 sends tau
     for (int s2 = 0; s2 < 2; ++s2) {
-      const int c = rank * region + s2 * kRouteThreads + tid;
+      const int c = cpos[s2];
       if (c < a.nb_cap) {
         float pr = 0.f;
         if (c < NB) {
@@ -309,10 +341,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     lz[warp][lane] = cl_z[warp][lane];
     li[warp][lane] = cl_i[warp][lane];
   }
-  if (tid == 0) {
-    s_cnt = 0;
-    s_best = 0ull;
-  }
+  if (tid == 0) s_cnt = 0;
   __syncthreads();
   merge_lists(lz, li, a.csize, warp, lane);
   for (int r = 0; r < a.csize; ++r) {
@@ -336,6 +365,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     sy[r] = yi;
   }
   __syncthreads();
+  float* tau_r = reinterpret_cast<float*>(ci);  // tau_k by rank k - 1 (ci is free after the ranking)
+  int best = 0;
   for (int r = tid; r < K; r += kRouteThreads) {
     float s1 = 0.f, s2 = 0.f;
     for (int j = 0; j <= r; ++j) {
@@ -346,14 +377,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     const float k = (float)(r + 1);
     const float mean = s1 / k;
     const float delta = (1.f - (s2 - s1 * mean)) / k;
-    if (delta >= 0.f) {
-      const float t = mean - sqrtf(delta);
-      if (t < sy[r])
-        atomicMax(&s_best, ((unsigned long long)(r + 1) << 32) | (unsigned long long)__float_as_uint(t));
-    }
+    const float t = mean - sqrtf(fmaxf(delta, 0.f));
+    tau_r[r] = t;
+    if (delta >= 0.f && t < sy[r]) best = r + 1;
   }
+  best = __reduce_max_sync(0xffffffffu, (unsigned)best);
+  if (lane == 0) red_i[warp] = best;
   __syncthreads();
-  const float tau_y = __uint_as_float((unsigned)(s_best & 0xffffffffull));
+#pragma unroll
+  for (int w = 0; w < kRouteWarps; ++w) best = max(best, red_i[w]);
+  const float tau_y = best > 0 ? tau_r[best - 1] : 0.f;
   if (a.tau && tid == 0) a.tau[b] = tau_y + xmax;
   if (warp == 0 && lane < a.topk) {
     const int64_t o = (int64_t)b * a.topk + lane;
@@ -373,9 +406,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       cluster.map_shared_rank(&s_tau_y, tid)[0] = tau_y;
       cluster.map_shared_rank(&s_xmax, tid)[0] = xmax;
     }
-    cluster.sync();
+    if (a.csize > 1)
+      cluster.sync();
+    else
+      __syncthreads();
     for (int s2 = 0; s2 < 2; ++s2) {
-      const int c = s2 * kRouteThreads + tid;
+      const int c = cpos[s2];
       if (c < a.nb_cap) {
         float pr = 0.f;
         if (c < NB) {
