@@ -12,19 +12,18 @@
 // The path is HBM-bound (about 1 FLOP per byte), so the kernel spends its
 // effort on bytes in flight, not on tensor cores:
 //  * the grid is one wave of resident CTAs (two per SM); each walks its items
-//    in turn and a producer warp keeps a 6-stage shared-memory ring filled
-//    with cp.async.bulk copies (8 KiB of K and 8 KiB of V per stage) across
-//    item boundaries, so the copy pipeline never drains between items;
-//  * six consumer warps take the tiles round-robin, one stage each (a sweep of
-//    2-8 consumer warps and 1-3 stages per warp put this shape first for the
-//    batched, 32K-history and ragged long-horizon workloads alike); stage s
-//    always belongs to warp s mod 6, so each warp meets its stages' mbarrier
-//    phases in order.
-//    In a warp, lane (g, c) holds dims 8c..8c+7 and rows 2j+g; the 16 partial
+//    in turn. Every warp owns one 16 KiB shared-memory stage (8 KiB of K and
+//    8 KiB of V) and streams its own tiles through it with cp.async.bulk: the
+//    CTA-local tiles w, w + 6, w + 12, ... belong to warp w, and right after a
+//    warp has read a tile it issues the copy of its next one into the same
+//    stage, across item boundaries, so there is no producer hand-over on the
+//    refill path and the six copies of a CTA's first tiles start at once;
+//  * in a warp, lane (g, c) holds dims 8c..8c+7 and rows 2j+g; the 16 partial
 //    dot products of a half-warp are reduce-scattered in 15 shuffles, the
 //    online softmax runs in the exp2 domain, and P.V broadcasts each row's
-//    weight with a shuffle;
-//  * at the end of an item the consumer warps merge (named barrier) and either
+//    weight with a shuffle; dots and accumulators use paired f32 FMAs
+//    (fma.rn.f32x2), and full tiles skip the per-row bounds checks;
+//  * at the end of an item the warps merge through shared memory and either
 //    write the output (one split) or a (max, sum, acc) partial; the last item
 //    of a (sequence, head) to finish (atomic counter) merges the partials by
 //    log-sum-exp and resets the counter.
@@ -44,16 +43,14 @@ namespace {
 #ifndef RSWA_DECODE_STAGES_PER_WARP
 #define RSWA_DECODE_STAGES_PER_WARP 1
 #endif
-// Local tile li goes to consumer warp li % kConsumerWarps and to stage
-// li % kStages. kStages is a multiple of kConsumerWarps, so every stage has
-// exactly one consumer warp, which meets that stage's uses in order: the
-// parity of each mbarrier wait then names the right phase (a warp can never
-// wait on a stage two phases ahead of the copy in flight).
-constexpr int kConsumerWarps = RSWA_DECODE_WARPS;
-constexpr int kStages = RSWA_DECODE_WARPS * RSWA_DECODE_STAGES_PER_WARP;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
-static_assert(kStages % kConsumerWarps == 0, "each stage needs a single consumer warp");
+// CTA-local tile li goes to warp li % kWarps; the warp's k-th tile uses its stage
+// warp * kStagesPerWarp + k % kStagesPerWarp. A stage has a single owner warp,
+// which tracks the stage's mbarrier phase itself (empty tiles issue no copy).
+constexpr int kWarps = RSWA_DECODE_WARPS;
+constexpr int kStagesPerWarp = RSWA_DECODE_STAGES_PER_WARP;
+constexpr int kStages = kWarps * kStagesPerWarp;
+constexpr int kDecodeThreads = kWarps * 32;
+static_assert(kStagesPerWarp >= 1 && kStagesPerWarp <= 4, "stages per warp");
 constexpr int kTileBytes = kBlock * kRowBytes;  // 8 KiB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -61,21 +58,16 @@ constexpr float kLn2 = 0.6931471805599453f;
 struct DecodeSmem {
   uint8_t stage[kStages][2][kTileBytes];
   uint64_t full[kStages];
-  uint64_t empty[kStages];
-  int rows[kStages];
-  int tile_id[kStages];  // producer's local tile index for the stage's current use
-  float bias[kStages];   // log2 domain
-  float wm[kConsumerWarps];
-  float wl[kConsumerWarps];
-  float wacc[kConsumerWarps][kHeadDim];
-  int abort_flag;
+  float wm[kWarps];
+  float wl[kWarps];
+  float wacc[kWarps][kHeadDim];
   int is_last;
 };
 
 constexpr int kDecodeMinBlocks =
     (227 * 1024) / (int)sizeof(DecodeSmem) > 0 ? (227 * 1024) / (int)sizeof(DecodeSmem) : 1;
 
-// What the producer needs to enumerate a (sequence, head)'s tiles.
+// What a warp needs to enumerate a (sequence, head)'s tiles.
 struct SeqView {
   const uint16_t* pk;  // prefix rows of this (b, h)
   const uint16_t* pv;
@@ -165,8 +157,126 @@ __device__ __forceinline__ void tile_at(const SeqView& v, int t, int c, float lp
   val = v.rv + (int64_t)start * kHeadDim;
 }
 
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kConsumerThreads) : "memory");
+// An item (sequence, head, split) as one warp sees it while issuing its tiles:
+// the (sequence, head) view, the split's first tile and this lane's route entry.
+struct ItemView {
+  int item;  // -1: none loaded yet
+  int t0;
+  SeqView v;
+  int c;
+  float lp;
+};
+
+template <bool kSparse>
+__device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lane, ItemView& iv) {
+  const int bh = item / a.splits, split = item - bh * a.splits;
+  const int b = bh / a.H, h = bh - b * a.H;
+  iv.item = item;
+  iv.t0 = split * a.tiles_per_item;
+  iv.v = make_view<kSparse>(a, b, h, lane == 0 && split == 0 && h == 0);
+  iv.c = -1;
+  iv.lp = -INFINITY;
+  if (kSparse && lane < a.topk) {
+    iv.c = a.blk_idx[(int64_t)b * a.topk + lane];
+    iv.lp = a.blk_logp[(int64_t)b * a.topk + lane];
+  }
+}
+
+// Issues CTA-local tile li (if it exists) into stage s: one bulk copy of its K rows and
+// one of its V rows on full[s]. Warp-collective. Returns the tile's row count (0: empty
+// or past the CTA's last item, nothing issued) and, in `bias`, its log2-domain bias.
+template <bool kSparse>
+__device__ __forceinline__ int issue_tile(const DecodeArgs& a, DecodeSmem& sm, int li, int s, int lane,
+                                          ItemView& iv, float& bias) {
+  const int P = a.tiles_per_item;
+  const int it = li / P;
+  const int64_t item = (int64_t)blockIdx.x + (int64_t)it * gridDim.x;
+  bias = 0.f;
+  if (item >= a.items) return 0;
+  if (iv.item != (int)item) load_item<kSparse>(a, (int)item, lane, iv);
+  const int tile = iv.t0 + (li - it * P);
+  const int c = __shfl_sync(0xffffffffu, iv.c, tile & 31);
+  const float lp = __shfl_sync(0xffffffffu, iv.lp, tile & 31);
+  const uint16_t *kp, *vp;
+  int rows;
+  tile_at<kSparse>(iv.v, tile, c, lp, kp, vp, rows, bias, lane == 0 ? a.status : nullptr);
+  if (rows > 0 && lane == 0) {
+    const uint32_t bytes = (uint32_t)rows * kRowBytes;
+    mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+    bulk_copy_g2s(sm.stage[s][0], kp, bytes, &sm.full[s]);
+    bulk_copy_g2s(sm.stage[s][1], vp, bytes, &sm.full[s]);
+  }
+  return rows;
+}
+
+__device__ __forceinline__ float2 bf16x2_f2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+
+// One tile for this warp: the 32 scores, the online-softmax update and P.V.
+// kFull: all 32 rows valid (no bounds checks).
+template <bool kFull>
+__device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* vt, int rows, float bias,
+                                             const float2 (&q2)[4], int g, int c, float& m_run, float& l_lane,
+                                             float2 (&acc)[4]) {
+  float pd[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint4 w = *reinterpret_cast<const uint4*>(kt + (2 * j + g) * kRowBytes + c * 16);
+    float2 d = __fmul2_rn(q2[0], bf16x2_f2(w.x));
+    d = __ffma2_rn(q2[1], bf16x2_f2(w.y), d);
+    d = __ffma2_rn(q2[2], bf16x2_f2(w.z), d);
+    d = __ffma2_rn(q2[3], bf16x2_f2(w.w), d);
+    pd[j] = d.x + d.y;
+  }
+  // reduce-scatter the 16 partial dots over the 16 lanes of this half-warp
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = c & 8;
+    const float send = up ? pd[i] : pd[i + 8];
+    const float keep = up ? pd[i + 8] : pd[i];
+    pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = c & 4;
+    const float send = up ? pd[i] : pd[i + 4];
+    const float keep = up ? pd[i + 4] : pd[i];
+    pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = c & 2;
+    const float send = up ? pd[i] : pd[i + 2];
+    const float keep = up ? pd[i + 2] : pd[i];
+    pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  {
+    const bool up = c & 1;
+    const float send = up ? pd[0] : pd[1];
+    const float keep = up ? pd[1] : pd[0];
+    pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  }
+  // this lane now holds the score of tile row 2c + g
+  const float sc = (kFull || 2 * c + g < rows) ? pd[0] + bias : -INFINITY;
+  const float m_new = fmaxf(m_run, warp_max(sc));
+  const float alpha = exp2f(m_run - m_new);
+  const float p = exp2f(sc - m_new);
+  l_lane = fmaf(l_lane, alpha, p);
+  const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] = __fmul2_rn(acc[e], a2);
+  m_run = m_new;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float pj = __shfl_sync(0xffffffffu, p, (g << 4) | j);
+    if (kFull || 2 * j + g < rows) {
+      const uint4 w = *reinterpret_cast<const uint4*>(vt + (2 * j + g) * kRowBytes + c * 16);
+      const float2 p2 = make_float2(pj, pj);
+      acc[0] = __ffma2_rn(p2, bf16x2_f2(w.x), acc[0]);
+      acc[1] = __ffma2_rn(p2, bf16x2_f2(w.y), acc[1]);
+      acc[2] = __ffma2_rn(p2, bf16x2_f2(w.z), acc[2]);
+      acc[3] = __ffma2_rn(p2, bf16x2_f2(w.w), acc[3]);
+    }
+  }
 }
 
 template <bool kSparse>
@@ -177,237 +287,121 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
   const int P = a.tiles_per_item;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
-    }
-    sm.abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
     fence_mbar_init();
   }
   __syncthreads();
   griddep_wait();               // inputs may be written by the previous kernel in the stream
   griddep_launch_dependents();  // the next kernel may start its prologue
 
-  if (warp == kConsumerWarps) {
-    // ---------------- producer warp: lane 0 issues, the warp fetches route entries ----------------
-    int li = 0, issued = 0;
-    bool aborted = false;
-    for (int item = blockIdx.x; item < a.items && !aborted; item += gridDim.x) {
-      const int bh = item / a.splits, split = item - bh * a.splits;
-      const int b = bh / a.H, h = bh - b * a.H;
-      const SeqView v = make_view<kSparse>(a, b, h, lane == 0 && split == 0 && h == 0);
-      int my_c = -1;
-      float my_lp = -INFINITY;
-      if (kSparse && lane < a.topk) {
-        my_c = a.blk_idx[(int64_t)b * a.topk + lane];
-        my_lp = a.blk_logp[(int64_t)b * a.topk + lane];
-      }
-      const int t0 = split * P;
-      for (int t = 0; t < P; ++t, ++li) {
-        const int s = li % kStages;
-        if (li >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ((li / kStages) - 1) & 1))) {
-          aborted = true;
-          break;
-        }
-        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) {
-          aborted = true;
-          break;
-        }
-        const int tile = t0 + t;
-        const int c = __shfl_sync(0xffffffffu, my_c, tile & 31);
-        const float lp = __shfl_sync(0xffffffffu, my_lp, tile & 31);
-        if (lane == 0) {
-          const uint16_t *kp, *vp;
-          int rows;
-          float bias;
-          tile_at<kSparse>(v, tile, c, lp, kp, vp, rows, bias, a.status);
-          sm.rows[s] = rows;
-          sm.bias[s] = bias;
-          sm.tile_id[s] = li;
-          if (rows > 0) {
-            const uint32_t bytes = (uint32_t)rows * kRowBytes;
-            mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
-            bulk_copy_g2s(sm.stage[s][0], kp, bytes, &sm.full[s]);
-            bulk_copy_g2s(sm.stage[s][1], vp, bytes, &sm.full[s]);
-          } else {
-            mbar_arrive(&sm.full[s]);
-          }
-        }
-        __syncwarp();
-        issued = li + 1;
-      }
-    }
-    if (aborted && lane == 0) {
-      sm.abort_flag = 1;
-      set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
-      // let every copy still in flight land before the CTA's shared memory goes away
-      for (int j = max(0, issued - kStages); j < issued; ++j) mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
-    }
-    return;
-  }
-
-  // ---------------- consumer warps ----------------
-  const int g = lane >> 4, c = lane & 15;
-  int li_base = 0;
+  // In-flight tiles of this warp, oldest first: row count and bias of the warp's
+  // tiles k .. k + kStagesPerWarp - 1 (rows 0: nothing issued).
+  ItemView iv;
+  iv.item = -1;
+  int fl_rows[kStagesPerWarp];
+  float fl_bias[kStagesPerWarp];
+#pragma unroll
+  for (int j = 0; j < kStagesPerWarp; ++j)
+    fl_rows[j] = issue_tile<kSparse>(a, sm, warp + j * kWarps, warp * kStagesPerWarp + j, lane, iv, fl_bias[j]);
+  uint32_t phase = 0;  // bit j: parity of the next completion of this warp's stage j
+  int k = 0;           // tiles of this warp consumed so far
   bool ok = true;
+
+  const int g = lane >> 4, c = lane & 15;
   // the next item's query is loaded while the current item streams
   uint4 q_next = make_uint4(0, 0, 0, 0);
   if (blockIdx.x < a.items)
     q_next = *reinterpret_cast<const uint4*>(a.q + (int64_t)(blockIdx.x / a.splits) * kHeadDim + c * 8);
+  int li_base = 0;
   for (int item = blockIdx.x; item < a.items; item += gridDim.x, li_base += P) {
     const int bh = item / a.splits, split = item - bh * a.splits;
     const uint4 q_cur = q_next;
     if (item + (int)gridDim.x < a.items)
       q_next = *reinterpret_cast<const uint4*>(a.q + (int64_t)((item + gridDim.x) / a.splits) * kHeadDim + c * 8);
-    float qf[8];
+    float2 q2[4];
     {
-      const uint4 w = q_cur;
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t ws[4] = {q_cur.x, q_cur.y, q_cur.z, q_cur.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        qf[2 * e] = bf16lo(ws[e]) * a.qscale;
-        qf[2 * e + 1] = bf16hi(ws[e]) * a.qscale;
-      }
+      for (int e = 0; e < 4; ++e) q2[e] = make_float2(bf16lo(ws[e]) * a.qscale, bf16hi(ws[e]) * a.qscale);
     }
     float m_run = -INFINITY, l_lane = 0.f;
-    float acc[8];
+    float2 acc[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
 
-    const int first = li_base + ((warp - li_base % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
-    for (int li = first; ok && li < li_base + P; li += kConsumerWarps) {
-      const int s = li % kStages;
-      // every lane waits (each needs the acquire), then the warp agrees
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (li / kStages) & 1))) {
-        if (lane == 0) {
-          sm.abort_flag = 1;
-          set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
-        }
-        ok = false;
-        break;
-      }
-      if (sm.tile_id[s] != li) {  // protocol check: never compute on another tile's data
-        if (lane == 0) {
-          sm.abort_flag = 1;
-          set_status(a.status, RSWA_DEVICE_PIPELINE);
-        }
-        ok = false;
-        break;
-      }
-      const int rows = sm.rows[s];
+    const int first = li_base + ((warp - li_base % kWarps) + kWarps) % kWarps;
+    for (int li = first; ok && li < li_base + P; li += kWarps) {
+      const int j = k % kStagesPerWarp;
+      const int s = warp * kStagesPerWarp + j;
+      const int rows = fl_rows[0];
       if (rows > 0) {
-        const float bias = sm.bias[s];
-        const uint8_t* kt = sm.stage[s][0];
-        const uint8_t* vt = sm.stage[s][1];
-        float pd[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint4 w = *reinterpret_cast<const uint4*>(kt + (2 * j + g) * kRowBytes + c * 16);
-          float d = qf[0] * bf16lo(w.x);
-          d = fmaf(qf[1], bf16hi(w.x), d);
-          d = fmaf(qf[2], bf16lo(w.y), d);
-          d = fmaf(qf[3], bf16hi(w.y), d);
-          d = fmaf(qf[4], bf16lo(w.z), d);
-          d = fmaf(qf[5], bf16hi(w.z), d);
-          d = fmaf(qf[6], bf16lo(w.w), d);
-          d = fmaf(qf[7], bf16hi(w.w), d);
-          pd[j] = d;
+        // every lane waits (each needs the acquire), then the warp agrees
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (phase >> j) & 1u))) {
+          if (lane == 0) set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
+          ok = false;
+          break;
         }
-        // reduce-scatter the 16 partial dots over the 16 lanes of this half-warp
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const bool up = c & 8;
-          const float send = up ? pd[i] : pd[i + 8];
-          const float keep = up ? pd[i + 8] : pd[i];
-          pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const bool up = c & 4;
-          const float send = up ? pd[i] : pd[i + 4];
-          const float keep = up ? pd[i + 4] : pd[i];
-          pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const bool up = c & 2;
-          const float send = up ? pd[i] : pd[i + 2];
-          const float keep = up ? pd[i + 2] : pd[i];
-          pd[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-        }
-        {
-          const bool up = c & 1;
-          const float send = up ? pd[0] : pd[1];
-          const float keep = up ? pd[1] : pd[0];
-          pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-        }
-        // this lane now holds the score of tile row 2c + g
-        const float sc = (2 * c + g < rows) ? pd[0] + bias : -INFINITY;
-        const float m_new = fmaxf(m_run, warp_max(sc));
-        const float alpha = exp2f(m_run - m_new);
-        const float p = exp2f(sc - m_new);
-        l_lane = fmaf(l_lane, alpha, p);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= alpha;
-        m_run = m_new;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float pj = __shfl_sync(0xffffffffu, p, (g << 4) | j);
-          if (2 * j + g < rows) {
-            const uint4 w = *reinterpret_cast<const uint4*>(vt + (2 * j + g) * kRowBytes + c * 16);
-            acc[0] = fmaf(pj, bf16lo(w.x), acc[0]);
-            acc[1] = fmaf(pj, bf16hi(w.x), acc[1]);
-            acc[2] = fmaf(pj, bf16lo(w.y), acc[2]);
-            acc[3] = fmaf(pj, bf16hi(w.y), acc[3]);
-            acc[4] = fmaf(pj, bf16lo(w.z), acc[4]);
-            acc[5] = fmaf(pj, bf16hi(w.z), acc[5]);
-            acc[6] = fmaf(pj, bf16lo(w.w), acc[6]);
-            acc[7] = fmaf(pj, bf16hi(w.w), acc[7]);
-          }
-        }
+        phase ^= 1u << j;
+        if (rows == kBlock)
+          consume_tile<true>(sm.stage[s][0], sm.stage[s][1], rows, fl_bias[0], q2, g, c, m_run, l_lane, acc);
+        else
+          consume_tile<false>(sm.stage[s][0], sm.stage[s][1], rows, fl_bias[0], q2, g, c, m_run, l_lane, acc);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      __syncwarp();  // every lane has read the stage before it is refilled
+#pragma unroll
+      for (int i = 0; i + 1 < kStagesPerWarp; ++i) {
+        fl_rows[i] = fl_rows[i + 1];
+        fl_bias[i] = fl_bias[i + 1];
+      }
+      fl_rows[kStagesPerWarp - 1] =
+          issue_tile<kSparse>(a, sm, li + kWarps * kStagesPerWarp, s, lane, iv, fl_bias[kStagesPerWarp - 1]);
+      ++k;
     }
     // fold the two half-warps (same dims, different rows) and the lanes' sums
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    for (int e = 0; e < 4; ++e) {
+      acc[e].x += __shfl_xor_sync(0xffffffffu, acc[e].x, 16);
+      acc[e].y += __shfl_xor_sync(0xffffffffu, acc[e].y, 16);
+    }
     const float l = warp_sum(l_lane);
     if (g == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sm.wacc[warp][c * 8 + e] = acc[e];
+      for (int e = 0; e < 4; ++e) {
+        sm.wacc[warp][c * 8 + 2 * e] = acc[e].x;
+        sm.wacc[warp][c * 8 + 2 * e + 1] = acc[e].y;
+      }
     }
     if (lane == 0) {
       sm.wm[warp] = m_run;
       sm.wl[warp] = l;
     }
-    consumer_sync();
+    __syncthreads();
 
-    // ---------------- merge the consumer warps ----------------
+    // ---------------- merge the warps ----------------
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w]);
-    float fw[kConsumerWarps];
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm.wm[w]);
+    float fw[kWarps];
     float L = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       fw[w] = M > -INFINITY ? exp2f(sm.wm[w] - M) : 0.f;
       L = fmaf(sm.wl[w], fw[w], L);
     }
     if (a.splits == 1) {
-      for (int d = tid; d < kHeadDim; d += kConsumerThreads) {
+      for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
         float A = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
+        for (int w = 0; w < kWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
         a.out[(int64_t)bh * kHeadDim + d] = L > 0.f ? A / L : 0.f;
       }
       if (tid == 0 && a.lse) a.lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     } else {
       float* rec = a.partials + ((int64_t)bh * a.splits + split) * (kHeadDim + 2);
-      for (int d = tid; d < kHeadDim; d += kConsumerThreads) {
+      for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
         float A = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
+        for (int w = 0; w < kWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
         rec[2 + d] = A;
       }
       if (tid == 0) {
@@ -415,9 +409,9 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
         rec[1] = L;
       }
       __threadfence();
-      consumer_sync();
+      __syncthreads();
       if (tid == 0) sm.is_last = (atomicAdd(&a.counters[bh], 1) == a.splits - 1);
-      consumer_sync();
+      __syncthreads();
       if (sm.is_last) {
         __threadfence();
         const float* recs = a.partials + (int64_t)bh * a.splits * (kHeadDim + 2);
@@ -429,7 +423,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
             const float* r = recs + s * (kHeadDim + 2);
             Lg = fmaf(__ldcg(r + 1), exp2f(__ldcg(r) - Mg), Lg);
           }
-        for (int d = tid; d < kHeadDim; d += kConsumerThreads) {
+        for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
           float Ag = 0.f;
           if (Mg > -INFINITY)
             for (int s = 0; s < a.splits; ++s) {
@@ -444,8 +438,18 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
         }
       }
     }
-    consumer_sync();  // the merge buffers are rewritten by the next item
+    // the merge buffers are rewritten by the next item; a warp that gave up ends the CTA
+    if (__syncthreads_or(!ok)) break;
   }
+  // after a give-up, copies issued for later tiles may still be in flight: let them land
+  // before the CTA's shared memory goes away (after a normal end none are left)
+#pragma unroll
+  for (int i = 0; i < kStagesPerWarp; ++i)
+    if (fl_rows[i] > 0) {
+      const int j = (k + i) % kStagesPerWarp;
+      mbar_wait(&sm.full[warp * kStagesPerWarp + j], (phase >> j) & 1u);
+      phase ^= 1u << j;
+    }
 }
 
 }  // namespace
