@@ -442,6 +442,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
         "qtok_per_s": steps_per_s * B * H,
         "seq_tok_per_s": steps_per_s * B,
         "hbm_gbs_step": world * K * (nbytes["attn"] + nbytes["route"]) / (ms_max / 1e3) / 1e9,
+        "bytes_per_step": {"attn": nbytes["attn"], "route": nbytes["route"]},
         "roofline": {"bound": "hbm", "kernel": "srswa decode_kernel<true>" if prob.sparse else
                      "rswa decode_kernel<false>", "achieved": achieved, "peak": peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
@@ -680,6 +681,34 @@ def run_reference(args, w: dict) -> dict:
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+SWEEP_LENGTHS = (8192, 16384, 32768, 65536, 102400)
+
+
+def run_length_sweep(args, world: int, rank: int, local: int) -> dict:
+    """The SR-SWA step at uniform history lengths (16 sequences, top-16 + 128-slot ring).
+
+    The attention reads the same 640 rows per (sequence, head) at every length; only the
+    router's block-key scan (128 B per 32-token block) grows with the history."""
+    import torch
+    rows = []
+    for m in SWEEP_LENGTHS:
+        w = workload(5)
+        w["plen"] = [m] * w["B"]
+        w["cap"] = m
+        w["name"] = f"SR-SWA decode, 16 sequences, 16 heads, head_dim 128, uniform history {m} tokens"
+        r = run_ours(args, w, world, rank, local)
+        rows.append({"history": m, "ms_per_step": r["ms_per_step"], "steps_per_s": r["value"],
+                     "kernels_us": r["kernels_us"], "attn_hbm_frac": r["roofline"]["frac"],
+                     "route_bytes_share": r["bytes_per_step"]["route"] / (r["bytes_per_step"]["attn"] +
+                                                                          r["bytes_per_step"]["route"]),
+                     "clocks": r["clocks"]})
+        torch.cuda.empty_cache()
+    steps = [x["ms_per_step"] for x in rows]
+    return {"metric": "SR-SWA decode step latency vs history length", "unit": "ms/step", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "data": "synthetic",
+            "impl": "ours", "sweep": rows, "max_over_min": max(steps) / min(steps)}
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -695,6 +724,9 @@ def main():
                     help="override the workload's batch (a smaller case, e.g. for an ncu capture)")
     ap.add_argument("--prefix", type=int, default=None,
                     help="override every sequence's prefix length (and the capacity) of the workload")
+    ap.add_argument("--length-sweep", action="store_true",
+                    help="SR-SWA latency against history length: 16 sequences at uniform lengths "
+                         f"{SWEEP_LENGTHS}, one JSON line with every length's step and kernel times")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -718,6 +750,11 @@ def main():
 
     world, rank, local = dist_setup(args)
     try:
+        if args.length_sweep:
+            res = run_length_sweep(args, world, rank, local)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res = run_ours(args, w, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w)
