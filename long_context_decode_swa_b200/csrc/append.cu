@@ -4,8 +4,9 @@
 // head, the pointer advances cyclically and the valid count saturates at n
 // (Unlimited-OCR-2 SR-SWA explainer, 环形缓冲; "百度 Unlimited OCR 深度实战"
 // tutorial §3.3.2). One CTA per sequence copies its H x 256 B of K and of V
-// with 16-byte loads/stores; thread 0 alone reads and advances wp/fill, so no
-// other thread of the launch touches them.
+// with 16-byte loads/stores; the rows are loaded while thread 0 reads wp/fill,
+// so the kernel costs one memory round trip before its stores. Thread 0 alone
+// reads and advances wp/fill, so no other thread of the launch touches them.
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,30 +25,58 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(int H, int n, ui
   const int b = blockIdx.x;
   griddep_wait();  // the previous kernel may still be reading the slot this one overwrites
   griddep_launch_dependents();
+  // the new rows are loaded while thread 0 reads the ring state (one round trip, not two)
+  constexpr int kVecPerRow = kHeadDim / 8;  // uint4 per 128-dim bf16 row
+  constexpr int kMaxVec = 4;  // rows held in registers: 4 x 128 uint4 covers K and V of H <= 16 heads
+  const int per_tensor = H * kVecPerRow;
+  int w = 0, f = 0;
   if (threadIdx.x == 0) {
-    const int w = wp[b], f = fill[b];
+    w = wp[b];
+    f = fill[b];
+  }
+  uint4 row[kMaxVec];
+  int cnt = 0;
+#pragma unroll
+  for (int u = 0; u < kMaxVec; ++u) {
+    const int i = threadIdx.x + u * kAppendThreads;
+    if (i < 2 * per_tensor) {
+      const int which = i / per_tensor;
+      const int j = i - which * per_tensor;
+      row[u] = reinterpret_cast<const uint4*>((which ? v_new : k_new) + (int64_t)b * H * kHeadDim)[j];
+      cnt = u + 1;
+    }
+  }
+  if (threadIdx.x == 0) {
     const bool ok = w >= 0 && w < n && f >= 0 && f <= n;
     if (!ok) set_status(status, RSWA_DEVICE_BAD_RING_STATE);
     s_slot = ok ? w : -1;
+    if (ok) {
+      wp[b] = (w + 1 == n) ? 0 : w + 1;
+      fill[b] = min(f + 1, n);
+      if (slot_out) slot_out[b] = w;
+    }
   }
   __syncthreads();
   const int slot = s_slot;
   if (slot < 0) return;
-  constexpr int kVecPerRow = kHeadDim / 8;  // uint4 per 128-dim bf16 row
-  const int per_tensor = H * kVecPerRow;
-  for (int i = threadIdx.x; i < 2 * per_tensor; i += kAppendThreads) {
+#pragma unroll
+  for (int u = 0; u < kMaxVec; ++u) {
+    if (u >= cnt) break;
+    const int i = threadIdx.x + u * kAppendThreads;
     const int which = i / per_tensor;
     const int j = i - which * per_tensor;
     const int h = j / kVecPerRow, e = j - h * kVecPerRow;
     const int64_t bh = (int64_t)b * H + h;
-    const uint4* src = reinterpret_cast<const uint4*>((which ? v_new : k_new) + bh * kHeadDim) + e;
-    uint4* dst = reinterpret_cast<uint4*>((which ? ring_v : ring_k) + (bh * n + slot) * kHeadDim) + e;
-    *dst = *src;
+    reinterpret_cast<uint4*>((which ? ring_v : ring_k) + (bh * n + slot) * kHeadDim)[e] = row[u];
   }
-  if (threadIdx.x == 0) {
-    wp[b] = (slot + 1 == n) ? 0 : slot + 1;
-    fill[b] = min(fill[b] + 1, n);
-    if (slot_out) slot_out[b] = slot;
+  // rows beyond what the registers held (H > 16): plain copy
+  for (int i = threadIdx.x + kMaxVec * kAppendThreads; i < 2 * per_tensor; i += kAppendThreads) {
+    const int which = i / per_tensor;
+    const int j = i - which * per_tensor;
+    const int h = j / kVecPerRow, e = j - h * kVecPerRow;
+    const int64_t bh = (int64_t)b * H + h;
+    reinterpret_cast<uint4*>((which ? ring_v : ring_k) + (bh * n + slot) * kHeadDim)[e] =
+        reinterpret_cast<const uint4*>((which ? v_new : k_new) + bh * kHeadDim)[e];
   }
 }
 

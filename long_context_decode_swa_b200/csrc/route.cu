@@ -18,6 +18,14 @@
 //     tau_k = S1/k - sqrt(delta_k);
 //   * the support size is the largest k with delta_k >= 0 and tau_k < y_(k).
 // Shifting by max x keeps the fp32 sums small (shift invariance of entmax).
+//
+// Top-k and candidates come from one set: the CTAs of a sequence's cluster
+// exchange their maxima, then each sends CTA 0 its candidates (z > max z - 2
+// over the sequence). When the sequence has at least k candidates they hold
+// its k largest scores; otherwise every CTA also sends the rest of its sorted
+// top-32 (warp bitonic networks and a merge tree), which holds its top-k.
+// CTA 0 ranks the union by counting (a bitonic network past 1024 entries),
+// reads the top-k off the front and takes the prefix sums with a block scan.
 #include <cooperative_groups.h>
 
 #include <cmath>
@@ -83,6 +91,7 @@ __device__ __forceinline__ bool ranks_before(float za, int ia, float zb, int ib)
 }
 
 constexpr int kNone = 0x7fffffff;
+constexpr int kRankByCounting = 1024;  // larger unions are sorted with a bitonic network instead
 constexpr int kMaxClusterCtas = 8;  // portable cluster size: up to 8 x 1024 = 8192 blocks
 constexpr int kList = 32;  // sorted candidates kept per warp / per chunk (>= the largest topk)
 
@@ -115,6 +124,13 @@ __device__ __forceinline__ void warp_merge(float& z, int& i, float bz, int bi, i
   }
 #pragma unroll
   for (int j = 16; j > 0; j >>= 1) cmp_xchg(z, i, j, (lane & j) == 0);
+}
+
+// Slots of the compacted union on CTA 0: the next power of two of csize * 1024.
+__host__ __device__ __forceinline__ int route_sort_capacity(int csize) {
+  int p = kRouteThreads * 2;
+  while (p < csize * kRouteThreads * 2) p <<= 1;
+  return p;
 }
 
 struct RouteArgs {
@@ -166,11 +182,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ float lz[kRouteWarps][kList];
   __shared__ int li[kRouteWarps][kList];
-  __shared__ float cl_z[kMaxClusterCtas][kList];  // on CTA 0: every CTA's sorted list
-  __shared__ int cl_i[kMaxClusterCtas][kList];
-  __shared__ float cl_max[kMaxClusterCtas];
-  __shared__ int cl_cnt[kMaxClusterCtas];
+  __shared__ float cl_max[kMaxClusterCtas];  // every CTA's maximum (on every CTA)
+  __shared__ int cl_cnt[kMaxClusterCtas];    // every CTA's candidate count (on every CTA)
+  __shared__ int cl_send[kMaxClusterCtas];   // on CTA 0: entries each CTA sent, lists included
   __shared__ float red[kRouteWarps];
+  __shared__ float scan2[kRouteWarps];
   __shared__ int red_i[kRouteWarps];
   __shared__ int s_cnt;
   __shared__ float s_tau_y, s_xmax;
@@ -180,14 +196,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   const int rank = (int)cluster.block_rank(), b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int region = kRouteThreads * 2;  // blocks per CTA
-  float* cand_z = reinterpret_cast<float*>(smem_raw);  // [csize * region] on CTA 0
+  // on CTA 0: what CTA r sends lands at [r * region, ...) of (cand_z, cand_i); the union
+  // is compacted into (uz, ui), whose size is a power of two for the bitonic sort
+  float* cand_z = reinterpret_cast<float*>(smem_raw);
   int* cand_i = reinterpret_cast<int*>(cand_z + a.csize * region);
-  float* cy = reinterpret_cast<float*>(cand_i + a.csize * region);  // compacted global candidates
-  int* ci = reinterpret_cast<int*>(cy + a.csize * region);
-  float* sy = cand_z;  // rank-ordered candidates (reuses cand_z once compacted)
+  float* uz = reinterpret_cast<float*>(cand_i + a.csize * region);
+  int* ui = reinterpret_cast<int*>(uz + route_sort_capacity(a.csize));
 
   griddep_wait();
   griddep_launch_dependents();
+  if (tid == 0) s_cnt = 1;
   int64_t m64 = a.prefix_len[b];
   // ---- score: warp w covers blocks [64 w, 64 w + 64) of the CTA's region ----
   // The keys are read coalesced, four blocks (512 B) per warp load: octet o = lane / 8
@@ -270,51 +288,81 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     cidx[s2] = cpos[s2] < NB ? cpos[s2] : kNone;
     z[s2] = cpos[s2] < NB ? a.idx_scale * dot[s2] : -INFINITY;
   }
-  // ---- this CTA's maximum and sorted top-32 ----
+  // ---- the sequence's maximum: every CTA of the cluster receives every CTA's ----
   const float wmax = warp_max(fmaxf(z[0], z[1]));
   if (lane == 0) red[warp] = wmax;
-  float za = z[0], zb = z[1];
-  int ia = cidx[0], ib = cidx[1];
-  warp_sort(za, ia, lane);
-  warp_sort(zb, ib, lane);
-  {  // merge the two sorted columns: lane l pairs A[l] with B[31 - l]
-    const float rz = __shfl_sync(0xffffffffu, zb, 31 - lane);
-    const int ri = __shfl_sync(0xffffffffu, ib, 31 - lane);
-    warp_merge(za, ia, rz, ri, lane);
-  }
-  lz[warp][lane] = za;
-  li[warp][lane] = ia;
-  if (tid == 0) s_cnt = 0;
   __syncthreads();
-  float lmax = red[0];
+  float zmax = red[0];
 #pragma unroll
-  for (int w = 1; w < kRouteWarps; ++w) lmax = fmaxf(lmax, red[w]);
-  merge_lists(lz, li, kRouteWarps, warp, lane);
-
-  // ---- publish list, maximum and candidates to CTA 0 ----
-  float* r_cand_z = cluster.map_shared_rank(cand_z, 0);
-  int* r_cand_i = cluster.map_shared_rank(cand_i, 0);
+  for (int w = 1; w < kRouteWarps; ++w) zmax = fmaxf(zmax, red[w]);
+  if (a.csize > 1) {  // uniform over the cluster
+    if (tid < a.csize) cluster.map_shared_rank(cl_max, tid)[rank] = zmax;
+    cluster.sync();
+    for (int r = 0; r < a.csize; ++r) zmax = fmaxf(zmax, cl_max[r]);
+  }
+  // ---- this CTA's candidates z > zmax - 2 go to CTA 0; every CTA learns every count ----
+  const bool cand0 = cidx[0] != kNone && z[0] > zmax - 2.f;
+  const bool cand1 = cidx[1] != kNone && z[1] > zmax - 2.f;
+  const unsigned bal0 = __ballot_sync(0xffffffffu, cand0), bal1 = __ballot_sync(0xffffffffu, cand1);
+  if (lane == 0) red_i[warp] = __popc(bal0) + __popc(bal1);
+  __syncthreads();
+  int n_cand = 0, before = 0;
 #pragma unroll
-  for (int s2 = 0; s2 < 2; ++s2) {
-    if (cidx[s2] != kNone && z[s2] > lmax - 2.f) {
-      const int k = atomicAdd(&s_cnt, 1);
-      r_cand_z[rank * region + k] = z[s2];
-      r_cand_i[rank * region + k] = cidx[s2];
+  for (int w = 0; w < kRouteWarps; ++w) {
+    before += w < warp ? red_i[w] : 0;
+    n_cand += red_i[w];
+  }
+  float* r_cand_z = cluster.map_shared_rank(cand_z, 0) + rank * region;
+  int* r_cand_i = cluster.map_shared_rank(cand_i, 0) + rank * region;
+  {
+    const unsigned lt = (1u << lane) - 1u;
+    if (cand0) {
+      const int k = before + __popc(bal0 & lt);
+      r_cand_z[k] = z[0];
+      r_cand_i[k] = cidx[0];
+    }
+    if (cand1) {
+      const int k = before + __popc(bal0) + __popc(bal1 & lt);
+      r_cand_z[k] = z[1];
+      r_cand_i[k] = cidx[1];
     }
   }
-  if (warp == 0) {
-    cluster.map_shared_rank(&cl_z[0][0], 0)[rank * kList + lane] = lz[0][lane];
-    cluster.map_shared_rank(&cl_i[0][0], 0)[rank * kList + lane] = li[0][lane];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    cluster.map_shared_rank(cl_max, 0)[rank] = lmax;
-    cluster.map_shared_rank(cl_cnt, 0)[rank] = s_cnt;
-  }
-  if (a.csize > 1)  // uniform over the cluster
+  if (tid < a.csize) cluster.map_shared_rank(cl_cnt, tid)[rank] = n_cand;
+  if (a.csize > 1)
     cluster.sync();
   else
     __syncthreads();
+  int total = 0;
+  for (int r = 0; r < a.csize; ++r) total += cl_cnt[r];
+  // ---- fewer than topk candidates in all: each CTA adds the rest of its sorted top-32 ----
+  // (the global top-k is within the CTAs' top-k; a CTA's candidates are its first n_cand)
+  const bool with_lists = total < a.topk;  // uniform over the cluster
+  if (with_lists) {
+    float za = z[0], zb = z[1];
+    int ia = cidx[0], ib = cidx[1];
+    warp_sort(za, ia, lane);
+    warp_sort(zb, ib, lane);
+    {  // merge the two sorted columns: lane l pairs A[l] with B[31 - l]
+      const float rz = __shfl_sync(0xffffffffu, zb, 31 - lane);
+      const int ri = __shfl_sync(0xffffffffu, ib, 31 - lane);
+      warp_merge(za, ia, rz, ri, lane);
+    }
+    lz[warp][lane] = za;
+    li[warp][lane] = ia;
+    __syncthreads();
+    merge_lists(lz, li, kRouteWarps, warp, lane);
+    // the valid entries are a prefix of the sorted list (missing blocks carry kNone, -inf)
+    const int n_valid = __popc(__ballot_sync(0xffffffffu, li[0][lane] != kNone));
+    if (warp == 0 && lane >= n_cand && lane < n_valid) {
+      r_cand_z[lane] = lz[0][lane];
+      r_cand_i[lane] = li[0][lane];
+    }
+    if (tid == 0) cluster.map_shared_rank(cl_send, 0)[rank] = max(n_valid, n_cand);
+    if (a.csize > 1)
+      cluster.sync();
+    else
+      __syncthreads();
+  }
 
   if (rank != 0) {
     if (a.probs == nullptr) return;
@@ -333,53 +381,114 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     return;
   }
 
-  // ---- CTA 0: merge the lists, gather the global candidates, exact threshold ----
-  float zmax = cl_max[0];
-  for (int r = 1; r < a.csize; ++r) zmax = fmaxf(zmax, cl_max[r]);
+  // ---- CTA 0: the union U of what the CTAs sent, in rank order ----
+  int n_u = 0;
+  for (int r = 0; r < a.csize; ++r) n_u += with_lists ? cl_send[r] : cl_cnt[r];
   const float xmax = 0.5f * zmax;
-  if (warp < a.csize) {
-    lz[warp][lane] = cl_z[warp][lane];
-    li[warp][lane] = cl_i[warp][lane];
-  }
-  if (tid == 0) s_cnt = 0;
-  __syncthreads();
-  merge_lists(lz, li, a.csize, warp, lane);
-  for (int r = 0; r < a.csize; ++r) {
-    const int cnt = cl_cnt[r];
-    for (int k = tid; k < cnt; k += kRouteThreads) {
-      const float y = fmaf(cand_z[r * region + k], 0.5f, -xmax);
-      if (y > -1.f) {
-        const int slot = atomicAdd(&s_cnt, 1);
-        cy[slot] = y;
-        ci[slot] = cand_i[r * region + k];
+  {  // compact U into (uz, ui)
+    int off = 0;
+    for (int r = 0; r < a.csize; ++r) {
+      const int cnt = with_lists ? cl_send[r] : cl_cnt[r];
+      for (int k = tid; k < cnt; k += kRouteThreads) {
+        uz[off + k] = cand_z[r * region + k];
+        ui[off + k] = cand_i[r * region + k];
       }
+      off += cnt;
     }
   }
   __syncthreads();
-  const int K = s_cnt;
-  for (int i = tid; i < K; i += kRouteThreads) {
-    const float yi = cy[i];
-    const int ii = ci[i];
-    int r = 0;
-    for (int j = 0; j < K; ++j) r += ranks_before(cy[j], ci[j], yi, ii) ? 1 : 0;
-    sy[r] = yi;
+  const float* oz;  // U sorted: larger score first, ties to the smaller block
+  const int* oi;
+  if (n_u <= kRankByCounting) {
+    for (int i = tid; i < n_u; i += kRouteThreads) {
+      const float zi = uz[i];
+      const int ii = ui[i];
+      int r = 0;
+      for (int j = 0; j < n_u; ++j) r += ranks_before(uz[j], ui[j], zi, ii) ? 1 : 0;
+      cand_z[r] = zi;
+      cand_i[r] = ii;
+    }
+    oz = cand_z;
+    oi = cand_i;
+  } else {  // bitonic sort of U in place, padded to a power of two
+    int np2 = 1;
+    while (np2 < n_u) np2 <<= 1;
+    for (int i = n_u + tid; i < np2; i += kRouteThreads) {
+      uz[i] = -INFINITY;
+      ui[i] = kNone;
+    }
+    for (int k = 2; k <= np2; k <<= 1)
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        __syncthreads();
+        for (int i = tid; i < np2; i += kRouteThreads) {
+          const int p = i ^ j;
+          if (p > i) {
+            const bool first_better = ranks_before(uz[i], ui[i], uz[p], ui[p]);
+            // ascending blocks of the network put the better element first
+            if (first_better != ((i & k) == 0)) {
+              const float tz = uz[i];
+              uz[i] = uz[p];
+              uz[p] = tz;
+              const int ti = ui[i];
+              ui[i] = ui[p];
+              ui[p] = ti;
+            }
+          }
+        }
+      }
+    oz = uz;
+    oi = ui;
   }
   __syncthreads();
-  float* tau_r = reinterpret_cast<float*>(ci);  // tau_k by rank k - 1 (ci is free after the ranking)
+
+  // ---- exact threshold over the candidates y = z/2 - max(z/2) > -1, a prefix of U ----
+  for (int r = tid; r < n_u; r += kRouteThreads) {
+    const bool in = fmaf(oz[r], 0.5f, -xmax) > -1.f;
+    const bool next_in = r + 1 < n_u && fmaf(oz[r + 1], 0.5f, -xmax) > -1.f;
+    if (in && !next_in) s_cnt = r + 1;
+  }
+  __syncthreads();
+  const int K = s_cnt;  // >= 1: the maximum itself has y = 0
+  // prefix sums of y and y^2 in rank order: thread t takes a contiguous run of ranks
+  const int per = (K + kRouteThreads - 1) / kRouteThreads;
+  const int r0 = min(K, tid * per), r1 = min(K, r0 + per);
+  float s1 = 0.f, s2 = 0.f;
+  for (int r = r0; r < r1; ++r) {
+    const float y = fmaf(oz[r], 0.5f, -xmax);
+    s1 += y;
+    s2 = fmaf(y, y, s2);
+  }
+  float i1 = s1, i2 = s2;  // inclusive scan over the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float t1 = __shfl_up_sync(0xffffffffu, i1, o), t2 = __shfl_up_sync(0xffffffffu, i2, o);
+    if (lane >= o) {
+      i1 += t1;
+      i2 += t2;
+    }
+  }
+  if (lane == 31) {
+    red[warp] = i1;
+    scan2[warp] = i2;
+  }
+  __syncthreads();
+  float e1 = i1 - s1, e2 = i2 - s2;  // exclusive prefix of this thread's run
+  for (int w = 0; w < warp; ++w) {
+    e1 += red[w];
+    e2 += scan2[w];
+  }
+  float* tau_r = uz == oz ? reinterpret_cast<float*>(cand_z) : uz;  // tau_k by rank k - 1
   int best = 0;
-  for (int r = tid; r < K; r += kRouteThreads) {
-    float s1 = 0.f, s2 = 0.f;
-    for (int j = 0; j <= r; ++j) {
-      const float y = sy[j];
-      s1 += y;
-      s2 = fmaf(y, y, s2);
-    }
+  for (int r = r0; r < r1; ++r) {
+    const float y = fmaf(oz[r], 0.5f, -xmax);
+    e1 += y;
+    e2 = fmaf(y, y, e2);
     const float k = (float)(r + 1);
-    const float mean = s1 / k;
-    const float delta = (1.f - (s2 - s1 * mean)) / k;
+    const float mean = e1 / k;
+    const float delta = (1.f - (e2 - e1 * mean)) / k;
     const float t = mean - sqrtf(fmaxf(delta, 0.f));
     tau_r[r] = t;
-    if (delta >= 0.f && t < sy[r]) best = r + 1;
+    if (delta >= 0.f && t < y) best = r + 1;
   }
   best = __reduce_max_sync(0xffffffffu, (unsigned)best);
   if (lane == 0) red_i[warp] = best;
@@ -388,14 +497,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   for (int w = 0; w < kRouteWarps; ++w) best = max(best, red_i[w]);
   const float tau_y = best > 0 ? tau_r[best - 1] : 0.f;
   if (a.tau && tid == 0) a.tau[b] = tau_y + xmax;
-  if (warp == 0 && lane < a.topk) {
-    const int64_t o = (int64_t)b * a.topk + lane;
-    const int bi = li[0][lane];
+  if (tid < a.topk) {
+    const int64_t o = (int64_t)b * a.topk + tid;
+    const int bi = tid < n_u ? oi[tid] : kNone;
     if (bi == kNone) {
       a.blk_idx[o] = -1;
       a.blk_logp[o] = -INFINITY;
     } else {
-      const float d = fmaf(lz[0][lane], 0.5f, -xmax) - tau_y;
+      const float d = fmaf(oz[tid], 0.5f, -xmax) - tau_y;
       const float pr = d > 0.f ? d * d : 0.f;
       a.blk_idx[o] = bi;
       a.blk_logp[o] = pr > 0.f ? logf(pr) : -INFINITY;
@@ -410,12 +519,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       cluster.sync();
     else
       __syncthreads();
-    for (int s2 = 0; s2 < 2; ++s2) {
-      const int c = cpos[s2];
+    for (int s2i = 0; s2i < 2; ++s2i) {
+      const int c = cpos[s2i];
       if (c < a.nb_cap) {
         float pr = 0.f;
         if (c < NB) {
-          const float r = fmaf(z[s2], 0.5f, -xmax) - tau_y;
+          const float r = fmaf(z[s2i], 0.5f, -xmax) - tau_y;
           pr = r > 0.f ? r * r : 0.f;
         }
         a.probs[(int64_t)b * a.nb_cap + c] = pr;
@@ -457,9 +566,11 @@ cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kb
   a.probs = probs;
   a.tau = tau;
   a.status = status;
-  const size_t smem = (size_t)a.csize * kRouteThreads * 2 * 16;
+  const size_t smem = (size_t)a.csize * kRouteThreads * 2 * 8 + (size_t)route_sort_capacity(a.csize) * 8;
   static unsigned long long done = 0;
-  cudaError_t e = ensure_smem_limit(route_kernel, (size_t)kMaxClusterCtas * kRouteThreads * 2 * 16, &done);
+  cudaError_t e = ensure_smem_limit(
+      route_kernel, (size_t)kMaxClusterCtas * kRouteThreads * 2 * 8 + (size_t)route_sort_capacity(kMaxClusterCtas) * 8,
+      &done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
