@@ -156,6 +156,13 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 2^x on the MUFU unit (the hardware's approximate base-2 exponential, flush-to-zero).
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -530,15 +537,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         uint32_t rr[32];
         tmem_ld32(s_cols + (uint32_t)ch * 32u, rr);
         tmem_wait_ld();
+        float m0 = tmax, m1 = -INFINITY;  // two chains of three-input maxima
         if (full) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(rr[e]));
+          for (int e = 0; e < 32; e += 4) {
+            m0 = max3(m0, __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
+            m1 = max3(m1, __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
+          }
         } else {
           float xv[32];
           mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, xv[e]);
+          for (int e = 0; e < 32; e += 4) {
+            m0 = max3(m0, xv[e], xv[e + 1]);
+            m1 = max3(m1, xv[e + 2], xv[e + 3]);
+          }
         }
+        tmax = fmaxf(m0, m1);
       }
       if (full) tmax *= a.qk_scale_log2;
       const bool rescale = tmax > m_used + kLazyRescaleLog2;
@@ -565,7 +580,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       const float m_sub = m_used == -INFINITY ? 0.f : m_used;  // a row with nothing visible yet: exp2(-inf) = 0
       // pass 2: P = 2^(s - m) as bf16 pairs, written over the first 64 columns of this tile's S
-      float lsum = 0.f, lusum = 0.f;
+      // (pairs of columns go through paired f32 FMA / add instructions)
+      float2 lsum = make_float2(0.f, 0.f), lusum = make_float2(0.f, 0.f);
+      const float2 neg_m = make_float2(-m_sub, -m_sub);
+      const float2 scale2 = make_float2(a.qk_scale_log2, a.qk_scale_log2);
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t rr[32];
@@ -575,30 +593,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (full) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(rr[2 * e]), a.qk_scale_log2, -m_sub));
-            const float p1 = ex2(fmaf(__uint_as_float(rr[2 * e + 1]), a.qk_scale_log2, -m_sub));
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(rr[2 * e]), __uint_as_float(rr[2 * e + 1])),
+                                         scale2, neg_m);
+            const float2 p2 = make_float2(ex2(x2.x), ex2(x2.y));
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p2.x, p2.y);
             pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
-            lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
-            lusum += p0 + p1;
+            lsum = __fadd2_rn(lsum, make_float2(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xffff0000u)));
+            lusum = __fadd2_rn(lusum, p2);
           }
         } else {
           float xv[32];
           mask_chunk(c, kind, start, i, ch * 32, a.qk_scale_log2, rr, xv);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(xv[2 * e] - m_sub);
-            const float p1 = ex2(xv[2 * e + 1] - m_sub);
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            const float2 x2 = __fadd2_rn(make_float2(xv[2 * e], xv[2 * e + 1]), neg_m);
+            const float2 p2 = make_float2(ex2(x2.x), ex2(x2.y));
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p2.x, p2.y);
             pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
-            lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
-            lusum += p0 + p1;
+            lsum = __fadd2_rn(lsum, make_float2(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xffff0000u)));
+            lusum = __fadd2_rn(lusum, p2);
           }
         }
         tmem_st16(s_cols + (uint32_t)ch * 16u, pk);
       }
-      l += lsum;
-      lu += lusum;
+      l += lsum.x + lsum.y;
+      lu += lusum.x + lusum.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[x]);
