@@ -64,6 +64,15 @@ def _L():
             lib.oracle_entmax15.restype = Dbl
             lib.oracle_route.argtypes = [I, I64, I, I, P, P, P, Dbl, I, P, P, P, P, P]
             lib.oracle_srswa_decode.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, I, P, P, P, P, Dbl, P, P]
+            lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_to_double.restype = Dbl
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode_array.argtypes = [I64, P, P]
+            lib.oracle_quantize_prefix.argtypes = [I, I, I, I64, I, P, P, P, P]
+            lib.oracle_rswa_decode_fp8.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, P, P, Dbl, P, P]
+            lib.oracle_srswa_decode_fp8.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, I, P, P, P, P, Dbl,
+                                                    P, P]
             _lib = lib
     return _lib
 
@@ -216,6 +225,86 @@ def srswa_decode(q, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, f
     _L().oracle_srswa_decode(B, H, D, n, cap, blk, _p(q), _p(pk), _p(pv), _p(prefix_len), _p(blk_idx),
                              _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp), _p(fill), float(scale),
                              _p(out), _p(lse))
+    return out, lse
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) prefix
+
+def e4m3_to_double(codes) -> np.ndarray:
+    """Values of E4M3 codes (uint8 array), from the format's definition (NaN for 0x7f / 0xff)."""
+    table = np.array([_L().oracle_e4m3_to_double(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, np.uint8)]
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest E4M3 codes of fp32 values (ties to even, saturating at 448, NaN -> 0x7f)."""
+    x = np.ascontiguousarray(x, np.float32)
+    out = np.zeros(x.shape, np.uint8)
+    _L().oracle_e4m3_encode_array(x.size, _p(x), _p(out))
+    return out
+
+
+def quantize_prefix(x, prefix_len, blk: int = BLOCK):
+    """E4M3 codes [B][H][cap][D] (uint8) and fp32 block scales [B][H][ceil(cap/blk)] of a bf16 prefix.
+
+    Blocks past prefix_len are left at zero (codes) / zero (scales) here."""
+    x = _u16(x, 4, "x")
+    prefix_len = _i32(prefix_len, "prefix_len")
+    B, H, cap, D = x.shape
+    codes = np.zeros((B, H, cap, D), np.uint8)
+    scales = np.zeros((B, H, (cap + blk - 1) // blk), np.float32)
+    _L().oracle_quantize_prefix(B, H, D, cap, blk, _p(x), _p(prefix_len), _p(codes), _p(scales))
+    return codes, scales
+
+
+def _u8(a, ndim: int, name: str) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint8 or a.ndim != ndim:
+        raise ValueError(f"{name}: expected uint8 with {ndim} dims, got {a.dtype} {a.shape}")
+    return a
+
+
+def rswa_decode_fp8(q, pk8, pv8, kscale, vscale, prefix_len, ring_k, ring_v, wp, fill, scale, blk: int = BLOCK):
+    """R-SWA decode over an E4M3 prefix (code * block scale). Returns (out fp64 [B][H][D], lse fp64 [B][H])."""
+    q = _u16(q, 3, "q")
+    pk8, pv8 = _u8(pk8, 4, "pk8"), _u8(pv8, 4, "pv8")
+    kscale = np.ascontiguousarray(kscale, np.float32)
+    vscale = np.ascontiguousarray(vscale, np.float32)
+    ring_k = _u16(ring_k, 4, "ring_k")
+    ring_v = _u16(ring_v, 4, "ring_v")
+    prefix_len, wp, fill = _i32(prefix_len, "prefix_len"), _i32(wp, "wp"), _i32(fill, "fill")
+    B, H, D = q.shape
+    cap = pk8.shape[2]
+    n = ring_k.shape[2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _L().oracle_rswa_decode_fp8(B, H, D, n, cap, blk, _p(q), _p(pk8), _p(pv8), _p(kscale), _p(vscale),
+                                _p(prefix_len), _p(ring_k), _p(ring_v), _p(wp), _p(fill), float(scale), _p(out),
+                                _p(lse))
+    return out, lse
+
+
+def srswa_decode_fp8(q, pk8, pv8, kscale, vscale, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, scale,
+                     blk: int = BLOCK):
+    """SR-SWA gathered-block decode over an E4M3 prefix. Returns (out fp64 [B][H][D], lse fp64 [B][H])."""
+    q = _u16(q, 3, "q")
+    pk8, pv8 = _u8(pk8, 4, "pk8"), _u8(pv8, 4, "pv8")
+    kscale = np.ascontiguousarray(kscale, np.float32)
+    vscale = np.ascontiguousarray(vscale, np.float32)
+    ring_k = _u16(ring_k, 4, "ring_k")
+    ring_v = _u16(ring_v, 4, "ring_v")
+    prefix_len, wp, fill = _i32(prefix_len, "prefix_len"), _i32(wp, "wp"), _i32(fill, "fill")
+    blk_idx = _i32(blk_idx, "blk_idx")
+    blk_logp = np.ascontiguousarray(blk_logp, np.float64)
+    B, H, D = q.shape
+    topk = blk_idx.shape[1]
+    cap = pk8.shape[2]
+    n = ring_k.shape[2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _L().oracle_srswa_decode_fp8(B, H, D, n, cap, blk, _p(q), _p(pk8), _p(pv8), _p(kscale), _p(vscale),
+                                 _p(prefix_len), _p(blk_idx), _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp),
+                                 _p(fill), float(scale), _p(out), _p(lse))
     return out, lse
 
 

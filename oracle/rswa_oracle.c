@@ -81,24 +81,38 @@ int oracle_get_threads(void) {
  * slot for SR-SWA's log-probability term.
  */
 typedef struct {
-  const uint16_t** krow;
+  const uint16_t** krow;  /* bf16 rows, or NULL when the key is stored as e4m3 codes */
   const uint16_t** vrow;
+  const uint8_t** k8;     /* e4m3 rows and their block scales (FP8 prefix) */
+  const uint8_t** v8;
+  double* kscale;
+  double* vscale;
   double* bias;
   double* s;
   int64_t count;
 } keylist;
 
+static void* alloc_keys(size_t elem, int64_t max_keys) { return malloc(elem * (size_t)(max_keys > 0 ? max_keys : 1)); }
+
 static void keylist_init(keylist* L, int64_t max_keys) {
-  L->krow = (const uint16_t**)malloc(sizeof(*L->krow) * (size_t)(max_keys > 0 ? max_keys : 1));
-  L->vrow = (const uint16_t**)malloc(sizeof(*L->vrow) * (size_t)(max_keys > 0 ? max_keys : 1));
-  L->bias = (double*)malloc(sizeof(double) * (size_t)(max_keys > 0 ? max_keys : 1));
-  L->s = (double*)malloc(sizeof(double) * (size_t)(max_keys > 0 ? max_keys : 1));
+  L->krow = (const uint16_t**)alloc_keys(sizeof(*L->krow), max_keys);
+  L->vrow = (const uint16_t**)alloc_keys(sizeof(*L->vrow), max_keys);
+  L->k8 = (const uint8_t**)alloc_keys(sizeof(*L->k8), max_keys);
+  L->v8 = (const uint8_t**)alloc_keys(sizeof(*L->v8), max_keys);
+  L->kscale = (double*)alloc_keys(sizeof(double), max_keys);
+  L->vscale = (double*)alloc_keys(sizeof(double), max_keys);
+  L->bias = (double*)alloc_keys(sizeof(double), max_keys);
+  L->s = (double*)alloc_keys(sizeof(double), max_keys);
   L->count = 0;
 }
 
 static void keylist_free(keylist* L) {
   free((void*)L->krow);
   free((void*)L->vrow);
+  free((void*)L->k8);
+  free((void*)L->v8);
+  free(L->kscale);
+  free(L->vscale);
   free(L->bias);
   free(L->s);
 }
@@ -106,8 +120,33 @@ static void keylist_free(keylist* L) {
 static void keylist_push(keylist* L, const uint16_t* k, const uint16_t* v, double bias) {
   L->krow[L->count] = k;
   L->vrow[L->count] = v;
+  L->k8[L->count] = NULL;
+  L->v8[L->count] = NULL;
   L->bias[L->count] = bias;
   L->count++;
+}
+
+double oracle_e4m3_to_double(uint8_t c);
+
+static void keylist_push8(keylist* L, const uint8_t* k, const uint8_t* v, double kscale, double vscale,
+                          double bias) {
+  L->krow[L->count] = NULL;
+  L->vrow[L->count] = NULL;
+  L->k8[L->count] = k;
+  L->v8[L->count] = v;
+  L->kscale[L->count] = kscale;
+  L->vscale[L->count] = vscale;
+  L->bias[L->count] = bias;
+  L->count++;
+}
+
+/* element d of key / value j, widened to double (an e4m3 code times its block scale) */
+static double key_at(const keylist* L, int64_t j, int d) {
+  return L->krow[j] ? bf16_to_double(L->krow[j][d]) : oracle_e4m3_to_double(L->k8[j][d]) * L->kscale[j];
+}
+
+static double val_at(const keylist* L, int64_t j, int d) {
+  return L->vrow[j] ? bf16_to_double(L->vrow[j][d]) : oracle_e4m3_to_double(L->v8[j][d]) * L->vscale[j];
 }
 
 static void attend(const keylist* L, const uint16_t* q, int D, double scale, double* out, double* lse) {
@@ -121,7 +160,7 @@ static void attend(const keylist* L, const uint16_t* q, int D, double scale, dou
   double M = -INFINITY;
   for (int64_t j = 0; j < L->count; ++j) {
     double dot = 0.0;
-    for (int d = 0; d < D; ++d) dot += qd[d] * bf16_to_double(L->krow[j][d]);
+    for (int d = 0; d < D; ++d) dot += qd[d] * key_at(L, j, d);
     L->s[j] = scale * dot + L->bias[j];
     if (L->s[j] > M) M = L->s[j];
   }
@@ -133,7 +172,7 @@ static void attend(const keylist* L, const uint16_t* q, int D, double scale, dou
   for (int64_t j = 0; j < L->count; ++j) {
     double w = exp(L->s[j] - M);
     denom += w;
-    for (int d = 0; d < D; ++d) out[d] += w * bf16_to_double(L->vrow[j][d]);
+    for (int d = 0; d < D; ++d) out[d] += w * val_at(L, j, d);
   }
   for (int d = 0; d < D; ++d) out[d] /= denom;
   *lse = M + log(denom);
@@ -488,4 +527,181 @@ void oracle_srswa_decode(int B, int H, int D, int n, int64_t cap, int blk, const
     }
     keylist_free(&L);
   }
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 (e4m3) prefix cache                                             */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The pages list quantised KV-cache compression as the next step after the
+ * window itself (Tutorial, "KV缓存压缩" under future directions) without fixing
+ * a format. Reading adopted: the prefix K and V are stored as OCP FP8 E4M3
+ * codes (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0
+ * holds the subnormals m/8 * 2^-6; S.1111.111 is NaN; no infinities; largest
+ * finite value 448), one fp32 scale per (sequence, head, 32-token block) for K
+ * and one for V. A stored element is code value * scale. The ring stays bf16.
+ */
+
+/* Value of an E4M3 code, from the format's definition. Pinned by: the format's
+ * landmarks (0x38 = 1, 0x7e = 448, 0x08 = 2^-6, 0x01 = 2^-9, 0x7f NaN) and by
+ * exact round trips through the encoder. */
+double oracle_e4m3_to_double(uint8_t c) {
+  int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m / 8.0, -6);
+  else
+    v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* Round half to even of a non-negative double holding an exact value. */
+static double round_half_even(double x) {
+  double f = floor(x), r = x - f;
+  if (r > 0.5) return f + 1.0;
+  if (r < 0.5) return f;
+  return fmod(f, 2.0) == 0.0 ? f : f + 1.0;
+}
+
+/* Nearest E4M3 code to x, ties to the even mantissa, magnitudes past 448
+ * clamped to 448 (saturating), NaN to 0x7f. The grid spacing in the binade
+ * [2^e, 2^(e+1)) is 2^(e-3) (2^-9 below 2^-6), so x / spacing is rounded to an
+ * integer; a result of 16 spacings is the next binade's first value.
+ * Pinned by: an exhaustive nearest-value search over the 127 non-negative
+ * finite codes (tests), round trips of every finite code, and the
+ * saturation and tie cases. */
+uint8_t oracle_e4m3_encode(float x) {
+  if (isnan(x)) return 0x7f;
+  int sign = signbit(x) ? 1 : 0;
+  double a = fabs((double)x);
+  uint8_t code;
+  if (a >= 448.0) {
+    code = 0x7e;
+  } else if (a < ldexp(1.0, -6)) {
+    double r = round_half_even(a / ldexp(1.0, -9)); /* 0..8 spacings of 2^-9 */
+    code = (uint8_t)r;                               /* 8 -> 0x08 = 2^-6, the first normal */
+  } else {
+    int e;
+    frexp(a, &e);
+    e -= 1; /* a in [2^e, 2^(e+1)) */
+    double r = round_half_even(a / ldexp(1.0, e - 3)); /* 8..16 spacings */
+    if (r >= 16.0) {
+      e += 1;
+      r = 8.0;
+    }
+    if (e > 8) { /* rounding past 448 (only from [448, 464) which is caught above) */
+      code = 0x7e;
+    } else {
+      code = (uint8_t)(((e + 7) << 3) | ((int)r - 8));
+      if (code == 0x7f) code = 0x7e;
+    }
+  }
+  return (uint8_t)(code | (sign << 7));
+}
+
+/*
+ * Quantises the prefix K and V: for each (sequence, head, block c) holding
+ * valid rows [32c, min(m, 32c + 32)), amax = the largest |x| over those rows
+ * and all D dims, scale = amax / 448 (in fp32; 1 when amax = 0), code =
+ * e4m3(x / scale) with the quotient in fp32. Rows of the block past m get
+ * code 0; blocks past m are not touched. codes [B][H][cap][D], scales
+ * [B][H][ceil(cap / 32)]. The fp32 steps are the stated reading (a quantised
+ * code is an integer decided by floating point; both sides take it in fp32).
+ */
+void oracle_quantize_prefix(int B, int H, int D, int64_t cap, int blk, const uint16_t* x, const int32_t* prefix_len,
+                            uint8_t* codes, float* scales) {
+  int64_t nb_cap = (cap + blk - 1) / blk;
+  for (int b = 0; b < B; ++b) {
+    int64_t m = prefix_len[b];
+    for (int h = 0; h < H; ++h) {
+      int64_t bh = (int64_t)b * H + h;
+      for (int64_t c = 0; c * blk < m; ++c) {
+        int64_t t0 = c * blk, t1 = t0 + blk < m ? t0 + blk : m;
+        float amax = 0.0f;
+        for (int64_t t = t0; t < t1; ++t)
+          for (int d = 0; d < D; ++d) {
+            float v = fabsf((float)bf16_to_double(x[(bh * cap + t) * D + d]));
+            if (v > amax) amax = v;
+          }
+        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scales[bh * nb_cap + c] = sc;
+        for (int64_t t = t0; t < t0 + blk && t < cap; ++t)
+          for (int d = 0; d < D; ++d) {
+            int64_t off = (bh * cap + t) * D + d;
+            codes[off] = t < t1 ? oracle_e4m3_encode((float)bf16_to_double(x[off]) / sc) : 0;
+          }
+      }
+    }
+  }
+}
+
+/*
+ * R-SWA decode over an FP8 prefix: oracle_rswa_decode with every prefix
+ * element read as code value * block scale (exact in double).
+ * Pinned by: data on the E4M3 grid with unit scales reproduces the bf16 decode
+ * of the same values, plus the bf16 decode's own pins.
+ */
+void oracle_rswa_decode_fp8(int B, int H, int D, int n, int64_t cap, int blk, const uint16_t* q, const uint8_t* pk8,
+                            const uint8_t* pv8, const float* kscale, const float* vscale, const int32_t* prefix_len,
+                            const uint16_t* ring_k, const uint16_t* ring_v, const int32_t* wp, const int32_t* fill,
+                            double scale, double* out, double* lse) {
+  int64_t BH = (int64_t)B * H, nb_cap = (cap + blk - 1) / blk;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, cap + n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+      int64_t b = bh / H;
+      L.count = 0;
+      for (int64_t j = 0; j < prefix_len[b]; ++j) {
+        int64_t off = (bh * cap + j) * D, sc = bh * nb_cap + j / blk;
+        keylist_push8(&L, pk8 + off, pv8 + off, kscale[sc], vscale[sc], 0.0);
+      }
+      push_ring(&L, ring_k, ring_v, bh, n, D, wp[b], fill[b]);
+      attend(&L, q + bh * D, D, scale, out + bh * D, lse + bh);
+    }
+    keylist_free(&L);
+  }
+}
+
+/* SR-SWA gathered decode over an FP8 prefix: oracle_srswa_decode with the
+ * routed blocks' elements read as code value * block scale. */
+void oracle_srswa_decode_fp8(int B, int H, int D, int n, int64_t cap, int blk, const uint16_t* q, const uint8_t* pk8,
+                             const uint8_t* pv8, const float* kscale, const float* vscale, const int32_t* prefix_len,
+                             const int32_t* blk_idx, const double* blk_logp, int topk, const uint16_t* ring_k,
+                             const uint16_t* ring_v, const int32_t* wp, const int32_t* fill, double scale, double* out,
+                             double* lse) {
+  int64_t BH = (int64_t)B * H, nb_cap = (cap + blk - 1) / blk;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, (int64_t)topk * blk + n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+      int64_t b = bh / H;
+      int64_t m = prefix_len[b];
+      L.count = 0;
+      for (int k = 0; k < topk; ++k) {
+        int64_t c = blk_idx[b * topk + k];
+        double bias = blk_logp[b * topk + k];
+        if (c < 0 || bias == -INFINITY) continue;
+        int64_t t1 = (c + 1) * blk < m ? (c + 1) * blk : m;
+        for (int64_t t = c * blk; t < t1; ++t) {
+          int64_t off = (bh * cap + t) * D, sc = bh * nb_cap + c;
+          keylist_push8(&L, pk8 + off, pv8 + off, kscale[sc], vscale[sc], bias);
+        }
+      }
+      push_ring(&L, ring_k, ring_v, bh, n, D, wp[b], fill[b]);
+      attend(&L, q + bh * D, D, scale, out + bh * D, lse + bh);
+    }
+    keylist_free(&L);
+  }
+}
+
+/* Element-wise oracle_e4m3_encode over an array (for the tests). */
+void oracle_e4m3_encode_array(int64_t count, const float* x, uint8_t* out) {
+  for (int64_t i = 0; i < count; ++i) out[i] = oracle_e4m3_encode(x[i]);
 }
