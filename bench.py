@@ -6,6 +6,8 @@
 A step is one decode step of the whole batch through the C ABI:
   configs 1, 2 (R-SWA):   rswa_append + rswa_decode
   configs 4, 5 (SR-SWA):  rswa_append + srswa_route + srswa_decode
+  configs 6, 7:           configs 2 and 4 over an FP8 (E4M3) prefix, quantised
+                          once before timing (rswa_decode_fp8 / srswa_decode_fp8)
 (the router's block index keys are pooled once per prefix, before timing).
 The default workload is the batched R-SWA decode: 512 sequences, 16 heads,
 head_dim 128, a 10-page prefix (2560 visual + 32 prompt tokens) and a full
@@ -77,6 +79,11 @@ def workload(cfg: int) -> dict:
         return dict(kind="srswa", B=16, H=16, D=128, n=128, plen=plen, cap=102400, wp0=None,
                     name="SR-SWA long-horizon decode, 16 sequences, 16 heads, head_dim 128, ragged histories "
                          "8192-102400 tokens (log-uniform pages x 256), top-16 blocks + 128-slot ring")
+    if cfg in (6, 7):  # the batched R-SWA and the 32K-history SR-SWA workloads over an FP8 (E4M3) prefix
+        w = workload(2 if cfg == 6 else 4)
+        w["fp8"] = True
+        w["name"] += "; prefix K/V stored as E4M3 codes with per-(sequence, head, 32-token block) f32 scales"
+        return w
     raise SystemExit(f"config {cfg} is not a decode benchmark here")
 
 
@@ -92,18 +99,22 @@ def algorithmic_bytes(w: dict, blk_rows=None) -> dict:
     """Bytes the method must move per attention launch (and per route launch).
 
     R-SWA: per (b, h): (prefix_len + ring fill) K and V rows of 256 B each, the
-    query (256 B), the f32 output (512 B) and lse (4 B).
+    query (256 B), the f32 output (512 B) and lse (4 B). With an FP8 prefix a
+    prefix row is 128 B of codes each for K and V, plus two f32 scales per block.
     SR-SWA: the same with the routed blocks' valid rows in place of the prefix.
     Router: per sequence the block keys (128 B per block), q_idx (128 B) and the
     top-k outputs (8 B each).
     """
     H, n = w["H"], w["n"]
     per_q = 256 + 512 + 4
+    # an FP8 prefix row is 128 + 128 B of codes, plus 8 B of scales per 32-row block
+    row = 256 if w.get("fp8") else 512
     if w["kind"] == "rswa":
-        attn = sum((m + n) * 512 + per_q for m in w["plen"]) * H
+        attn = sum(m * row + (8 * ((m + 31) // 32) if w.get("fp8") else 0) + n * 512 + per_q
+                   for m in w["plen"]) * H
         return dict(attn=attn, route=0)
     rows = blk_rows if blk_rows is not None else [16 * 32] * w["B"]
-    attn = sum((r + n) * 512 + per_q for r in rows) * H
+    attn = sum(r * row + (8 * ((r + 31) // 32) if w.get("fp8") else 0) + n * 512 + per_q for r in rows) * H
     route = sum(((m + 31) // 32) * 128 + 128 + 16 * 8 for m in w["plen"])
     return dict(attn=attn, route=route)
 
@@ -264,6 +275,11 @@ class Problem:
         self.out = torch.empty((B, H, D), dtype=torch.float32, device="cuda")
         self.lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
         self.sparse = w["kind"] == "srswa"
+        self.fp8 = bool(w.get("fp8"))
+        if self.fp8:  # the stored cache: the bf16 prefix quantised once, by the library
+            self.k8, self.v8, self.ks, self.vs = rswa.fp8_prefix_buffers(self.c.pk)
+            rswa.rswa_quantize_prefix(self.c.pk, self.c.pv, self.c.prefix_len, self.k8, self.v8, self.ks, self.vs,
+                                      status=self.ws)
         if self.sparse:
             n_dirs = 32
             pl = synth.plant_router_keys(w["plen"], w["cap"], n_dirs=n_dirs, seed=seed + 1, device="cuda")
@@ -289,8 +305,12 @@ class Problem:
         if not self.sparse:
             if ev is not None:
                 ev[0].record()
-            r.rswa_decode(q, c.pk, c.pv, c.prefix_len, c.ring_k, c.ring_v, c.wp, c.fill, self.out, self.ws,
-                          lse=self.lse, scale=c.scale)
+            if self.fp8:
+                r.rswa_decode_fp8(q, self.k8, self.v8, self.ks, self.vs, c.prefix_len, c.ring_k, c.ring_v, c.wp,
+                                  c.fill, self.out, self.ws, lse=self.lse, scale=c.scale)
+            else:
+                r.rswa_decode(q, c.pk, c.pv, c.prefix_len, c.ring_k, c.ring_v, c.wp, c.fill, self.out, self.ws,
+                              lse=self.lse, scale=c.scale)
             if ev is not None:
                 ev[1].record()
             return 2
@@ -301,8 +321,12 @@ class Problem:
         if ev is not None:
             ev[3].record()
             ev[0].record()
-        r.srswa_decode(q, c.pk, c.pv, c.prefix_len, self.blk, self.logp, c.ring_k, c.ring_v, c.wp, c.fill, self.out,
-                       self.ws, lse=self.lse, scale=c.scale)
+        if self.fp8:
+            r.srswa_decode_fp8(q, self.k8, self.v8, self.ks, self.vs, c.prefix_len, self.blk, self.logp, c.ring_k,
+                               c.ring_v, c.wp, c.fill, self.out, self.ws, lse=self.lse, scale=c.scale)
+        else:
+            r.srswa_decode(q, c.pk, c.pv, c.prefix_len, self.blk, self.logp, c.ring_k, c.ring_v, c.wp, c.fill,
+                           self.out, self.ws, lse=self.lse, scale=c.scale)
         if ev is not None:
             ev[1].record()
         return 3
@@ -430,7 +454,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
-        "storage_dtype": "bf16",
+        "storage_dtype": "e4m3 prefix (f32 block scales) + bf16 ring" if prob.fp8 else "bf16",
         "data": "synthetic",
         "impl": "ours",
         "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "global_batch": B * world,
@@ -443,8 +467,8 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
         "seq_tok_per_s": steps_per_s * B,
         "hbm_gbs_step": world * K * (nbytes["attn"] + nbytes["route"]) / (ms_max / 1e3) / 1e9,
         "bytes_per_step": {"attn": nbytes["attn"], "route": nbytes["route"]},
-        "roofline": {"bound": "hbm", "kernel": "srswa decode_kernel<true>" if prob.sparse else
-                     "rswa decode_kernel<false>", "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": ("srswa decode_kernel<true" if prob.sparse else "rswa decode_kernel<false")
+                     + (", fp8>" if prob.fp8 else ", bf16>"), "achieved": achieved, "peak": peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
                      "fallback 6650 GB/s", "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes["attn"], "avg_launch_us": attn_avg_s * 1e6},
@@ -614,6 +638,10 @@ def oracle_sample_step(w: dict, sample: int, seed: int):
     st = dict(q=u(c.q[0]), k=u(c.k_new[0]), v=u(c.v_new[0]), pk=u(c.pk), pv=u(c.pv), plen=c.prefix_len.numpy(),
               rk=u(c.ring_k).copy(), rv=u(c.ring_v).copy(), wp=c.wp.numpy().copy(), fill=c.fill.numpy().copy(),
               scale=c.scale)
+    if w.get("fp8"):
+        import oracle
+        st["k8"], st["ks"] = oracle.quantize_prefix(st["pk"], st["plen"])
+        st["v8"], st["vs"] = oracle.quantize_prefix(st["pv"], st["plen"])
     if w["kind"] == "srswa":
         pl = synth.plant_router_keys(plen, cap, n_dirs=1, seed=seed + 1)
         st["k_idx"] = u(pl.k_idx)
@@ -625,12 +653,18 @@ def oracle_step(st: dict, w: dict):
     import oracle
     oracle.append(st["rk"], st["rv"], st["k"], st["v"], st["wp"], st["fill"])
     if w["kind"] == "rswa":
+        if w.get("fp8"):
+            return oracle.rswa_decode_fp8(st["q"], st["k8"], st["v8"], st["ks"], st["vs"], st["plen"], st["rk"],
+                                          st["rv"], st["wp"], st["fill"], st["scale"])
         return oracle.rswa_decode(st["q"], st["pk"], st["pv"], st["plen"], st["rk"], st["rv"], st["wp"], st["fill"],
                                   st["scale"])
     kbar = st.get("kbar")
     if kbar is None:
         kbar = st["kbar"] = oracle.index_pool(st["k_idx"], st["plen"])   # once per prefix, as on the GPU
     r = oracle.route(st["q_idx"], kbar, st["plen"])
+    if w.get("fp8"):
+        return oracle.srswa_decode_fp8(st["q"], st["k8"], st["v8"], st["ks"], st["vs"], st["plen"], r["blk_idx"],
+                                       r["blk_logp"], st["rk"], st["rv"], st["wp"], st["fill"], st["scale"])
     return oracle.srswa_decode(st["q"], st["pk"], st["pv"], st["plen"], r["blk_idx"], r["blk_logp"], st["rk"],
                                st["rv"], st["wp"], st["fill"], st["scale"])
 
@@ -661,7 +695,7 @@ def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
 def run_reference(args, w: dict) -> dict:
     """The oracle as the reference arm, on the host cores, K timed steps of a bounded sample."""
     import oracle
-    sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1}.get(args.config, 1))
+    sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2}.get(args.config, 1))
     st = oracle_sample_step(w, sample, seed=99)
     for _ in range(args.warmup):
         oracle_step(st, w)
@@ -716,7 +750,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")

@@ -201,8 +201,9 @@ RSWA_API rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, 
  * tau      : f32 [B] or NULL: the threshold of the x = z/2 problem
  * workspace: zero-initialised, rswa_workspace_bytes(dims, RSWA_OP_ROUTE) bytes (status word)
  * One thread-block cluster of ceil(ceil(prefix_cap / 32) / 1024) CTAs per sequence scores
- * the blocks; the CTAs hand their sorted top-32 lists and candidates to the first CTA
- * through distributed shared memory, which merges them and solves the threshold.
+ * the blocks; the CTAs exchange their maxima and hand the first CTA, through distributed
+ * shared memory, the blocks with z > max z - 2 (plus their sorted top-32 when the sequence
+ * has fewer than topk such blocks); the first CTA ranks them and solves the threshold.
  * Unsupported: ceil(prefix_cap / 32) > 8192.
  */
 RSWA_API rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,
@@ -253,6 +254,52 @@ RSWA_API rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, c
                                          const int32_t* prefix_len, const void* ring_k, const void* ring_v,
                                          const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                                          int32_t* status, void* stream);
+
+/*
+ * FP8 prefix cache (the pages name quantised KV-cache compression as a next step,
+ * "百度 Unlimited OCR 深度实战" tutorial, future directions, KV缓存压缩, without fixing a
+ * format; the format below is this library's reading). The prefix K and V are stored
+ * as OCP FP8 E4M3 codes (bias 7, 3 mantissa bits, subnormals, largest finite 448, no
+ * infinities) with one f32 scale per (sequence, head, 32-token block) for K and one
+ * for V; an element is code value * scale. The ring stays bf16.
+ *
+ * rswa_quantize_prefix: for every (b, h) and block c with 32c < prefix_len[b],
+ *   scale = amax / 448 over the block's valid rows and all D dims (1 if amax = 0),
+ *   code  = E4M3(x / scale), round to nearest even, saturating at +-448,
+ * both steps in f32. Rows of a partial block past prefix_len get code 0; blocks past
+ * prefix_len are not written.
+ * pk, pv       : bf16 [B][H][prefix_cap][D]
+ * pk8, pv8     : uint8 codes [B][H][prefix_cap][D] (caller-owned, written)
+ * k_scale, v_scale : f32 [B][H][ceil(prefix_cap / 32)] (written)
+ * status       : int32 device word or NULL (RSWA_DEVICE_BAD_PREFIX_LEN)
+ * Errors: host validation as rswa_decode; nothing is launched on error.
+ */
+RSWA_API rswa_status rswa_quantize_prefix(const rswa_dims* dims, const void* pk, const void* pv,
+                                          const int32_t* prefix_len, uint8_t* pk8, uint8_t* pv8, float* k_scale,
+                                          float* v_scale, int32_t* status, void* stream);
+
+/*
+ * rswa_decode over an FP8 prefix: prefix rows are read as codes (128 B per row per
+ * head) and their block scales; the ring as bf16. Same key set, arguments and
+ * workspace (RSWA_OP_DECODE) as rswa_decode, with pk8 / pv8 / k_scale / v_scale in
+ * place of pk / pv. Streams half the prefix bytes of the bf16 call.
+ */
+RSWA_API rswa_status rswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                                     const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                                     const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill,
+                                     float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
+                                     void* stream);
+
+/*
+ * srswa_decode over an FP8 prefix: the routed blocks are read as codes and scales, the
+ * ring as bf16. Arguments and workspace (RSWA_OP_SRSWA_DECODE) as srswa_decode, with
+ * pk8 / pv8 / k_scale / v_scale in place of pk / pv.
+ */
+RSWA_API rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                                      const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                                      const int32_t* blk_idx, const float* blk_logp, int32_t topk, const void* ring_k,
+                                      const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
+                                      float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -35,7 +35,8 @@ DEVICE_WAIT_TIMEOUT = 0x8
 DEVICE_PIPELINE = 0x10
 
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
-            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill")
+            "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill",
+            "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8")
 
 
 class RswaError(RuntimeError):
@@ -89,6 +90,9 @@ def load(path: str | None = None):
             "srswa_decode": ([DP, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "rswa_decode_noalloc": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, P], ctypes.c_int),
             "rswa_prefill": ([DP, I32, P, P, P, P, P, P, P, P, P, P, F32, P, P, I32, P, SZ, P], ctypes.c_int),
+            "rswa_quantize_prefix": ([DP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "rswa_decode_fp8": ([DP, P, P, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_decode_fp8": ([DP, P, P, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -258,6 +262,93 @@ def srswa_decode(q, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, f
                                                _ptr(blk_idx), _ptr(blk_logp), topk, _ptr(ring_k), _ptr(ring_v),
                                                _ptr(wp), _ptr(fill), scale, _ptr(out), _ptr(lse), _ptr(workspace),
                                                workspace.numel(), _stream(stream)))
+
+
+def fp8_prefix_buffers(pk: torch.Tensor):
+    """Empty E4M3 code tensors (uint8, pk's shape) and f32 block-scale tensors [B][H][ceil(cap/32)] for K and V."""
+    B, H, cap, D = pk.shape
+    nb = (cap + 31) // 32
+    dev = pk.device
+    return (torch.empty((B, H, cap, D), dtype=torch.uint8, device=dev),
+            torch.empty((B, H, cap, D), dtype=torch.uint8, device=dev),
+            torch.zeros((B, H, nb), dtype=torch.float32, device=dev),
+            torch.zeros((B, H, nb), dtype=torch.float32, device=dev))
+
+
+def rswa_quantize_prefix(pk, pv, prefix_len, pk8, pv8, k_scale, v_scale, status=None, stream=None):
+    B, H, cap, D = pk.shape
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(pk8, "pk8", torch.uint8, pk.shape)
+    _want(pv8, "pv8", torch.uint8, pk.shape)
+    nb = (cap + 31) // 32
+    _want(k_scale, "k_scale", torch.float32, (B, H, nb))
+    _want(v_scale, "v_scale", torch.float32, (B, H, nb))
+    dims = Dims(B, H, D, 1, cap)
+    _check("rswa_quantize_prefix", load().rswa_quantize_prefix(ctypes.byref(dims), _ptr(pk), _ptr(pv),
+                                                               _ptr(prefix_len), _ptr(pk8), _ptr(pv8),
+                                                               _ptr(k_scale), _ptr(v_scale), _ptr(status),
+                                                               _stream(stream)))
+
+
+def _want_fp8_prefix(pk8, pv8, k_scale, v_scale):
+    B, H, cap, D = pk8.shape
+    _want(pk8, "pk8", torch.uint8)
+    _want(pv8, "pv8", torch.uint8, pk8.shape)
+    _want(k_scale, "k_scale", torch.float32, (B, H, (cap + 31) // 32))
+    _want(v_scale, "v_scale", torch.float32, (B, H, (cap + 31) // 32))
+    return B, H, cap, D
+
+
+def rswa_decode_fp8(q, pk8, pv8, k_scale, v_scale, prefix_len, ring_k, ring_v, wp, fill, out, workspace, lse=None,
+                    scale=None, stream=None):
+    B, H, cap, D = _want_fp8_prefix(pk8, pv8, k_scale, v_scale)
+    n = ring_k.shape[2]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("rswa_decode_fp8", load().rswa_decode_fp8(ctypes.byref(dims), _ptr(q), _ptr(pk8), _ptr(pv8),
+                                                     _ptr(k_scale), _ptr(v_scale), _ptr(prefix_len), _ptr(ring_k),
+                                                     _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(out),
+                                                     _ptr(lse), _ptr(workspace), workspace.numel(),
+                                                     _stream(stream)))
+
+
+def srswa_decode_fp8(q, pk8, pv8, k_scale, v_scale, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, out,
+                     workspace, lse=None, scale=None, stream=None):
+    B, H, cap, D = _want_fp8_prefix(pk8, pv8, k_scale, v_scale)
+    n = ring_k.shape[2]
+    topk = blk_idx.shape[1]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, topk))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_decode_fp8", load().srswa_decode_fp8(ctypes.byref(dims), _ptr(q), _ptr(pk8), _ptr(pv8),
+                                                       _ptr(k_scale), _ptr(v_scale), _ptr(prefix_len),
+                                                       _ptr(blk_idx), _ptr(blk_logp), topk, _ptr(ring_k),
+                                                       _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(out),
+                                                       _ptr(lse), _ptr(workspace), workspace.numel(),
+                                                       _stream(stream)))
 
 
 def rswa_prefill(q, k_out, v_out, pk, pv, prefix_len, out, workspace, lse=None, ring_k=None, ring_v=None, wp=None,

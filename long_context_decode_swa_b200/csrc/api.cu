@@ -142,17 +142,36 @@ rswa_status rswa_append(const rswa_dims* dims, void* ring_k, void* ring_v, const
   return ok();
 }
 
+// The prefix K/V of a decode call: bf16 rows, or E4M3 code rows with block scales.
+struct PrefixSrc {
+  const void* k;
+  const void* v;
+  const float* ks;
+  const float* vs;
+  bool fp8;
+};
+
+static PrefixSrc bf16_prefix(const void* pk, const void* pv) { return PrefixSrc{pk, pv, nullptr, nullptr, false}; }
+
 // plan_budget > 0: plan the split-KV work to fit a workspace of that many bytes.
-static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, const void* pk,
-                                 const void* pv, const int32_t* prefix_len, const int32_t* blk_idx,
+static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, PrefixSrc px,
+                                 const int32_t* prefix_len, const int32_t* blk_idx,
                                  const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                                  const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0) {
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q);
+  const void* pk = px.k;
+  const void* pv = px.v;
   REQUIRE_PTR(pk);
   REQUIRE_PTR(pv);
+  if (px.fp8) {
+    const float* k_scale = px.ks;
+    const float* v_scale = px.vs;
+    REQUIRE_PTR(k_scale);
+    REQUIRE_PTR(v_scale);
+  }
   REQUIRE_PTR(ring_k);
   REQUIRE_PTR(ring_v);
   REQUIRE_PTR(out);
@@ -182,8 +201,14 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   if (plan.items > INT32_MAX) return fail(RSWA_ERR_UNSUPPORTED, "%s: too many work items", fn);
   a.items = (int)plan.items;
   a.q = static_cast<const uint16_t*>(q);
-  a.pk = static_cast<const uint16_t*>(pk);
-  a.pv = static_cast<const uint16_t*>(pv);
+  a.fp8 = px.fp8 ? 1 : 0;
+  a.pk = px.fp8 ? nullptr : static_cast<const uint16_t*>(pk);
+  a.pv = px.fp8 ? nullptr : static_cast<const uint16_t*>(pv);
+  a.pk8 = px.fp8 ? static_cast<const uint8_t*>(pk) : nullptr;
+  a.pv8 = px.fp8 ? static_cast<const uint8_t*>(pv) : nullptr;
+  a.kscale = px.ks;
+  a.vscale = px.vs;
+  a.nb_cap = (dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock;
   a.prefix_len = prefix_len;
   a.ring_k = static_cast<const uint16_t*>(ring_k);
   a.ring_v = static_cast<const uint16_t*>(ring_v);
@@ -208,16 +233,56 @@ rswa_status rswa_decode(const rswa_dims* dims, const void* q, const void* pk, co
                         const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
                         const int32_t* fill, float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
                         void* stream) {
-  return decode_common("rswa_decode", false, dims, q, pk, pv, prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp,
-                       fill, scale, out, lse, workspace, ws_bytes, stream);
+  return decode_common("rswa_decode", false, dims, q, bf16_prefix(pk, pv), prefix_len, nullptr, nullptr, 0, ring_k,
+                       ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status rswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                            const float* k_scale, const float* v_scale, const int32_t* prefix_len, const void* ring_k,
+                            const void* ring_v, const int32_t* wp, const int32_t* fill, float scale, float* out,
+                            float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("rswa_decode_fp8", false, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, prefix_len,
+                       nullptr, nullptr, 0, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                             const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                             const int32_t* blk_idx, const float* blk_logp, int32_t topk, const void* ring_k,
+                             const void* ring_v, const int32_t* wp, const int32_t* fill, float scale, float* out,
+                             float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("srswa_decode_fp8", true, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, prefix_len,
+                       blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status rswa_quantize_prefix(const rswa_dims* dims, const void* pk, const void* pv, const int32_t* prefix_len,
+                                 uint8_t* pk8, uint8_t* pv8, float* k_scale, float* v_scale, int32_t* status,
+                                 void* stream) {
+  const char* fn = "rswa_quantize_prefix";
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(pk);
+  REQUIRE_PTR(pv);
+  REQUIRE_PTR(pk8);
+  REQUIRE_PTR(pv8);
+  REQUIRE_PTR(k_scale);
+  REQUIRE_PTR(v_scale);
+  if (prefix_len == nullptr) return fail(RSWA_ERR_INVALID, "%s: prefix_len must not be NULL", fn);
+  if ((int64_t)dims->batch * dims->heads > 65535)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: batch * heads above 65535", fn);
+  cudaError_t e = rswa::launch_quantize_prefix(dims->batch, dims->heads, dims->prefix_cap,
+                                               static_cast<const uint16_t*>(pk), static_cast<const uint16_t*>(pv),
+                                               prefix_len, pk8, pv8, k_scale, v_scale, status,
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
 }
 
 rswa_status srswa_decode(const rswa_dims* dims, const void* q, const void* pk, const void* pv,
                          const int32_t* prefix_len, const int32_t* blk_idx, const float* blk_logp, int32_t topk,
                          const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("srswa_decode", true, dims, q, pk, pv, prefix_len, blk_idx, blk_logp, topk, ring_k, ring_v, wp,
-                       fill, scale, out, lse, workspace, ws_bytes, stream);
+  return decode_common("srswa_decode", true, dims, q, bf16_prefix(pk, pv), prefix_len, blk_idx, blk_logp, topk, ring_k,
+                       ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
 rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,
@@ -397,8 +462,8 @@ rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void
   // completion counters (everything before the partials) before this call.
   cudaError_t e = cudaMemsetAsync(scratch, 0, plan.partials_off, s);
   if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: clearing the scratch counters");
-  st = decode_common(fn, false, dims, q, pk, pv, prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp, fill, scale,
-                     out, lse, scratch, kNoAllocScratchBytes, stream, kNoAllocScratchBytes);
+  st = decode_common(fn, false, dims, q, bf16_prefix(pk, pv), prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp,
+                     fill, scale, out, lse, scratch, kNoAllocScratchBytes, stream, kNoAllocScratchBytes);
   if (st != RSWA_OK) return st;
   if (status != nullptr) {
     e = cudaMemcpyAsync(status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);

@@ -28,6 +28,9 @@
 //    of a (sequence, head) to finish (atomic counter) merges the partials by
 //    log-sum-exp and resets the counter.
 // The split count is chosen per launch to minimise the busiest CTA's tile count.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include <cmath>
 
 #include "common.cuh"
@@ -69,19 +72,21 @@ constexpr int kDecodeMinBlocks =
 
 // What a warp needs to enumerate a (sequence, head)'s tiles.
 struct SeqView {
-  const uint16_t* pk;  // prefix rows of this (b, h)
-  const uint16_t* pv;
+  const uint8_t* pk;  // prefix rows of this (b, h): bf16 rows, or E4M3 code rows (FP8 prefix)
+  const uint8_t* pv;
+  const float* ks;    // FP8 prefix: this (b, h)'s block scales
+  const float* vs;
   const uint16_t* rk;  // ring rows of this (b, h)
   const uint16_t* rv;
   int m;               // valid prefix rows
-  int nb;              // prefix blocks (SR-SWA)
+  int nb;              // prefix blocks
   int n_first;         // tiles before the ring (prefix tiles, or topk route entries)
   int a0, len0, len1;  // ring slot ranges [a0, a0+len0) and [0, len1)
   int n_r0, n_r1;
   int total;
 };
 
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, bool report) {
   SeqView v;
   const int64_t bh = (int64_t)b * a.H + h;
@@ -96,8 +101,16 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
     w = 0;
     f = 0;
   }
-  v.pk = a.pk + bh * a.cap * kHeadDim;
-  v.pv = a.pv + bh * a.cap * kHeadDim;
+  if (kFp8) {
+    v.pk = a.pk8 + bh * a.cap * kHeadDim;
+    v.pv = a.pv8 + bh * a.cap * kHeadDim;
+    v.ks = a.kscale + bh * a.nb_cap;
+    v.vs = a.vscale + bh * a.nb_cap;
+  } else {
+    v.pk = reinterpret_cast<const uint8_t*>(a.pk + bh * a.cap * kHeadDim);
+    v.pv = reinterpret_cast<const uint8_t*>(a.pv + bh * a.cap * kHeadDim);
+    v.ks = v.vs = nullptr;
+  }
   v.rk = a.ring_k + bh * a.n * kHeadDim;
   v.rv = a.ring_v + bh * a.n * kHeadDim;
   v.m = m;
@@ -115,32 +128,45 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
   return v;
 }
 
-// Tile t of a (b, h): source rows, row count (0 = empty tile) and log2 bias.
-// For SR-SWA, (c, lp) is route entry t when t < topk.
-template <bool kSparse>
-__device__ __forceinline__ void tile_at(const SeqView& v, int t, int c, float lp, const uint16_t*& k,
-                                        const uint16_t*& val, int& rows, float& bias, int32_t* status) {
-  bias = 0.f;
-  k = val = v.pk;
-  rows = 0;
-  if (t >= v.total) return;
+// Tile t of a (b, h): where its K and V rows start, how many rows (0 = empty tile), the
+// log2 bias, and the prefix block it covers (-1 for a ring tile). For SR-SWA, (c, lp) is
+// route entry t when t < topk.
+struct TileRef {
+  const uint8_t* k;
+  const uint8_t* v;
+  int rows;
+  float bias;
+  int blk;
+};
+
+template <bool kSparse, bool kFp8>
+__device__ __forceinline__ TileRef tile_at(const SeqView& v, int t, int c, float lp, int32_t* status) {
+  TileRef r;
+  r.bias = 0.f;
+  r.k = r.v = v.pk;
+  r.rows = 0;
+  r.blk = -1;
+  if (t >= v.total) return r;
   if (t < v.n_first) {
-    int start;
+    int blk;
     if (kSparse) {
-      if (c < 0 || !(lp > -INFINITY)) return;
+      if (c < 0 || !(lp > -INFINITY)) return r;
       if (c >= v.nb) {
         set_status(status, RSWA_DEVICE_BAD_BLOCK_IDX);
-        return;
+        return r;
       }
-      start = c * kBlock;
-      bias = lp * kLog2e;
+      blk = c;
+      r.bias = lp * kLog2e;
     } else {
-      start = t * kBlock;
+      blk = t;
     }
-    rows = min(kBlock, v.m - start);
-    k = v.pk + (int64_t)start * kHeadDim;
-    val = v.pv + (int64_t)start * kHeadDim;
-    return;
+    const int start = blk * kBlock;
+    const int64_t row_bytes = kFp8 ? kHeadDim : kRowBytes;
+    r.rows = min(kBlock, v.m - start);
+    r.k = v.pk + (int64_t)start * row_bytes;
+    r.v = v.pv + (int64_t)start * row_bytes;
+    r.blk = blk;
+    return r;
   }
   t -= v.n_first;
   int start, len;
@@ -152,9 +178,10 @@ __device__ __forceinline__ void tile_at(const SeqView& v, int t, int c, float lp
     start = t * kBlock;
     len = v.len1 - t * kBlock;
   }
-  rows = min(kBlock, len);
-  k = v.rk + (int64_t)start * kHeadDim;
-  val = v.rv + (int64_t)start * kHeadDim;
+  r.rows = min(kBlock, len);
+  r.k = reinterpret_cast<const uint8_t*>(v.rk + (int64_t)start * kHeadDim);
+  r.v = reinterpret_cast<const uint8_t*>(v.rv + (int64_t)start * kHeadDim);
+  return r;
 }
 
 // An item (sequence, head, split) as one warp sees it while issuing its tiles:
@@ -167,13 +194,13 @@ struct ItemView {
   float lp;
 };
 
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 __device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lane, ItemView& iv) {
   const int bh = item / a.splits, split = item - bh * a.splits;
   const int b = bh / a.H, h = bh - b * a.H;
   iv.item = item;
   iv.t0 = split * a.tiles_per_item;
-  iv.v = make_view<kSparse>(a, b, h, lane == 0 && split == 0 && h == 0);
+  iv.v = make_view<kSparse, kFp8>(a, b, h, lane == 0 && split == 0 && h == 0);
   iv.c = -1;
   iv.lp = -INFINITY;
   if (kSparse && lane < a.topk) {
@@ -182,59 +209,93 @@ __device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lan
   }
 }
 
+// A tile in flight: its row count (0: nothing issued), bias, and for an FP8 prefix tile
+// its K / V block scales (loaded at issue time, used at consume time).
+struct InFlight {
+  int rows;
+  float bias;
+  bool fp8;
+  float ks, vs;
+};
+
 // Issues CTA-local tile li (if it exists) into stage s: one bulk copy of its K rows and
-// one of its V rows on full[s]. Warp-collective. Returns the tile's row count (0: empty
-// or past the CTA's last item, nothing issued) and, in `bias`, its log2-domain bias.
-template <bool kSparse>
-__device__ __forceinline__ int issue_tile(const DecodeArgs& a, DecodeSmem& sm, int li, int s, int lane,
-                                          ItemView& iv, float& bias) {
+// one of its V rows on full[s]. Warp-collective.
+template <bool kSparse, bool kFp8>
+__device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& sm, int li, int s, int lane,
+                                               ItemView& iv) {
   const int P = a.tiles_per_item;
   const int it = li / P;
   const int64_t item = (int64_t)blockIdx.x + (int64_t)it * gridDim.x;
-  bias = 0.f;
-  if (item >= a.items) return 0;
-  if (iv.item != (int)item) load_item<kSparse>(a, (int)item, lane, iv);
+  InFlight f;
+  f.rows = 0;
+  f.bias = 0.f;
+  f.fp8 = false;
+  f.ks = f.vs = 1.f;
+  if (item >= a.items) return f;
+  if (iv.item != (int)item) load_item<kSparse, kFp8>(a, (int)item, lane, iv);
   const int tile = iv.t0 + (li - it * P);
   const int c = __shfl_sync(0xffffffffu, iv.c, tile & 31);
   const float lp = __shfl_sync(0xffffffffu, iv.lp, tile & 31);
-  const uint16_t *kp, *vp;
-  int rows;
-  tile_at<kSparse>(iv.v, tile, c, lp, kp, vp, rows, bias, lane == 0 ? a.status : nullptr);
-  if (rows > 0 && lane == 0) {
-    const uint32_t bytes = (uint32_t)rows * kRowBytes;
+  const TileRef r = tile_at<kSparse, kFp8>(iv.v, tile, c, lp, lane == 0 ? a.status : nullptr);
+  f.rows = r.rows;
+  f.bias = r.bias;
+  f.fp8 = kFp8 && r.blk >= 0;
+  if (f.fp8 && r.rows > 0) {
+    f.ks = iv.v.ks[r.blk];
+    f.vs = iv.v.vs[r.blk];
+  }
+  if (r.rows > 0 && lane == 0) {
+    const uint32_t bytes = (uint32_t)r.rows * (f.fp8 ? (uint32_t)kHeadDim : (uint32_t)kRowBytes);
     mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
-    if (kSparse && tile < iv.v.n_first) {
+    if (kSparse && r.blk >= 0) {
       // routed blocks change from step to step: mark them first to leave L2, so the ring,
       // which every step reads again, stays there (measured: 32K-history attention
       // 61.9 -> 57.0 us; the dense R-SWA prefix is streamed with the default policy, which
       // measured 1% faster there and keeps small prefixes L2-resident across steps)
       const uint64_t pol = l2_policy_evict_first();
-      bulk_copy_g2s_stream(sm.stage[s][0], kp, bytes, &sm.full[s], pol);
-      bulk_copy_g2s_stream(sm.stage[s][1], vp, bytes, &sm.full[s], pol);
+      bulk_copy_g2s_stream(sm.stage[s][0], r.k, bytes, &sm.full[s], pol);
+      bulk_copy_g2s_stream(sm.stage[s][1], r.v, bytes, &sm.full[s], pol);
     } else {
-      bulk_copy_g2s(sm.stage[s][0], kp, bytes, &sm.full[s]);
-      bulk_copy_g2s(sm.stage[s][1], vp, bytes, &sm.full[s]);
+      bulk_copy_g2s(sm.stage[s][0], r.k, bytes, &sm.full[s]);
+      bulk_copy_g2s(sm.stage[s][1], r.v, bytes, &sm.full[s]);
     }
   }
-  return rows;
+  return f;
+}
+
+// two E4M3 codes (low byte first) -> two floats, exactly (via f16)
+__device__ __forceinline__ float2 e4m3x2_f2(uint32_t pair) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(pair & 0xffffu), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 __device__ __forceinline__ float2 bf16x2_f2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
 
 // One tile for this warp: the 32 scores, the online-softmax update and P.V.
-// kFull: all 32 rows valid (no bounds checks).
-template <bool kFull>
-__device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* vt, int rows, float bias,
-                                             const float2 (&q2)[4], int g, int c, float& m_run, float& l_lane,
-                                             float2 (&acc)[4]) {
+// kFull: all 32 rows valid (no bounds checks). kFp8: the tile holds E4M3 code rows
+// (128 B) of one prefix block with scales (ks, vs), folded into the score and into the
+// row weight of P.V; otherwise bf16 rows (256 B) and ks = vs = 1.
+template <bool kFull, bool kFp8>
+__device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* vt, int rows, float bias, float ks,
+                                             float vs, const float2 (&q2)[4], int g, int c, float& m_run,
+                                             float& l_lane, float2 (&acc)[4]) {
   float pd[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const uint4 w = *reinterpret_cast<const uint4*>(kt + (2 * j + g) * kRowBytes + c * 16);
-    float2 d = __fmul2_rn(q2[0], bf16x2_f2(w.x));
-    d = __ffma2_rn(q2[1], bf16x2_f2(w.y), d);
-    d = __ffma2_rn(q2[2], bf16x2_f2(w.z), d);
-    d = __ffma2_rn(q2[3], bf16x2_f2(w.w), d);
+    float2 d;
+    if (kFp8) {
+      const uint2 w = *reinterpret_cast<const uint2*>(kt + (2 * j + g) * kHeadDim + c * 8);
+      d = __fmul2_rn(q2[0], e4m3x2_f2(w.x));
+      d = __ffma2_rn(q2[1], e4m3x2_f2(w.x >> 16), d);
+      d = __ffma2_rn(q2[2], e4m3x2_f2(w.y), d);
+      d = __ffma2_rn(q2[3], e4m3x2_f2(w.y >> 16), d);
+    } else {
+      const uint4 w = *reinterpret_cast<const uint4*>(kt + (2 * j + g) * kRowBytes + c * 16);
+      d = __fmul2_rn(q2[0], bf16x2_f2(w.x));
+      d = __ffma2_rn(q2[1], bf16x2_f2(w.y), d);
+      d = __ffma2_rn(q2[2], bf16x2_f2(w.z), d);
+      d = __ffma2_rn(q2[3], bf16x2_f2(w.w), d);
+    }
     pd[j] = d.x + d.y;
   }
   // reduce-scatter the 16 partial dots over the 16 lanes of this half-warp
@@ -266,7 +327,7 @@ __device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* v
     pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
   }
   // this lane now holds the score of tile row 2c + g
-  const float sc = (kFull || 2 * c + g < rows) ? pd[0] + bias : -INFINITY;
+  const float sc = (kFull || 2 * c + g < rows) ? (kFp8 ? fmaf(pd[0], ks, bias) : pd[0] + bias) : -INFINITY;
   const float m_new = fmaxf(m_run, warp_max(sc));
   const float alpha = exp2f(m_run - m_new);
   const float p = exp2f(sc - m_new);
@@ -275,21 +336,30 @@ __device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* v
 #pragma unroll
   for (int e = 0; e < 4; ++e) acc[e] = __fmul2_rn(acc[e], a2);
   m_run = m_new;
+  const float pw = kFp8 ? p * vs : p;  // the V block scale rides on the row weight
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const float pj = __shfl_sync(0xffffffffu, p, (g << 4) | j);
+    const float pj = __shfl_sync(0xffffffffu, pw, (g << 4) | j);
     if (kFull || 2 * j + g < rows) {
-      const uint4 w = *reinterpret_cast<const uint4*>(vt + (2 * j + g) * kRowBytes + c * 16);
       const float2 p2 = make_float2(pj, pj);
-      acc[0] = __ffma2_rn(p2, bf16x2_f2(w.x), acc[0]);
-      acc[1] = __ffma2_rn(p2, bf16x2_f2(w.y), acc[1]);
-      acc[2] = __ffma2_rn(p2, bf16x2_f2(w.z), acc[2]);
-      acc[3] = __ffma2_rn(p2, bf16x2_f2(w.w), acc[3]);
+      if (kFp8) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vt + (2 * j + g) * kHeadDim + c * 8);
+        acc[0] = __ffma2_rn(p2, e4m3x2_f2(w.x), acc[0]);
+        acc[1] = __ffma2_rn(p2, e4m3x2_f2(w.x >> 16), acc[1]);
+        acc[2] = __ffma2_rn(p2, e4m3x2_f2(w.y), acc[2]);
+        acc[3] = __ffma2_rn(p2, e4m3x2_f2(w.y >> 16), acc[3]);
+      } else {
+        const uint4 w = *reinterpret_cast<const uint4*>(vt + (2 * j + g) * kRowBytes + c * 16);
+        acc[0] = __ffma2_rn(p2, bf16x2_f2(w.x), acc[0]);
+        acc[1] = __ffma2_rn(p2, bf16x2_f2(w.y), acc[1]);
+        acc[2] = __ffma2_rn(p2, bf16x2_f2(w.z), acc[2]);
+        acc[3] = __ffma2_rn(p2, bf16x2_f2(w.w), acc[3]);
+      }
     }
   }
 }
 
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
@@ -304,15 +374,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
   griddep_wait();               // inputs may be written by the previous kernel in the stream
   griddep_launch_dependents();  // the next kernel may start its prologue
 
-  // In-flight tiles of this warp, oldest first: row count and bias of the warp's
-  // tiles k .. k + kStagesPerWarp - 1 (rows 0: nothing issued).
+  // In-flight tiles of this warp, oldest first: the warp's tiles k .. k + kStagesPerWarp - 1
+  // (rows 0: nothing issued).
   ItemView iv;
   iv.item = -1;
-  int fl_rows[kStagesPerWarp];
-  float fl_bias[kStagesPerWarp];
+  InFlight fl[kStagesPerWarp];
 #pragma unroll
   for (int j = 0; j < kStagesPerWarp; ++j)
-    fl_rows[j] = issue_tile<kSparse>(a, sm, warp + j * kWarps, warp * kStagesPerWarp + j, lane, iv, fl_bias[j]);
+    fl[j] = issue_tile<kSparse, kFp8>(a, sm, warp + j * kWarps, warp * kStagesPerWarp + j, lane, iv);
   uint32_t phase = 0;  // bit j: parity of the next completion of this warp's stage j
   int k = 0;           // tiles of this warp consumed so far
   bool ok = true;
@@ -343,7 +412,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
     for (int li = first; ok && li < li_base + P; li += kWarps) {
       const int j = k % kStagesPerWarp;
       const int s = warp * kStagesPerWarp + j;
-      const int rows = fl_rows[0];
+      const InFlight cur = fl[0];
+      const int rows = cur.rows;
       if (rows > 0) {
         // every lane waits (each needs the acquire), then the warp agrees
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (phase >> j) & 1u))) {
@@ -352,19 +422,24 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
           break;
         }
         phase ^= 1u << j;
-        if (rows == kBlock)
-          consume_tile<true>(sm.stage[s][0], sm.stage[s][1], rows, fl_bias[0], q2, g, c, m_run, l_lane, acc);
-        else
-          consume_tile<false>(sm.stage[s][0], sm.stage[s][1], rows, fl_bias[0], q2, g, c, m_run, l_lane, acc);
+        const uint8_t* kt = sm.stage[s][0];
+        const uint8_t* vt = sm.stage[s][1];
+        if (kFp8 && cur.fp8) {
+          if (rows == kBlock)
+            consume_tile<true, true>(kt, vt, rows, cur.bias, cur.ks, cur.vs, q2, g, c, m_run, l_lane, acc);
+          else
+            consume_tile<false, true>(kt, vt, rows, cur.bias, cur.ks, cur.vs, q2, g, c, m_run, l_lane, acc);
+        } else {
+          if (rows == kBlock)
+            consume_tile<true, false>(kt, vt, rows, cur.bias, 1.f, 1.f, q2, g, c, m_run, l_lane, acc);
+          else
+            consume_tile<false, false>(kt, vt, rows, cur.bias, 1.f, 1.f, q2, g, c, m_run, l_lane, acc);
+        }
       }
       __syncwarp();  // every lane has read the stage before it is refilled
 #pragma unroll
-      for (int i = 0; i + 1 < kStagesPerWarp; ++i) {
-        fl_rows[i] = fl_rows[i + 1];
-        fl_bias[i] = fl_bias[i + 1];
-      }
-      fl_rows[kStagesPerWarp - 1] =
-          issue_tile<kSparse>(a, sm, li + kWarps * kStagesPerWarp, s, lane, iv, fl_bias[kStagesPerWarp - 1]);
+      for (int i = 0; i + 1 < kStagesPerWarp; ++i) fl[i] = fl[i + 1];
+      fl[kStagesPerWarp - 1] = issue_tile<kSparse, kFp8>(a, sm, li + kWarps * kStagesPerWarp, s, lane, iv);
       ++k;
     }
     // fold the two half-warps (same dims, different rows) and the lanes' sums
@@ -455,7 +530,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
   // before the CTA's shared memory goes away (after a normal end none are left)
 #pragma unroll
   for (int i = 0; i < kStagesPerWarp; ++i)
-    if (fl_rows[i] > 0) {
+    if (fl[i].rows > 0) {
       const int j = (k + i) % kStagesPerWarp;
       mbar_wait(&sm.full[warp * kStagesPerWarp + j], (phase >> j) & 1u);
       phase ^= 1u << j;
@@ -506,15 +581,15 @@ WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_coun
 
 cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem);
-  static unsigned long long done_sparse = 0, done_dense = 0;
-  cudaError_t e = sparse ? ensure_smem_limit(decode_kernel<true>, smem, &done_sparse)
-                         : ensure_smem_limit(decode_kernel<false>, smem, &done_dense);
+  static unsigned long long done[4] = {0, 0, 0, 0};
+  auto kernel = sparse ? (a.fp8 ? decode_kernel<true, true> : decode_kernel<true, false>)
+                       : (a.fp8 ? decode_kernel<false, true> : decode_kernel<false, false>);
+  cudaError_t e = ensure_smem_limit(kernel, smem, &done[(sparse ? 2 : 0) + (a.fp8 ? 1 : 0)]);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   fill_launch_config(cfg, attr, dim3(grid), dim3(kDecodeThreads), smem, stream);
-  if (sparse) return cudaLaunchKernelEx(&cfg, decode_kernel<true>, a);
-  return cudaLaunchKernelEx(&cfg, decode_kernel<false>, a);
+  return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 }  // namespace rswa

@@ -31,6 +31,13 @@ struct DecodeArgs {
   const int32_t* blk_idx;
   const float* blk_logp;
   int topk;
+  // FP8 prefix (E4M3 codes + per (b, h, 32-token block) scales); pk / pv unused then
+  const uint8_t* pk8;
+  const uint8_t* pv8;
+  const float* kscale;  // [B*H][nb_cap]
+  const float* vscale;
+  int64_t nb_cap;
+  int fp8;
 };
 
 // Workspace layout shared by every op: [status: 256 B][counters][partials].
@@ -50,6 +57,9 @@ cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_
                           const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status,
                           cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream);
+cudaError_t launch_quantize_prefix(int B, int H, int64_t cap, const uint16_t* pk, const uint16_t* pv,
+                                   const int32_t* prefix_len, uint8_t* pk8, uint8_t* pv8, float* k_scale,
+                                   float* v_scale, int32_t* status, cudaStream_t stream);
 cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const int32_t* prefix_len, float* kbar,
                               cudaStream_t stream);
 // CTAs per sequence of the router (its thread-block cluster size).

@@ -15,6 +15,9 @@ page plus a 32-token prompt as the reference prefix, a 128-slot output ring):
 * SR-SWA router inputs are planted (``plant_router_keys``): for each query
   direction the generator fixes which 16 blocks score highest and in which
   order, with gaps of 0.04 in score, so the top-16 is known by construction.
+* An FP8 prefix drawn directly (``fp8_prefix``): uniformly random finite E4M3
+  code bytes (the two NaN codes excluded) and log-uniform positive block
+  scales, a valid stored cache without going through any quantiser.
 """
 from __future__ import annotations
 
@@ -212,6 +215,20 @@ def plant_router_keys(prefix_len, cap: int, n_dirs: int, seed: int, device="cpu"
     poison_(k_idx, rows[None, :] >= plen_t[:, None])
     q_idx = (Hm[:n_dirs] * qs).to(torch.float32)[:, None, :].expand(n_dirs, B, DI).contiguous()
     return RouterPlant(k_idx, q_idx, planted, n_dirs)
+
+
+def fp8_prefix(B: int, H: int, cap: int, seed: int, device="cpu", D: int = 128):
+    """Random E4M3 codes (uint8 [B][H][cap][D], 0x7f / 0xff excluded) and block scales
+    (f32 [B][H][ceil(cap/32)], log-uniform in [2^-10, 2^-4]) for K and for V."""
+    g = _gen(seed, device)
+    nb = (cap + BLOCK - 1) // BLOCK
+    out = []
+    for _ in range(2):
+        codes = torch.randint(0, 254, (B, H, cap, D), generator=g, device=device, dtype=torch.int32)
+        codes = codes + (codes >= 0x7f).int()                          # skip 0x7f; 254 values -> 0..0xfe
+        scales = torch.exp2(torch.rand((B, H, nb), generator=g, device=device) * 6.0 - 10.0)
+        out += [codes.to(torch.uint8), scales.float()]
+    return out[0], out[2], out[1], out[3]                               # k8, v8, k_scale, v_scale
 
 
 def log_uniform_pages(B: int, lo: int, hi: int, seed: int) -> list[int]:
