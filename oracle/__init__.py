@@ -64,6 +64,9 @@ def _L():
             lib.oracle_entmax15.restype = Dbl
             lib.oracle_route.argtypes = [I, I64, I, I, P, P, P, Dbl, I, P, P, P, P, P]
             lib.oracle_srswa_decode.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, I, P, P, P, P, Dbl, P, P]
+            lib.oracle_route_tokens.argtypes = [I, I, I64, I, I, P, P, P, Dbl, I, P, P]
+            lib.oracle_srswa_prefill.argtypes = [I, I, I, I, I64, I, I, P, P, P, P, P, P, P, P, I, P, P, P, P, Dbl,
+                                                 P, I, P, P]
             lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
             lib.oracle_e4m3_to_double.restype = Dbl
             lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
@@ -225,6 +228,60 @@ def srswa_decode(q, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, f
     _L().oracle_srswa_decode(B, H, D, n, cap, blk, _p(q), _p(pk), _p(pv), _p(prefix_len), _p(blk_idx),
                              _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp), _p(fill), float(scale),
                              _p(out), _p(lse))
+    return out, lse
+
+
+# ---------------------------------------------------------------- SR-SWA chunked prefill
+
+def route_tokens(q_idx, kbar, prefix_len, topk: int = 16, idx_scale: float = 1.0, blk: int = BLOCK):
+    """Per-token routes of a prefill chunk: q_idx fp32 [B][T][DI] against kbar [B][NBcap][DI].
+    Returns (blk_idx int32 [B][T][topk], blk_logp fp64 [B][T][topk])."""
+    q_idx = np.ascontiguousarray(q_idx, np.float32)
+    kbar = np.ascontiguousarray(kbar, np.float64)
+    prefix_len = _i32(prefix_len, "prefix_len")
+    B, nb_cap, DI = kbar.shape
+    if q_idx.ndim != 3 or q_idx.shape[0] != B or q_idx.shape[2] != DI:
+        raise ValueError("q_idx shape")
+    T = q_idx.shape[1]
+    blk_idx = np.zeros((B, T, topk), np.int32)
+    blk_logp = np.zeros((B, T, topk), np.float64)
+    _L().oracle_route_tokens(B, T, nb_cap, DI, blk, _p(q_idx), _p(kbar), _p(prefix_len), float(idx_scale),
+                             int(topk), _p(blk_idx), _p(blk_logp))
+    return blk_idx, blk_logp
+
+
+def srswa_prefill(q, k_out, v_out, pk, pv, prefix_len, blk_idx, blk_logp, scale, rows, n, ring_k=None, ring_v=None,
+                  wp=None, fill=None, blk: int = BLOCK):
+    """SR-SWA chunked prefill for the listed query rows, routes given ([B][T][topk]).
+    Returns (out [B][H][R][D], lse [B][H][R])."""
+    q = _u16(q, 4, "q")
+    k_out = _u16(k_out, 4, "k_out")
+    v_out = _u16(v_out, 4, "v_out")
+    pk = _u16(pk, 4, "pk")
+    pv = _u16(pv, 4, "pv")
+    B, H, T, D = q.shape
+    cap = pk.shape[2]
+    prefix_len = _i32(prefix_len, "prefix_len")
+    blk_idx = _i32(blk_idx, "blk_idx")
+    blk_logp = np.ascontiguousarray(blk_logp, np.float64)
+    if blk_idx.ndim != 3 or blk_idx.shape[:2] != (B, T):
+        raise ValueError("blk_idx shape")
+    topk = blk_idx.shape[2]
+    rows = _i32(np.asarray(rows, np.int32), "rows")
+    if rows.size and (rows.min() < 0 or rows.max() >= T):
+        raise ValueError("row index out of range")
+    if ring_k is not None:
+        ring_k = _u16(ring_k, 4, "ring_k")
+        ring_v = _u16(ring_v, 4, "ring_v")
+        wp, fill = _i32(wp, "wp"), _i32(fill, "fill")
+        if ring_k.shape[2] != n:
+            raise ValueError("ring slots != n")
+    R = rows.size
+    out = np.zeros((B, H, R, D), np.float64)
+    lse = np.zeros((B, H, R), np.float64)
+    _L().oracle_srswa_prefill(B, H, D, int(n), cap, T, blk, _p(q), _p(k_out), _p(v_out), _p(pk), _p(pv),
+                              _p(prefix_len), _p(blk_idx), _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp),
+                              _p(fill), float(scale), _p(rows), R, _p(out), _p(lse))
     return out, lse
 
 

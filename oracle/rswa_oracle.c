@@ -436,49 +436,55 @@ static int cmp_rank(const void* a, const void* b) {
  * zero past NB), tau [B] (nullable, tau of the x = z/2 problem),
  * z_out [B][NBcap] (nullable).
  */
+/* One router query against one sequence's NB block keys (the body of oracle_route). */
+static void route_one(int64_t NB, int64_t nb_cap, int DI, const float* qv, const double* kb, double idx_scale,
+                      int topk, int32_t* blk_idx, double* blk_logp, double* probs, double* tau, double* z_out) {
+  double* z = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
+  double* x = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
+  double* p = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
+  zc_pair* r = (zc_pair*)malloc(sizeof(zc_pair) * (size_t)(NB > 0 ? NB : 1));
+  for (int64_t c = 0; c < NB; ++c) {
+    double dot = 0.0;
+    for (int d = 0; d < DI; ++d) dot += (double)qv[d] * kb[c * DI + d];
+    z[c] = idx_scale * dot;
+    x[c] = z[c] / 2.0;
+  }
+  double t = oracle_entmax15(NB, x, p);
+  for (int64_t c = 0; c < NB; ++c) {
+    r[c].z = (float)z[c];
+    r[c].c = c;
+  }
+  qsort(r, (size_t)NB, sizeof(zc_pair), cmp_rank);
+  for (int k = 0; k < topk; ++k) {
+    if (k < NB) {
+      int64_t c = r[k].c;
+      blk_idx[k] = (int32_t)c;
+      blk_logp[k] = p[c] > 0.0 ? log(p[c]) : -INFINITY;
+    } else {
+      blk_idx[k] = -1;
+      blk_logp[k] = -INFINITY;
+    }
+  }
+  if (probs)
+    for (int64_t c = 0; c < nb_cap; ++c) probs[c] = c < NB ? p[c] : 0.0;
+  if (z_out)
+    for (int64_t c = 0; c < nb_cap; ++c) z_out[c] = c < NB ? z[c] : 0.0;
+  if (tau) *tau = t;
+  free(z);
+  free(x);
+  free(p);
+  free(r);
+}
+
 void oracle_route(int B, int64_t nb_cap, int DI, int blk, const float* q_idx, const double* kbar,
                   const int32_t* prefix_len, double idx_scale, int topk, int32_t* blk_idx, double* blk_logp,
                   double* probs, double* tau, double* z_out) {
 #pragma omp parallel for schedule(dynamic, 1)
   for (int b = 0; b < B; ++b) {
-    int64_t m = prefix_len[b];
-    int64_t NB = (m + blk - 1) / blk;
-    double* z = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
-    double* x = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
-    double* p = (double*)malloc(sizeof(double) * (size_t)(NB > 0 ? NB : 1));
-    zc_pair* r = (zc_pair*)malloc(sizeof(zc_pair) * (size_t)(NB > 0 ? NB : 1));
-    for (int64_t c = 0; c < NB; ++c) {
-      double dot = 0.0;
-      for (int d = 0; d < DI; ++d) dot += (double)q_idx[(int64_t)b * DI + d] * kbar[((int64_t)b * nb_cap + c) * DI + d];
-      z[c] = idx_scale * dot;
-      x[c] = z[c] / 2.0;
-    }
-    double t = oracle_entmax15(NB, x, p);
-    for (int64_t c = 0; c < NB; ++c) {
-      r[c].z = (float)z[c];
-      r[c].c = c;
-    }
-    qsort(r, (size_t)NB, sizeof(zc_pair), cmp_rank);
-    for (int k = 0; k < topk; ++k) {
-      int64_t o = (int64_t)b * topk + k;
-      if (k < NB) {
-        int64_t c = r[k].c;
-        blk_idx[o] = (int32_t)c;
-        blk_logp[o] = p[c] > 0.0 ? log(p[c]) : -INFINITY;
-      } else {
-        blk_idx[o] = -1;
-        blk_logp[o] = -INFINITY;
-      }
-    }
-    if (probs)
-      for (int64_t c = 0; c < nb_cap; ++c) probs[(int64_t)b * nb_cap + c] = c < NB ? p[c] : 0.0;
-    if (z_out)
-      for (int64_t c = 0; c < nb_cap; ++c) z_out[(int64_t)b * nb_cap + c] = c < NB ? z[c] : 0.0;
-    if (tau) tau[b] = t;
-    free(z);
-    free(x);
-    free(p);
-    free(r);
+    int64_t NB = ((int64_t)prefix_len[b] + blk - 1) / blk;
+    route_one(NB, nb_cap, DI, q_idx + (int64_t)b * DI, kbar + (int64_t)b * nb_cap * DI, idx_scale, topk,
+              blk_idx + (int64_t)b * topk, blk_logp + (int64_t)b * topk, probs ? probs + (int64_t)b * nb_cap : NULL,
+              tau ? tau + b : NULL, z_out ? z_out + (int64_t)b * nb_cap : NULL);
   }
 }
 
@@ -704,4 +710,87 @@ void oracle_srswa_decode_fp8(int B, int H, int D, int n, int64_t cap, int blk, c
 /* Element-wise oracle_e4m3_encode over an array (for the tests). */
 void oracle_e4m3_encode_array(int64_t count, const float* x, uint8_t* out) {
   for (int64_t i = 0; i < count; ++i) out[i] = oracle_e4m3_encode(x[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* next row: SR-SWA chunked prefill                                    */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Per-token routing of a prefill chunk: output-side query i of sequence b has
+ * its own router query q_idx[b][i] and is routed exactly as a decode query
+ * (oracle_route) against the sequence's block keys. The pages name this
+ * per-token router for prefill through its [tokens, context/32] score tensor
+ * (serving notes, --max-prefill-tokens); its rule is the decode router's.
+ * q_idx [B][T][DI]; outputs blk_idx, blk_logp [B][T][topk].
+ * Pinned by: every token equals oracle_route called on that token alone.
+ */
+void oracle_route_tokens(int B, int T, int64_t nb_cap, int DI, int blk, const float* q_idx, const double* kbar,
+                         const int32_t* prefix_len, double idx_scale, int topk, int32_t* blk_idx, double* blk_logp) {
+  int64_t BT = (int64_t)B * T;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t bt = 0; bt < BT; ++bt) {
+    int64_t b = bt / T;
+    int64_t NB = ((int64_t)prefix_len[b] + blk - 1) / blk;
+    route_one(NB, nb_cap, DI, q_idx + bt * DI, kbar + b * nb_cap * DI, idx_scale, topk, blk_idx + bt * topk,
+              blk_logp + bt * topk, NULL, NULL, NULL);
+  }
+}
+
+/*
+ * SR-SWA chunked prefill rows: output-side query i of (b, h) attends to its
+ * routed prefix blocks (their valid tokens, bias ln p, as in
+ * oracle_srswa_decode) and to the outputs j with i - n < j <= i (bias 0),
+ * positions j < 0 coming from the previous chunk's ring as in
+ * oracle_rswa_prefill. Routes blk_idx / blk_logp [B][T][topk] are inputs.
+ * out [B][H][nrows][D], lse [B][H][nrows].
+ * Pinned by: row i equals oracle_srswa_decode after appending outputs 0..i
+ * with row i's route; every block routed with zero bias equals
+ * oracle_rswa_prefill.
+ */
+void oracle_srswa_prefill(int B, int H, int D, int n, int64_t cap, int T, int blk, const uint16_t* q,
+                          const uint16_t* k_out, const uint16_t* v_out, const uint16_t* pk, const uint16_t* pv,
+                          const int32_t* prefix_len, const int32_t* blk_idx, const double* blk_logp, int topk,
+                          const uint16_t* ring_k, const uint16_t* ring_v, const int32_t* wp, const int32_t* fill,
+                          double scale, const int32_t* rows, int nrows, double* out, double* lse) {
+  int64_t work = (int64_t)B * H * nrows;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, (int64_t)topk * blk + n + 1);
+#pragma omp for schedule(dynamic, 8)
+    for (int64_t w = 0; w < work; ++w) {
+      int64_t bh = w / nrows;
+      int64_t r = w % nrows;
+      int64_t b = bh / H;
+      int64_t i = rows[r];
+      int64_t m = prefix_len[b];
+      L.count = 0;
+      for (int k = 0; k < topk; ++k) {
+        int64_t c = blk_idx[(b * T + i) * topk + k];
+        double bias = blk_logp[(b * T + i) * topk + k];
+        if (c < 0 || bias == -INFINITY) continue;
+        int64_t t1 = (c + 1) * blk < m ? (c + 1) * blk : m;
+        for (int64_t t = c * blk; t < t1; ++t) {
+          int64_t off = (bh * cap + t) * D;
+          keylist_push(&L, pk + off, pv + off, bias);
+        }
+      }
+      for (int64_t j = i - n + 1; j <= i; ++j) {
+        if (j >= 0) {
+          int64_t off = (bh * T + j) * D;
+          keylist_push(&L, k_out + off, v_out + off, 0.0);
+        } else if (ring_k != NULL) {
+          int64_t back = -j;
+          if (back <= fill[b]) {
+            int64_t slot = pos_mod((int64_t)wp[b] - back, n);
+            int64_t off = (bh * n + slot) * D;
+            keylist_push(&L, ring_k + off, ring_v + off, 0.0);
+          }
+        }
+      }
+      attend(&L, q + (bh * T + i) * D, D, scale, out + (bh * nrows + r) * D, lse + bh * nrows + r);
+    }
+    keylist_free(&L);
+  }
 }
