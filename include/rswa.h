@@ -256,6 +256,38 @@ RSWA_API rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, c
                                          int32_t* status, void* stream);
 
 /*
+ * SR-SWA chunked prefill (the survey's next row 1). The pages size prefill memory by a
+ * per-token router score tensor of about [tokens, context/32] (serving notes,
+ * --max-prefill-tokens), i.e. every output-side token of a chunk is routed by itself;
+ * the rule is the decode router's (srswa_route). Reading adopted: query i of a chunk of
+ * T outputs attends to its own top-k routed prefix blocks (bias ln p) and to the outputs
+ * j with i - n < j <= i (bias 0); positions j < 0 come from the previous chunk's ring, as
+ * in rswa_prefill.
+ *
+ * srswa_route_tokens: srswa_route for T router queries per sequence.
+ *   q_idx    : f32 [B][T][32];  kbar : f32 [B][ceil(prefix_cap / 32)][32]
+ *   blk_idx  : int32 [B][T][topk];  blk_logp : f32 [B][T][topk]
+ *   workspace: >= 256 bytes (status word).  Unsupported: B * T > 65535.
+ * srswa_prefill: the attention of the chunk's T queries.
+ *   q, k_out, v_out : bf16 [B][H][T][D] (the chunk's queries and output K/V)
+ *   pk, pv, prefix_len : as srswa_decode;  blk_idx / blk_logp from srswa_route_tokens
+ *   ring_k, ring_v, wp, fill : the previous chunk's ring, or all NULL for the first chunk
+ *   out : f32 [B][H][T][D];  lse : f32 [B][H][T] or NULL
+ *   workspace: >= 256 bytes (status word; every query is one work item).
+ * Each query runs through the gathered-decode pipeline (its routed blocks, then the ring
+ * part, then the band, as 32-row tiles).
+ */
+RSWA_API rswa_status srswa_route_tokens(const rswa_dims* dims, int32_t T, const float* q_idx, const float* kbar,
+                                        const int32_t* prefix_len, float idx_scale, int32_t topk, int32_t* blk_idx,
+                                        float* blk_logp, void* workspace, size_t ws_bytes, void* stream);
+
+RSWA_API rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out,
+                                   const void* v_out, const void* pk, const void* pv, const int32_t* prefix_len,
+                                   const int32_t* blk_idx, const float* blk_logp, int32_t topk, const void* ring_k,
+                                   const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
+                                   float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * FP8 prefix cache (the pages name quantised KV-cache compression as a next step,
  * "百度 Unlimited OCR 深度实战" tutorial, future directions, KV缓存压缩, without fixing a
  * format; the format below is this library's reading). The prefix K and V are stored

@@ -36,7 +36,7 @@ DEVICE_PIPELINE = 0x10
 
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
             "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill",
-            "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8")
+            "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill")
 
 
 class RswaError(RuntimeError):
@@ -93,6 +93,8 @@ def load(path: str | None = None):
             "rswa_quantize_prefix": ([DP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "rswa_decode_fp8": ([DP, P, P, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_decode_fp8": ([DP, P, P, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_route_tokens": ([DP, I32, P, P, P, F32, I32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_prefill": ([DP, I32, P, P, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -349,6 +351,59 @@ def srswa_decode_fp8(q, pk8, pv8, k_scale, v_scale, prefix_len, blk_idx, blk_log
                                                        _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(out),
                                                        _ptr(lse), _ptr(workspace), workspace.numel(),
                                                        _stream(stream)))
+
+
+def srswa_route_tokens(q_idx, kbar, prefix_len, blk_idx, blk_logp, workspace, idx_scale=1.0, prefix_cap=None,
+                       stream=None):
+    """Per-token routes of a chunk: q_idx f32 [B][T][32] -> blk_idx int32 / blk_logp f32 [B][T][topk]."""
+    B, nb_cap, DI = kbar.shape
+    T = q_idx.shape[1]
+    topk = blk_idx.shape[2]
+    _want(q_idx, "q_idx", torch.float32, (B, T, DI))
+    _want(kbar, "kbar", torch.float32)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, T, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, T, topk))
+    _want(workspace, "workspace", torch.uint8)
+    cap = nb_cap * 32 if prefix_cap is None else int(prefix_cap)
+    dims = Dims(B, 1, 128, 1, cap)
+    _check("srswa_route_tokens", load().srswa_route_tokens(ctypes.byref(dims), T, _ptr(q_idx), _ptr(kbar),
+                                                           _ptr(prefix_len), float(idx_scale), topk, _ptr(blk_idx),
+                                                           _ptr(blk_logp), _ptr(workspace), workspace.numel(),
+                                                           _stream(stream)))
+
+
+def srswa_prefill(q, k_out, v_out, pk, pv, prefix_len, blk_idx, blk_logp, out, workspace, lse=None, ring_k=None,
+                  ring_v=None, wp=None, fill=None, scale=None, ring: int = 128, stream=None):
+    """SR-SWA chunked prefill of T queries per (sequence, head), routes given per token."""
+    B, H, T, D = q.shape
+    cap = pk.shape[2]
+    topk = blk_idx.shape[2]
+    _want(q, "q", torch.bfloat16, (B, H, T, D))
+    _want(k_out, "k_out", torch.bfloat16, (B, H, T, D))
+    _want(v_out, "v_out", torch.bfloat16, (B, H, T, D))
+    _want(pk, "pk", torch.bfloat16, (B, H, cap, D))
+    _want(pv, "pv", torch.bfloat16, (B, H, cap, D))
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, T, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, T, topk))
+    _want(out, "out", torch.float32, (B, H, T, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H, T))
+    n = ring
+    if ring_k is not None:
+        n = ring_k.shape[2]
+        _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+        _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+        _want(wp, "wp", torch.int32, (B,))
+        _want(fill, "fill", torch.int32, (B,))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_prefill", load().srswa_prefill(ctypes.byref(dims), T, _ptr(q), _ptr(k_out), _ptr(v_out), _ptr(pk),
+                                                 _ptr(pv), _ptr(prefix_len), _ptr(blk_idx), _ptr(blk_logp), topk,
+                                                 _ptr(ring_k), _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(out),
+                                                 _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def rswa_prefill(q, k_out, v_out, pk, pv, prefix_len, out, workspace, lse=None, ring_k=None, ring_v=None, wp=None,

@@ -153,9 +153,18 @@ struct PrefixSrc {
 
 static PrefixSrc bf16_prefix(const void* pk, const void* pv) { return PrefixSrc{pk, pv, nullptr, nullptr, false}; }
 
+// SR-SWA chunked prefill: T queries per (sequence, head) whose causal band is read from the
+// chunk's output K/V; T = 1 and no band for decode.
+struct BandSrc {
+  int T;
+  const void* k_out;
+  const void* v_out;
+};
+constexpr BandSrc kNoBand{1, nullptr, nullptr};
+
 // plan_budget > 0: plan the split-KV work to fit a workspace of that many bytes.
 static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, PrefixSrc px,
-                                 const int32_t* prefix_len, const int32_t* blk_idx,
+                                 BandSrc band, const int32_t* prefix_len, const int32_t* blk_idx,
                                  const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                                  const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0) {
@@ -172,22 +181,53 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
     REQUIRE_PTR(k_scale);
     REQUIRE_PTR(v_scale);
   }
-  REQUIRE_PTR(ring_k);
-  REQUIRE_PTR(ring_v);
+  const bool prefill = band.k_out != nullptr;
+  if (prefill) {  // the ring (the previous chunk) is optional
+    const void* k_out = band.k_out;
+    const void* v_out = band.v_out;
+    REQUIRE_PTR(k_out);
+    REQUIRE_PTR(v_out);
+    if (band.T < 1) return fail(RSWA_ERR_INVALID, "%s: T must be >= 1 (got %d)", fn, band.T);
+    if ((ring_k == nullptr) != (ring_v == nullptr))
+      return fail(RSWA_ERR_INVALID, "%s: ring_k and ring_v must both be given or both be NULL", fn);
+    if (ring_k != nullptr && (wp == nullptr || fill == nullptr))
+      return fail(RSWA_ERR_INVALID, "%s: a ring needs wp and fill", fn);
+    REQUIRE_PTR_OR_NULL(ring_k);
+    REQUIRE_PTR_OR_NULL(ring_v);
+    if (prefix_len == nullptr) return fail(RSWA_ERR_INVALID, "%s: prefix_len must not be NULL", fn);
+  } else {
+    REQUIRE_PTR(ring_k);
+    REQUIRE_PTR(ring_v);
+    if (prefix_len == nullptr || wp == nullptr || fill == nullptr)
+      return fail(RSWA_ERR_INVALID, "%s: prefix_len, wp and fill must not be NULL", fn);
+  }
   REQUIRE_PTR(out);
   REQUIRE_PTR(workspace);
-  if (prefix_len == nullptr || wp == nullptr || fill == nullptr)
-    return fail(RSWA_ERR_INVALID, "%s: prefix_len, wp and fill must not be NULL", fn);
   if (sparse) {
     if (blk_idx == nullptr || blk_logp == nullptr)
       return fail(RSWA_ERR_INVALID, "%s: blk_idx and blk_logp must not be NULL", fn);
     if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
   }
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
-  const int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(topk, dims->ring)
-                                   : rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring);
-  const rswa::WorkspacePlan plan =
-      rswa::plan_decode_workspace(dims->batch, dims->heads, max_tiles, rswa::device_sm_count(), plan_budget);
+  int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(topk, dims->ring)
+                             : rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring);
+  rswa::WorkspacePlan plan;
+  if (prefill) {
+    // ring part and band together cover n keys in at most three ranges: two tiles beyond a decode's
+    max_tiles += 2;
+    const int64_t queries = (int64_t)dims->batch * dims->heads * band.T;
+    if (queries > INT32_MAX) return fail(RSWA_ERR_UNSUPPORTED, "%s: too many queries", fn);
+    // many queries: one split each (the status word is all the workspace needed)
+    const int64_t slots = (int64_t)rswa::device_sm_count() * rswa::decode_ctas_per_sm();
+    plan.splits = 1;
+    plan.tiles_per_item = (int)max_tiles;
+    plan.items = queries;
+    plan.grid = (int)(queries < slots ? queries : slots);
+    plan.counters_off = plan.partials_off = 0;
+    plan.bytes = 256;
+  } else {
+    plan = rswa::plan_decode_workspace(dims->batch, dims->heads, max_tiles, rswa::device_sm_count(), plan_budget);
+  }
   if (ws_bytes < plan.bytes)
     return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes,
                 plan.bytes);
@@ -209,6 +249,9 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.kscale = px.ks;
   a.vscale = px.vs;
   a.nb_cap = (dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock;
+  a.T = prefill ? band.T : 1;
+  a.k_out = static_cast<const uint16_t*>(band.k_out);
+  a.v_out = static_cast<const uint16_t*>(band.v_out);
   a.prefix_len = prefix_len;
   a.ring_k = static_cast<const uint16_t*>(ring_k);
   a.ring_v = static_cast<const uint16_t*>(ring_v);
@@ -219,8 +262,8 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = ws_status(workspace);
-  a.counters = reinterpret_cast<int32_t*>(ws + plan.counters_off);
-  a.partials = reinterpret_cast<float*>(ws + plan.partials_off);
+  a.counters = prefill ? nullptr : reinterpret_cast<int32_t*>(ws + plan.counters_off);
+  a.partials = prefill ? nullptr : reinterpret_cast<float*>(ws + plan.partials_off);
   a.blk_idx = blk_idx;
   a.blk_logp = blk_logp;
   a.topk = sparse ? topk : 0;
@@ -233,7 +276,8 @@ rswa_status rswa_decode(const rswa_dims* dims, const void* q, const void* pk, co
                         const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
                         const int32_t* fill, float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
                         void* stream) {
-  return decode_common("rswa_decode", false, dims, q, bf16_prefix(pk, pv), prefix_len, nullptr, nullptr, 0, ring_k,
+  return decode_common("rswa_decode", false, dims, q, bf16_prefix(pk, pv), kNoBand, prefix_len, nullptr, nullptr, 0,
+                       ring_k,
                        ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -241,7 +285,8 @@ rswa_status rswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t*
                             const float* k_scale, const float* v_scale, const int32_t* prefix_len, const void* ring_k,
                             const void* ring_v, const int32_t* wp, const int32_t* fill, float scale, float* out,
                             float* lse, void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("rswa_decode_fp8", false, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, prefix_len,
+  return decode_common("rswa_decode_fp8", false, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
+                       prefix_len,
                        nullptr, nullptr, 0, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -250,7 +295,8 @@ rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t
                              const int32_t* blk_idx, const float* blk_logp, int32_t topk, const void* ring_k,
                              const void* ring_v, const int32_t* wp, const int32_t* fill, float scale, float* out,
                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("srswa_decode_fp8", true, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, prefix_len,
+  return decode_common("srswa_decode_fp8", true, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
+                       prefix_len,
                        blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -281,7 +327,8 @@ rswa_status srswa_decode(const rswa_dims* dims, const void* q, const void* pk, c
                          const int32_t* prefix_len, const int32_t* blk_idx, const float* blk_logp, int32_t topk,
                          const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("srswa_decode", true, dims, q, bf16_prefix(pk, pv), prefix_len, blk_idx, blk_logp, topk, ring_k,
+  return decode_common("srswa_decode", true, dims, q, bf16_prefix(pk, pv), kNoBand, prefix_len, blk_idx, blk_logp, topk,
+                       ring_k,
                        ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -363,10 +410,10 @@ rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, const int
   return ok();
 }
 
-rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,
-                        float idx_scale, int32_t topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                        void* workspace, size_t ws_bytes, void* stream) {
-  const char* fn = "srswa_route";
+static rswa_status route_common(const char* fn, const rswa_dims* dims, int tokens, const float* q_idx,
+                                const float* kbar, const int32_t* prefix_len, float idx_scale, int32_t topk,
+                                int32_t* blk_idx, float* blk_logp, float* probs, float* tau, void* workspace,
+                                size_t ws_bytes, void* stream) {
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q_idx);
@@ -377,16 +424,44 @@ rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* 
     return fail(RSWA_ERR_INVALID, "%s: prefix_len, blk_idx and blk_logp must not be NULL", fn);
   if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
   if (!std::isfinite(idx_scale)) return fail(RSWA_ERR_INVALID, "%s: idx_scale must be finite", fn);
+  if (tokens < 1) return fail(RSWA_ERR_INVALID, "%s: T must be >= 1 (got %d)", fn, tokens);
+  if ((int64_t)dims->batch * tokens > 65535)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: batch * T above 65535 router queries", fn);
   const int64_t nb_cap = (dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock;
   if (nb_cap > rswa::kMaxRouteBlocks)
     return fail(RSWA_ERR_UNSUPPORTED, "%s: %lld prefix blocks exceed the router's limit of %d", fn,
                 (long long)nb_cap, rswa::kMaxRouteBlocks);
   if (nb_cap == 0) return fail(RSWA_ERR_INVALID, "%s: prefix_cap must be >= 1", fn);
   if (ws_bytes < 256) return fail(RSWA_ERR_INVALID, "%s: workspace must be at least 256 bytes", fn);
-  cudaError_t e = rswa::launch_route(dims->batch, dims->prefix_cap, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx,
-                                     blk_logp, probs, tau, ws_status(workspace), static_cast<cudaStream_t>(stream));
+  cudaError_t e = rswa::launch_route(dims->batch, tokens, dims->prefix_cap, q_idx, kbar, prefix_len, idx_scale, topk,
+                                     blk_idx, blk_logp, probs, tau, ws_status(workspace),
+                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
+}
+
+rswa_status srswa_route(const rswa_dims* dims, const float* q_idx, const float* kbar, const int32_t* prefix_len,
+                        float idx_scale, int32_t topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  return route_common("srswa_route", dims, 1, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx, blk_logp, probs,
+                      tau, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_route_tokens(const rswa_dims* dims, int32_t T, const float* q_idx, const float* kbar,
+                               const int32_t* prefix_len, float idx_scale, int32_t topk, int32_t* blk_idx,
+                               float* blk_logp, void* workspace, size_t ws_bytes, void* stream) {
+  return route_common("srswa_route_tokens", dims, T, q_idx, kbar, prefix_len, idx_scale, topk, blk_idx, blk_logp,
+                      nullptr, nullptr, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,
+                          const void* pk, const void* pv, const int32_t* prefix_len, const int32_t* blk_idx,
+                          const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
+                          const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("srswa_prefill", true, dims, q, bf16_prefix(pk, pv), BandSrc{T, k_out, v_out}, prefix_len,
+                       blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes,
+                       stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -462,7 +537,8 @@ rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void
   // completion counters (everything before the partials) before this call.
   cudaError_t e = cudaMemsetAsync(scratch, 0, plan.partials_off, s);
   if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: clearing the scratch counters");
-  st = decode_common(fn, false, dims, q, bf16_prefix(pk, pv), prefix_len, nullptr, nullptr, 0, ring_k, ring_v, wp,
+  st = decode_common(fn, false, dims, q, bf16_prefix(pk, pv), kNoBand, prefix_len, nullptr, nullptr, 0, ring_k, ring_v,
+                     wp,
                      fill, scale, out, lse, scratch, kNoAllocScratchBytes, stream, kNoAllocScratchBytes);
   if (st != RSWA_OK) return st;
   if (status != nullptr) {

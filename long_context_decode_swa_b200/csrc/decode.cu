@@ -78,28 +78,40 @@ struct SeqView {
   const float* vs;
   const uint16_t* rk;  // ring rows of this (b, h)
   const uint16_t* rv;
+  const uint16_t* bk;  // chunked prefill: the query's causal band of output rows (null for decode)
+  const uint16_t* bv;
   int m;               // valid prefix rows
   int nb;              // prefix blocks
   int n_first;         // tiles before the ring (prefix tiles, or topk route entries)
   int a0, len0, len1;  // ring slot ranges [a0, a0+len0) and [0, len1)
   int n_r0, n_r1;
+  int blen, n_band;    // band rows and tiles (chunked prefill)
   int total;
 };
 
+// The key set of query i of (b, h) (i = 0 for decode). Decode: the prefix (or routed
+// blocks) and the ring's valid slots. Chunked prefill: the routed blocks, the outputs
+// j with i - n < j <= i of the chunk (the band) and, for j < 0, the previous chunk's
+// last outputs from the ring: the min(n - 1 - i, fill) most recently written slots.
 template <bool kSparse, bool kFp8>
-__device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, bool report) {
+__device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, int i, bool report) {
   SeqView v;
   const int64_t bh = (int64_t)b * a.H + h;
+  const bool band = a.k_out != nullptr;
   int m = a.prefix_len[b];
   if (m < 0 || m > a.cap) {
     if (report) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
     m = 0;
   }
-  int w = a.wp[b], f = a.fill[b];
-  if (w < 0 || w >= a.n || f < 0 || f > a.n) {
-    if (report) set_status(a.status, RSWA_DEVICE_BAD_RING_STATE);
-    w = 0;
-    f = 0;
+  int w = 0, f = 0;
+  if (a.ring_k != nullptr) {
+    w = a.wp[b];
+    f = a.fill[b];
+    if (w < 0 || w >= a.n || f < 0 || f > a.n) {
+      if (report) set_status(a.status, RSWA_DEVICE_BAD_RING_STATE);
+      w = 0;
+      f = 0;
+    }
   }
   if (kFp8) {
     v.pk = a.pk8 + bh * a.cap * kHeadDim;
@@ -111,20 +123,31 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
     v.pv = reinterpret_cast<const uint8_t*>(a.pv + bh * a.cap * kHeadDim);
     v.ks = v.vs = nullptr;
   }
-  v.rk = a.ring_k + bh * a.n * kHeadDim;
-  v.rv = a.ring_v + bh * a.n * kHeadDim;
+  v.rk = a.ring_k ? a.ring_k + bh * a.n * kHeadDim : nullptr;
+  v.rv = a.ring_v ? a.ring_v + bh * a.n * kHeadDim : nullptr;
   v.m = m;
   v.nb = (m + kBlock - 1) / kBlock;
-  // valid slots are (w - f + i) mod n, i < f; a full ring is read as [0, n)
-  int a0 = f == a.n ? 0 : (w - f) % a.n;
+  int cnt = f;  // ring slots read: the cnt most recently written, (w - cnt + i) mod n for i < cnt
+  if (band) cnt = min(max(a.n - 1 - i, 0), f);
+  // a full ring is read as [0, n)
+  int a0 = cnt == a.n ? 0 : (w - cnt) % a.n;
   if (a0 < 0) a0 += a.n;
   v.a0 = a0;
-  v.len0 = min(f, a.n - a0);
-  v.len1 = f - v.len0;
+  v.len0 = min(cnt, a.n - a0);
+  v.len1 = cnt - v.len0;
   v.n_r0 = (v.len0 + kBlock - 1) / kBlock;
   v.n_r1 = (v.len1 + kBlock - 1) / kBlock;
   v.n_first = kSparse ? a.topk : v.nb;
-  v.total = v.n_first + v.n_r0 + v.n_r1;
+  v.bk = v.bv = nullptr;
+  v.blen = v.n_band = 0;
+  if (band) {
+    const int start = max(0, i - a.n + 1);
+    v.blen = i - start + 1;
+    v.n_band = (v.blen + kBlock - 1) / kBlock;
+    v.bk = a.k_out + (bh * a.T + start) * kHeadDim;
+    v.bv = a.v_out + (bh * a.T + start) * kHeadDim;
+  }
+  v.total = v.n_first + v.n_r0 + v.n_r1 + v.n_band;
   return v;
 }
 
@@ -169,6 +192,13 @@ __device__ __forceinline__ TileRef tile_at(const SeqView& v, int t, int c, float
     return r;
   }
   t -= v.n_first;
+  if (t >= v.n_r0 + v.n_r1) {  // the causal band of a chunked-prefill query
+    t -= v.n_r0 + v.n_r1;
+    r.rows = min(kBlock, v.blen - t * kBlock);
+    r.k = reinterpret_cast<const uint8_t*>(v.bk + (int64_t)t * kBlock * kHeadDim);
+    r.v = reinterpret_cast<const uint8_t*>(v.bv + (int64_t)t * kBlock * kHeadDim);
+    return r;
+  }
   int start, len;
   if (t < v.n_r0) {
     start = v.a0 + t * kBlock;
@@ -194,18 +224,21 @@ struct ItemView {
   float lp;
 };
 
+// Items are (query, split) with query vq = (b * H + h) * T + i.
 template <bool kSparse, bool kFp8>
 __device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lane, ItemView& iv) {
-  const int bh = item / a.splits, split = item - bh * a.splits;
+  const int vq = item / a.splits, split = item - vq * a.splits;
+  const int bh = vq / a.T, i = vq - bh * a.T;
   const int b = bh / a.H, h = bh - b * a.H;
   iv.item = item;
   iv.t0 = split * a.tiles_per_item;
-  iv.v = make_view<kSparse, kFp8>(a, b, h, lane == 0 && split == 0 && h == 0);
+  iv.v = make_view<kSparse, kFp8>(a, b, h, i, lane == 0 && split == 0 && h == 0 && i == 0);
   iv.c = -1;
   iv.lp = -INFINITY;
   if (kSparse && lane < a.topk) {
-    iv.c = a.blk_idx[(int64_t)b * a.topk + lane];
-    iv.lp = a.blk_logp[(int64_t)b * a.topk + lane];
+    const int64_t ri = ((int64_t)b * a.T + i) * a.topk + lane;  // the route of query i of sequence b
+    iv.c = a.blk_idx[ri];
+    iv.lp = a.blk_logp[ri];
   }
 }
 
@@ -393,7 +426,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
     q_next = *reinterpret_cast<const uint4*>(a.q + (int64_t)(blockIdx.x / a.splits) * kHeadDim + c * 8);
   int li_base = 0;
   for (int item = blockIdx.x; item < a.items; item += gridDim.x, li_base += P) {
-    const int bh = item / a.splits, split = item - bh * a.splits;
+    // vq: the item's query, (b * H + h) * T + i; q, out, lse and the split partials are per query
+    const int vq = item / a.splits, split = item - vq * a.splits;
     const uint4 q_cur = q_next;
     if (item + (int)gridDim.x < a.items)
       q_next = *reinterpret_cast<const uint4*>(a.q + (int64_t)((item + gridDim.x) / a.splits) * kHeadDim + c * 8);
@@ -478,11 +512,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
         float A = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) A = fmaf(sm.wacc[w][d], fw[w], A);
-        a.out[(int64_t)bh * kHeadDim + d] = L > 0.f ? A / L : 0.f;
+        a.out[(int64_t)vq * kHeadDim + d] = L > 0.f ? A / L : 0.f;
       }
-      if (tid == 0 && a.lse) a.lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+      if (tid == 0 && a.lse) a.lse[vq] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     } else {
-      float* rec = a.partials + ((int64_t)bh * a.splits + split) * (kHeadDim + 2);
+      float* rec = a.partials + ((int64_t)vq * a.splits + split) * (kHeadDim + 2);
       for (int d = tid; d < kHeadDim; d += kDecodeThreads) {
         float A = 0.f;
 #pragma unroll
@@ -495,11 +529,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
       }
       __threadfence();
       __syncthreads();
-      if (tid == 0) sm.is_last = (atomicAdd(&a.counters[bh], 1) == a.splits - 1);
+      if (tid == 0) sm.is_last = (atomicAdd(&a.counters[vq], 1) == a.splits - 1);
       __syncthreads();
       if (sm.is_last) {
         __threadfence();
-        const float* recs = a.partials + (int64_t)bh * a.splits * (kHeadDim + 2);
+        const float* recs = a.partials + (int64_t)vq * a.splits * (kHeadDim + 2);
         float Mg = -INFINITY;
         for (int s = 0; s < a.splits; ++s) Mg = fmaxf(Mg, __ldcg(recs + s * (kHeadDim + 2)));
         float Lg = 0.f;
@@ -515,11 +549,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
               const float* r = recs + s * (kHeadDim + 2);
               Ag = fmaf(__ldcg(r + 2 + d), exp2f(__ldcg(r) - Mg), Ag);
             }
-          a.out[(int64_t)bh * kHeadDim + d] = Lg > 0.f ? Ag / Lg : 0.f;
+          a.out[(int64_t)vq * kHeadDim + d] = Lg > 0.f ? Ag / Lg : 0.f;
         }
         if (tid == 0) {
-          if (a.lse) a.lse[bh] = Lg > 0.f ? (Mg + log2f(Lg)) * kLn2 : -INFINITY;
-          a.counters[bh] = 0;
+          if (a.lse) a.lse[vq] = Lg > 0.f ? (Mg + log2f(Lg)) * kLn2 : -INFINITY;
+          a.counters[vq] = 0;
         }
       }
     }
@@ -538,6 +572,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
 }
 
 }  // namespace
+
+int decode_ctas_per_sm() { return kDecodeMinBlocks; }
 
 int64_t decode_max_tiles_dense(int64_t cap, int n) {
   return (cap + kBlock - 1) / kBlock + (n + kBlock - 1) / kBlock + 1;

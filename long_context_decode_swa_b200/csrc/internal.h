@@ -38,6 +38,11 @@ struct DecodeArgs {
   const float* vscale;
   int64_t nb_cap;
   int fp8;
+  // SR-SWA chunked prefill: T queries per (sequence, head) and the chunk's output K/V
+  // [B][H][T][D], read as each query's causal band; T = 1 and k_out = null for decode
+  int T;
+  const uint16_t* k_out;
+  const uint16_t* v_out;
 };
 
 // Workspace layout shared by every op: [status: 256 B][counters][partials].
@@ -50,6 +55,7 @@ struct WorkspacePlan {
 // max_bytes > 0 restricts the split count to plans whose workspace fits that many bytes.
 WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_count, size_t max_bytes = 0);
 int64_t decode_max_tiles_dense(int64_t cap, int n);
+int decode_ctas_per_sm();  // resident decode CTAs per SM (shared-memory bound)
 int64_t decode_max_tiles_sparse(int topk, int n);
 int device_sm_count();
 
@@ -64,9 +70,10 @@ cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const i
                               cudaStream_t stream);
 // CTAs per sequence of the router (its thread-block cluster size).
 int route_cluster_size(int64_t cap);
-cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
-                         float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                         int32_t* status, cudaStream_t stream);
+// tokens: router queries per sequence (q_idx [B][tokens][32], outputs [B][tokens][topk])
+cudaError_t launch_route(int B, int tokens, int64_t cap, const float* q_idx, const float* kbar,
+                         const int32_t* prefix_len, float idx_scale, int topk, int32_t* blk_idx, float* blk_logp,
+                         float* probs, float* tau, int32_t* status, cudaStream_t stream);
 
 struct PrefillLaunch {
   int B, H, n, T;

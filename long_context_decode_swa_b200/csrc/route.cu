@@ -135,6 +135,7 @@ __host__ __device__ __forceinline__ int route_sort_capacity(int csize) {
 
 struct RouteArgs {
   int64_t cap;
+  int tokens;  // router queries per sequence: 1 (decode) or the chunk length (per-token prefill routing)
   int nb_cap, csize, topk;  // csize: CTAs per sequence (the cluster size)
   float idx_scale;
   const float* q_idx;
@@ -193,7 +194,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
 
-  const int rank = (int)cluster.block_rank(), b = blockIdx.y;
+  // blockIdx.y is the router query: (sequence b, token t) with t < a.tokens (1 for decode)
+  const int rank = (int)cluster.block_rank(), row = blockIdx.y, b = row / a.tokens;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int region = kRouteThreads * 2;  // blocks per CTA
   // on CTA 0: what CTA r sends lands at [r * region, ...) of (cand_z, cand_i); the union
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   {
     const int o = lane >> 3, j = lane & 7;
     const int wbase = rank * region + warp * 64;
-    const float4 qv = reinterpret_cast<const float4*>(a.q_idx + (int64_t)b * kIndexDim)[j];
+    const float4 qv = reinterpret_cast<const float4*>(a.q_idx + (int64_t)row * kIndexDim)[j];
     const float4* k4 = reinterpret_cast<const float4*>(a.kbar + (int64_t)b * a.nb_cap * kIndexDim);
     float4 kv[16];
 #pragma unroll
@@ -271,12 +273,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   if (NB == 0) {  // uniform over the cluster: no barrier is reached
     if (rank == 0) {
       if (tid < a.topk) {
-        a.blk_idx[(int64_t)b * a.topk + tid] = -1;
-        a.blk_logp[(int64_t)b * a.topk + tid] = -INFINITY;
+        a.blk_idx[(int64_t)row * a.topk + tid] = -1;
+        a.blk_logp[(int64_t)row * a.topk + tid] = -INFINITY;
       }
       if (a.probs)
-        for (int c = tid; c < a.nb_cap; c += kRouteThreads) a.probs[(int64_t)b * a.nb_cap + c] = 0.f;
-      if (a.tau && tid == 0) a.tau[b] = NAN;
+        for (int c = tid; c < a.nb_cap; c += kRouteThreads) a.probs[(int64_t)row * a.nb_cap + c] = 0.f;
+      if (a.tau && tid == 0) a.tau[row] = NAN;
     }
     return;
   }
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
           const float r = fmaf(z[s2], 0.5f, -s_xmax) - s_tau_y;
           pr = r > 0.f ? r * r : 0.f;
         }
-        a.probs[(int64_t)b * a.nb_cap + c] = pr;
+        a.probs[(int64_t)row * a.nb_cap + c] = pr;
       }
     }
     return;
@@ -496,9 +498,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
 #pragma unroll
   for (int w = 0; w < kRouteWarps; ++w) best = max(best, red_i[w]);
   const float tau_y = best > 0 ? tau_r[best - 1] : 0.f;
-  if (a.tau && tid == 0) a.tau[b] = tau_y + xmax;
+  if (a.tau && tid == 0) a.tau[row] = tau_y + xmax;
   if (tid < a.topk) {
-    const int64_t o = (int64_t)b * a.topk + tid;
+    const int64_t o = (int64_t)row * a.topk + tid;
     const int bi = tid < n_u ? oi[tid] : kNone;
     if (bi == kNone) {
       a.blk_idx[o] = -1;
@@ -527,7 +529,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
           const float r = fmaf(z[s2i], 0.5f, -xmax) - tau_y;
           pr = r > 0.f ? r * r : 0.f;
         }
-        a.probs[(int64_t)b * a.nb_cap + c] = pr;
+        a.probs[(int64_t)row * a.nb_cap + c] = pr;
       }
     }
   }
@@ -549,11 +551,12 @@ int route_cluster_size(int64_t cap) {
   return (nb_cap + per - 1) / per;
 }
 
-cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kbar, const int32_t* prefix_len,
-                         float idx_scale, int topk, int32_t* blk_idx, float* blk_logp, float* probs, float* tau,
-                         int32_t* status, cudaStream_t stream) {
+cudaError_t launch_route(int B, int tokens, int64_t cap, const float* q_idx, const float* kbar,
+                         const int32_t* prefix_len, float idx_scale, int topk, int32_t* blk_idx, float* blk_logp,
+                         float* probs, float* tau, int32_t* status, cudaStream_t stream) {
   RouteArgs a;
   a.cap = cap;
+  a.tokens = tokens;
   a.nb_cap = (int)((cap + kBlock - 1) / kBlock);
   a.csize = route_cluster_size(cap);
   a.topk = topk;
@@ -574,7 +577,7 @@ cudaError_t launch_route(int B, int64_t cap, const float* q_idx, const float* kb
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
-  fill_launch_config(cfg, attr, dim3(a.csize, B), dim3(kRouteThreads), smem, stream);
+  fill_launch_config(cfg, attr, dim3(a.csize, B * tokens), dim3(kRouteThreads), smem, stream);
   attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
   attr[cfg.numAttrs].val.clusterDim.x = a.csize;
   attr[cfg.numAttrs].val.clusterDim.y = 1;
