@@ -8,6 +8,7 @@ A step is one decode step of the whole batch through the C ABI:
   configs 4, 5 (SR-SWA):  rswa_append + srswa_route + srswa_decode
   configs 6, 7:           configs 2 and 4 over an FP8 (E4M3) prefix, quantised
                           once before timing (rswa_decode_fp8 / srswa_decode_fp8)
+  config 8 (SR-SWA chunked prefill): srswa_route_tokens + srswa_prefill
 (the router's block index keys are pooled once per prefix, before timing).
 The default workload is the batched R-SWA decode: 512 sequences, 16 heads,
 head_dim 128, a 10-page prefix (2560 visual + 32 prompt tokens) and a full
@@ -79,6 +80,11 @@ def workload(cfg: int) -> dict:
         return dict(kind="srswa", B=16, H=16, D=128, n=128, plen=plen, cap=102400, wp0=None,
                     name="SR-SWA long-horizon decode, 16 sequences, 16 heads, head_dim 128, ragged histories "
                          "8192-102400 tokens (log-uniform pages x 256), top-16 blocks + 128-slot ring")
+    if cfg == 8:
+        return dict(kind="srswa_prefill", B=4, H=16, D=128, n=128, plen=[32768] * 4, cap=32768, T=4096, wp0=None,
+                    name="SR-SWA chunked prefill, 4 sequences, 16 heads, head_dim 128, 32768-token history (1024 "
+                         "blocks), 4096 output-side queries each routed to its own top-16 blocks (planted, 32 "
+                         "directions cycled over the tokens) + causal band 128")
     if cfg in (6, 7):  # the batched R-SWA and the 32K-history SR-SWA workloads over an FP8 (E4M3) prefix
         w = workload(2 if cfg == 6 else 4)
         w["fp8"] = True
@@ -93,6 +99,21 @@ def prefill_flops(w: dict) -> float:
     T, n, D, H = w["T"], w["n"], w["D"], w["H"]
     band = sum(min(n, i + 1) for i in range(T))
     return float(sum(4 * D * (m * T + band) for m in w["plen"]) * H)
+
+
+def srswa_prefill_flops(w: dict, blk, logp) -> float:
+    """FLOPs of the SR-SWA prefill attention: per (b, h) and query t, 4 x 128 x (the valid rows of
+    its routed blocks with finite bias + its band min(n, t + 1))."""
+    import numpy as np
+    T, n, D, H = w["T"], w["n"], w["D"], w["H"]
+    total = 0
+    for b, m in enumerate(w["plen"]):
+        c = blk[b].astype(np.int64)
+        ok = (c >= 0) & np.isfinite(logp[b])
+        rows = np.where(ok, np.minimum(32, m - 32 * c), 0).sum()
+        band = sum(min(n, t + 1) for t in range(T))
+        total += 4 * D * (int(rows) + band)
+    return float(total * H)
 
 
 def algorithmic_bytes(w: dict, blk_rows=None) -> dict:
@@ -363,6 +384,54 @@ class PrefillProblem:
         return 1
 
 
+class SrswaPrefillProblem:
+    """SR-SWA chunked prefill: a step is srswa_route_tokens (every query routed) + srswa_prefill."""
+
+    def __init__(self, w: dict, seed: int):
+        import torch
+
+        import long_context_decode_swa_b200 as rswa
+        from long_context_decode_swa_b200 import synth
+        self.rswa = rswa
+        self.w = w
+        B, H, T = w["B"], w["H"], w["T"]
+        self.d = synth.prefill_case(B, H, w["D"], w["plen"], w["cap"], T, seed=seed, device="cuda", poison=False)
+        pl = synth.plant_router_keys(w["plen"], w["cap"], n_dirs=32, seed=seed + 1, device="cuda")
+        nb_cap = (w["cap"] + 31) // 32
+        self.kbar = torch.empty((B, nb_cap, 32), dtype=torch.float32, device="cuda")
+        rswa.srswa_index_pool(pl.k_idx, self.d["prefix_len"], self.kbar)
+        self.q_tok = pl.q_idx[torch.arange(T, device="cuda") % 32].permute(1, 0, 2).contiguous()   # [B][T][32]
+        del pl
+        self.blk = torch.empty((B, T, 16), dtype=torch.int32, device="cuda")
+        self.logp = torch.empty((B, T, 16), dtype=torch.float32, device="cuda")
+        self.out = torch.empty((B, H, T, w["D"]), dtype=torch.float32, device="cuda")
+        self.lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+        self.ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        self.sparse = True
+        torch.cuda.synchronize()
+
+    def step(self, i: int, q=None, k_new=None, v_new=None, ev=None):
+        d, r = self.d, self.rswa
+        if ev is not None:
+            ev[2].record()
+        r.srswa_route_tokens(self.q_tok, self.kbar, d["prefix_len"], self.blk, self.logp, self.ws,
+                             prefix_cap=self.w["cap"])
+        if ev is not None:
+            ev[3].record()
+            ev[0].record()
+        r.srswa_prefill(d["q"] if q is None else q, d["k_out"] if k_new is None else k_new,
+                        d["v_out"] if v_new is None else v_new, d["pk"], d["pv"], d["prefix_len"], self.blk,
+                        self.logp, self.out, self.ws, lse=self.lse, scale=d["scale"], ring=self.w["n"])
+        if ev is not None:
+            ev[1].record()
+        return 2
+
+
+def alu_peak_tflops() -> float:
+    """FP32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the recipe's SM count and max clock)."""
+    return 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def measured_tensor_peak(sustained: bool):
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -375,7 +444,7 @@ def measured_tensor_peak(sustained: bool):
 def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     import torch
     K, W = args.steps, args.warmup
-    if w["kind"] == "prefill":
+    if w["kind"] in ("prefill", "srswa_prefill"):
         return run_prefill(args, w, world, rank, local)
     prob = Problem(w, K + W, seed=1000 * args.config + rank)
     stream = torch.cuda.Stream()
@@ -485,14 +554,15 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
 def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
     import torch
     K, W = args.steps, args.warmup
-    prob = PrefillProblem(w, seed=1000 * args.config + rank)
+    sparse = w["kind"] == "srswa_prefill"
+    prob = (SrswaPrefillProblem if sparse else PrefillProblem)(w, seed=1000 * args.config + rank)
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         for i in range(W):
             prob.step(i)
     stream.synchronize()
     sampled = list(range(0, K, EVENT_EVERY))
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in sampled]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4 if sparse else 2)] for _ in sampled]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(K):
@@ -519,10 +589,15 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
     ms_total = start.elapsed_time(end)
     ms_max = max_over_ranks(world, ms_total)
     kern_s = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    route_s = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) / 1e3 if sparse else 0.0
     del graph
-    flops = prefill_flops(w)
-    sustained = ms_total > 1000.0
-    peak, src = measured_tensor_peak(sustained)
+    if sparse:
+        flops = srswa_prefill_flops(w, prob.blk.cpu().numpy(), prob.logp.cpu().numpy())
+        peak, src = alu_peak_tflops(), "derived"
+    else:
+        flops = prefill_flops(w)
+        sustained = ms_total > 1000.0
+        peak, src = measured_tensor_peak(sustained)
     achieved = flops / kern_s / 1e12
     e2e = run_prefill_e2e(prob, K, W) if not args.no_e2e else {"ms": float("nan"), "h2d": 0, "d2h": 0}
     e2e_ms = max_over_ranks(world, e2e["ms"])
@@ -531,19 +606,26 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
     return {
         "metric": METRIC, "value": value, "unit": "prefill chunks/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "dtype": "f32" if sparse else "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
         "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "heads": H,
                    "head_dim": w["D"], "ring": w["n"], "chunk": T, "prefix_tokens_mean": statistics.mean(w["plen"]),
                    "parallelism": f"replicas x{world}", "timing": "K launches in one CUDA graph replay, CUDA events; kernel durations from "
                              f"event brackets in every {EVENT_EVERY}th step"},
         "qtok_per_s": value * B * H * T,
-        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (tcgen05)", "achieved": achieved, "peak": peak,
-                     "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)",
-                     "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": committed_traffic(f"rswa_prefill_config{args.config}", kernel_source_hash("prefill")),
-                     "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6},
-        "kernels_us": {"prefill": kern_s * 1e6},
-        "gpu_launches": K,
+        "roofline": ({"bound": "alu", "kernel": "srswa decode_kernel<true, bf16> (chunked-prefill queries)",
+                      "achieved": achieved, "peak": peak,
+                      "peak_source": "derived: FP32 FMA, 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (no measured ALU "
+                                     "peak); gathered rows mostly hit L2",
+                      "unit": "TFLOP/s", "frac": achieved / peak,
+                      "traffic": committed_traffic(f"srswa_prefill_config{args.config}", kernel_source_hash("sparse")),
+                      "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6} if sparse else
+                     {"bound": "tensor", "kernel": "prefill_kernel (tcgen05)", "achieved": achieved, "peak": peak,
+                      "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)",
+                      "unit": "TFLOP/s", "frac": achieved / peak,
+                      "traffic": committed_traffic(f"rswa_prefill_config{args.config}", kernel_source_hash("prefill")),
+                      "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6}),
+        "kernels_us": {"prefill": kern_s * 1e6, **({"route": route_s * 1e6} if sparse else {})},
+        "gpu_launches": K * (2 if sparse else 1),
         "clocks": clk,
         "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "prefill chunks/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
@@ -669,8 +751,58 @@ def oracle_step(st: dict, w: dict):
                                st["rv"], st["wp"], st["fill"], st["scale"])
 
 
+PREFILL_ORACLE_ROWS = 64  # query rows per sampled sequence in the prefill oracle arms
+
+
+def oracle_prefill_case(w: dict, sample: int, seed: int):
+    """Host inputs of `sample` sequences of a prefill workload, PREFILL_ORACLE_ROWS rows each
+    (evenly spaced over the chunk), and the work fraction they stand for."""
+    import numpy as np
+
+    import oracle
+    from long_context_decode_swa_b200 import synth
+    plen = w["plen"][:sample]
+    d = synth.prefill_case(sample, w["H"], w["D"], plen, w["cap"], w["T"], seed=seed, poison=False)
+    u = synth.to_u16
+    st = dict(q=u(d["q"]), k=u(d["k_out"]), v=u(d["v_out"]), pk=u(d["pk"]), pv=u(d["pv"]),
+              plen=d["prefix_len"].numpy(), scale=d["scale"])
+    rows = np.unique(np.linspace(0, w["T"] - 1, PREFILL_ORACLE_ROWS).astype(np.int32))
+    st["rows"] = rows
+    if w["kind"] == "srswa_prefill":
+        pl = synth.plant_router_keys(plen, w["cap"], n_dirs=32, seed=seed + 1)
+        kbar = oracle.index_pool(u(pl.k_idx), st["plen"])
+        q_tok = pl.q_idx.numpy()[rows % 32].transpose(1, 0, 2).copy()          # routes of the sampled rows
+        b_rows, l_rows = oracle.route_tokens(q_tok, kbar, st["plen"])
+        st["blk"] = np.full((sample, w["T"], 16), -1, np.int32)
+        st["logp"] = np.full((sample, w["T"], 16), -np.inf)
+        st["blk"][:, rows], st["logp"][:, rows] = b_rows, l_rows
+        st["q_tok"], st["kbar"] = q_tok, kbar
+    return st, (sample / w["B"]) * (len(rows) / w["T"])
+
+
+def oracle_prefill_step(st: dict, w: dict):
+    import oracle
+    if w["kind"] == "srswa_prefill":
+        st["blk_rows"] = oracle.route_tokens(st["q_tok"], st["kbar"], st["plen"])      # the step's routing
+        return oracle.srswa_prefill(st["q"], st["k"], st["v"], st["pk"], st["pv"], st["plen"], st["blk"],
+                                    st["logp"], st["scale"], st["rows"], w["n"])
+    return oracle.rswa_prefill(st["q"], st["k"], st["v"], st["pk"], st["pv"], st["plen"], st["scale"], st["rows"],
+                               w["n"])
+
+
 def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
     import oracle
+    if w["kind"] in ("prefill", "srswa_prefill"):
+        st, frac = oracle_prefill_case(w, 1, seed=77)
+        oracle_prefill_step(st, w)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 1 or (time.perf_counter() - t0 < budget_s and reps < 20):
+            oracle_prefill_step(st, w)
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+        return {"value": frac / dt, "unit": "prefill chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
+                "sample": f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows (all heads), "
+                          f"{reps} steps timed; chunks/s extrapolated by the sample fraction; fp64 C oracle"}
     sample = min(w["B"], 2)
     st = oracle_sample_step(w, sample, seed=77)
     oracle_step(st, w)                               # warm (and pool the router keys)
@@ -695,6 +827,24 @@ def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
 def run_reference(args, w: dict) -> dict:
     """The oracle as the reference arm, on the host cores, K timed steps of a bounded sample."""
     import oracle
+    if w["kind"] in ("prefill", "srswa_prefill"):
+        st, frac = oracle_prefill_case(w, 1, seed=99)
+        for _ in range(args.warmup):
+            oracle_prefill_step(st, w)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_prefill_step(st, w)
+        value = frac / ((time.perf_counter() - t0) / args.steps)
+        cb = {"value": value, "unit": "prefill chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
+              "sample": f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows per step (all heads); "
+                        f"chunks/s extrapolated by the sample fraction; fp64 C oracle on the host cores"}
+        return {"metric": METRIC, "value": value, "unit": "prefill chunks/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": w["B"]},
+                "cpu_baseline": cb,
+                "e2e": {"value": value, "unit": "prefill chunks/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2}.get(args.config, 1))
     st = oracle_sample_step(w, sample, seed=99)
     for _ in range(args.warmup):
@@ -750,7 +900,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
