@@ -256,6 +256,31 @@ RSWA_API rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, c
                                          int32_t* status, void* stream);
 
 /*
+ * One decode step in one launch: rswa_append followed by rswa_decode (respectively
+ * srswa_decode), fused. This step's token joins the key set straight from k_new / v_new
+ * (its own key, as after an append), the oldest slot of a full ring is left out, the
+ * token is written into ring slot wp[b] (slot_out[b] <- wp[b]), and wp / fill advance
+ * as rswa_append advances them once the launch has read them. Same results as the two
+ * calls; one kernel boundary fewer per step.
+ * Arguments: those of rswa_append and rswa_decode (srswa_decode), with the ring, wp and
+ * fill writable. workspace: rswa_workspace_bytes(dims, RSWA_OP_DECODE) (resp.
+ * RSWA_OP_SRSWA_DECODE), zero-initialised; bytes 128..131 of its status area hold the
+ * launch's completion counter, which every launch leaves at zero.
+ * A sequence whose wp / fill are out of range is flagged (RSWA_DEVICE_BAD_RING_STATE)
+ * and left untouched, its ring read as empty and its new token not attended.
+ */
+RSWA_API rswa_status rswa_decode_append(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new,
+                                        const void* pk, const void* pv, const int32_t* prefix_len, void* ring_k,
+                                        void* ring_v, int32_t* wp, int32_t* fill, int32_t* slot_out, float scale,
+                                        float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+RSWA_API rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new,
+                                         const void* pk, const void* pv, const int32_t* prefix_len,
+                                         const int32_t* blk_idx, const float* blk_logp, int32_t topk, void* ring_k,
+                                         void* ring_v, int32_t* wp, int32_t* fill, int32_t* slot_out, float scale,
+                                         float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * SR-SWA chunked prefill (the survey's next row 1). The pages size prefill memory by a
  * per-token router score tensor of about [tokens, context/32] (serving notes,
  * --max-prefill-tokens), i.e. every output-side token of a chunk is routed by itself;

@@ -6,12 +6,14 @@ seeded synthetic-input generators. There is no CPU fallback.
 """
 from .binding import (  # noqa: F401
     EXPORTED, LIB_PATH, OP_DECODE, OP_PREFILL, OP_ROUTE, OP_SRSWA_DECODE, Dims, RswaError, check_status, dims_of,
-    fp8_prefix_buffers, load, new_workspace, route_workspace, rswa_append, rswa_decode, rswa_decode_fp8, rswa_prefill,
-    rswa_quantize_prefix, srswa_decode, srswa_decode_fp8, srswa_index_pool, srswa_prefill, srswa_route,
+    fp8_prefix_buffers, load, new_workspace, route_workspace, rswa_append, rswa_decode, rswa_decode_append,
+    rswa_decode_fp8, rswa_prefill,
+    rswa_quantize_prefix, srswa_decode, srswa_decode_append, srswa_decode_fp8, srswa_index_pool, srswa_prefill,
+    srswa_route,
     srswa_route_tokens, workspace_bytes,
 )
 
 __all__ = ["load", "Dims", "RswaError", "rswa_append", "rswa_decode", "rswa_prefill", "srswa_index_pool", "srswa_route",
            "srswa_decode", "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "fp8_prefix_buffers",
-           "srswa_route_tokens", "srswa_prefill",
+           "srswa_route_tokens", "srswa_prefill", "rswa_decode_append", "srswa_decode_append",
            "workspace_bytes", "new_workspace", "route_workspace", "check_status", "dims_of"]

@@ -36,7 +36,8 @@ DEVICE_PIPELINE = 0x10
 
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
             "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill",
-            "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill")
+            "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill",
+            "rswa_decode_append", "srswa_decode_append")
 
 
 class RswaError(RuntimeError):
@@ -95,6 +96,9 @@ def load(path: str | None = None):
             "srswa_decode_fp8": ([DP, P, P, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_route_tokens": ([DP, I32, P, P, P, F32, I32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_prefill": ([DP, I32, P, P, P, P, P, P, P, P, I32, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "rswa_decode_append": ([DP, P, P, P, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_decode_append": ([DP, P, P, P, P, P, P, P, P, I32, P, P, P, P, P, F32, P, P, P, SZ, P],
+                                    ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -351,6 +355,70 @@ def srswa_decode_fp8(q, pk8, pv8, k_scale, v_scale, prefix_len, blk_idx, blk_log
                                                        _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(out),
                                                        _ptr(lse), _ptr(workspace), workspace.numel(),
                                                        _stream(stream)))
+
+
+def rswa_decode_append(q, k_new, v_new, pk, pv, prefix_len, ring_k, ring_v, wp, fill, out, workspace, lse=None,
+                       slot_out=None, scale=None, stream=None):
+    """rswa_append + rswa_decode in one launch (same results; wp / fill / ring updated)."""
+    B, H, cap, D = pk.shape
+    n = ring_k.shape[2]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("rswa_decode_append", load().rswa_decode_append(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                                           _ptr(pk), _ptr(pv), _ptr(prefix_len), _ptr(ring_k),
+                                                           _ptr(ring_v), _ptr(wp), _ptr(fill), _ptr(slot_out), scale,
+                                                           _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                                           _stream(stream)))
+
+
+def srswa_decode_append(q, k_new, v_new, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, out,
+                        workspace, lse=None, slot_out=None, scale=None, stream=None):
+    """rswa_append + srswa_decode in one launch (same results; wp / fill / ring updated)."""
+    B, H, cap, D = pk.shape
+    n = ring_k.shape[2]
+    topk = blk_idx.shape[1]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, topk))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_decode_append", load().srswa_decode_append(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                                             _ptr(pk), _ptr(pv), _ptr(prefix_len), _ptr(blk_idx),
+                                                             _ptr(blk_logp), topk, _ptr(ring_k), _ptr(ring_v),
+                                                             _ptr(wp), _ptr(fill), _ptr(slot_out), scale, _ptr(out),
+                                                             _ptr(lse), _ptr(workspace), workspace.numel(),
+                                                             _stream(stream)))
 
 
 def srswa_route_tokens(q_idx, kbar, prefix_len, blk_idx, blk_logp, workspace, idx_scale=1.0, prefix_cap=None,

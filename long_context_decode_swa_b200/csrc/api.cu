@@ -81,20 +81,28 @@ size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
   const char* fn = "rswa_workspace_bytes";
   if (check_dims(fn, dims, true) != RSWA_OK) return 0;
   switch (op) {
-    case RSWA_OP_DECODE:
-      return rswa::plan_decode_workspace(dims->batch, dims->heads, rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring),
-                                         rswa::device_sm_count())
-          .bytes;
-    case RSWA_OP_SRSWA_DECODE: {
-      // the plan depends on topk: size for the largest plan over every allowed topk
+    case RSWA_OP_DECODE: {
+      // sized for rswa_decode and for the fused rswa_decode_append (one tile more)
+      const int64_t t = rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring);
       size_t most = 0;
-      for (int k = 1; k <= rswa::kMaxTopk; ++k) {
-        const size_t b = rswa::plan_decode_workspace(dims->batch, dims->heads,
-                                                     rswa::decode_max_tiles_sparse(k, dims->ring),
-                                                     rswa::device_sm_count())
-                             .bytes;
+      for (int64_t extra = 0; extra <= 1; ++extra) {
+        const size_t b =
+            rswa::plan_decode_workspace(dims->batch, dims->heads, t + extra, rswa::device_sm_count()).bytes;
         most = b > most ? b : most;
       }
+      return most;
+    }
+    case RSWA_OP_SRSWA_DECODE: {
+      // the plan depends on topk (and the fused append's extra tile): size for the largest
+      size_t most = 0;
+      for (int k = 1; k <= rswa::kMaxTopk; ++k)
+        for (int64_t extra = 0; extra <= 1; ++extra) {
+          const size_t b = rswa::plan_decode_workspace(dims->batch, dims->heads,
+                                                       rswa::decode_max_tiles_sparse(k, dims->ring) + extra,
+                                                       rswa::device_sm_count())
+                               .bytes;
+          most = b > most ? b : most;
+        }
       return most;
     }
     case RSWA_OP_ROUTE:
@@ -162,9 +170,22 @@ struct BandSrc {
 };
 constexpr BandSrc kNoBand{1, nullptr, nullptr};
 
+// Fused ring append: this step's K / V join the ring inside the decode launch.
+struct AppendSrc {
+  const void* k_new;
+  const void* v_new;
+  void* ring_k;  // the same ring as the decode reads, writable
+  void* ring_v;
+  int32_t* wp;
+  int32_t* fill;
+  int32_t* slot_out;
+};
+constexpr AppendSrc kNoAppend{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+constexpr size_t kGridCounterOffset = 128;  // an int32 inside the workspace's 256-byte status area
+
 // plan_budget > 0: plan the split-KV work to fit a workspace of that many bytes.
 static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, PrefixSrc px,
-                                 BandSrc band, const int32_t* prefix_len, const int32_t* blk_idx,
+                                 BandSrc band, AppendSrc app, const int32_t* prefix_len, const int32_t* blk_idx,
                                  const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                                  const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0) {
@@ -203,6 +224,12 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   }
   REQUIRE_PTR(out);
   REQUIRE_PTR(workspace);
+  if (app.k_new != nullptr) {
+    const void* k_new = app.k_new;
+    const void* v_new = app.v_new;
+    REQUIRE_PTR(k_new);
+    REQUIRE_PTR(v_new);
+  }
   if (sparse) {
     if (blk_idx == nullptr || blk_logp == nullptr)
       return fail(RSWA_ERR_INVALID, "%s: blk_idx and blk_logp must not be NULL", fn);
@@ -211,6 +238,7 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
   int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(topk, dims->ring)
                              : rswa::decode_max_tiles_dense(dims->prefix_cap, dims->ring);
+  if (app.k_new != nullptr) max_tiles += 1;  // this step's token
   rswa::WorkspacePlan plan;
   if (prefill) {
     // ring part and band together cover n keys in at most three ranges: two tiles beyond a decode's
@@ -252,6 +280,14 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.T = prefill ? band.T : 1;
   a.k_out = static_cast<const uint16_t*>(band.k_out);
   a.v_out = static_cast<const uint16_t*>(band.v_out);
+  a.k_new = static_cast<const uint16_t*>(app.k_new);
+  a.v_new = static_cast<const uint16_t*>(app.v_new);
+  a.ring_k_w = static_cast<uint16_t*>(app.ring_k);
+  a.ring_v_w = static_cast<uint16_t*>(app.ring_v);
+  a.wp_w = app.wp;
+  a.fill_w = app.fill;
+  a.slot_out = app.slot_out;
+  a.grid_counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kGridCounterOffset);
   a.prefix_len = prefix_len;
   a.ring_k = static_cast<const uint16_t*>(ring_k);
   a.ring_v = static_cast<const uint16_t*>(ring_v);
@@ -276,8 +312,8 @@ rswa_status rswa_decode(const rswa_dims* dims, const void* q, const void* pk, co
                         const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
                         const int32_t* fill, float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
                         void* stream) {
-  return decode_common("rswa_decode", false, dims, q, bf16_prefix(pk, pv), kNoBand, prefix_len, nullptr, nullptr, 0,
-                       ring_k,
+  return decode_common("rswa_decode", false, dims, q, bf16_prefix(pk, pv), kNoBand, kNoAppend, prefix_len, nullptr,
+                       nullptr, 0, ring_k,
                        ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -286,7 +322,7 @@ rswa_status rswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t*
                             const void* ring_v, const int32_t* wp, const int32_t* fill, float scale, float* out,
                             float* lse, void* workspace, size_t ws_bytes, void* stream) {
   return decode_common("rswa_decode_fp8", false, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
-                       prefix_len,
+                       kNoAppend, prefix_len,
                        nullptr, nullptr, 0, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -296,7 +332,7 @@ rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t
                              const void* ring_v, const int32_t* wp, const int32_t* fill, float scale, float* out,
                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
   return decode_common("srswa_decode_fp8", true, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
-                       prefix_len,
+                       kNoAppend, prefix_len,
                        blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -327,9 +363,28 @@ rswa_status srswa_decode(const rswa_dims* dims, const void* q, const void* pk, c
                          const int32_t* prefix_len, const int32_t* blk_idx, const float* blk_logp, int32_t topk,
                          const void* ring_k, const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("srswa_decode", true, dims, q, bf16_prefix(pk, pv), kNoBand, prefix_len, blk_idx, blk_logp, topk,
-                       ring_k,
+  return decode_common("srswa_decode", true, dims, q, bf16_prefix(pk, pv), kNoBand, kNoAppend, prefix_len, blk_idx,
+                       blk_logp, topk, ring_k,
                        ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status rswa_decode_append(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new,
+                               const void* pk, const void* pv, const int32_t* prefix_len, void* ring_k, void* ring_v,
+                               int32_t* wp, int32_t* fill, int32_t* slot_out, float scale, float* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("rswa_decode_append", false, dims, q, bf16_prefix(pk, pv), kNoBand,
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, nullptr, nullptr, 0,
+                       ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new,
+                                const void* pk, const void* pv, const int32_t* prefix_len, const int32_t* blk_idx,
+                                const float* blk_logp, int32_t topk, void* ring_k, void* ring_v, int32_t* wp,
+                                int32_t* fill, int32_t* slot_out, float scale, float* out, float* lse,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("srswa_decode_append", true, dims, q, bf16_prefix(pk, pv), kNoBand,
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, blk_idx, blk_logp,
+                       topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
 rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,
@@ -459,7 +514,8 @@ rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const
                           const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                           const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                           void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("srswa_prefill", true, dims, q, bf16_prefix(pk, pv), BandSrc{T, k_out, v_out}, prefix_len,
+  return decode_common("srswa_prefill", true, dims, q, bf16_prefix(pk, pv), BandSrc{T, k_out, v_out}, kNoAppend,
+                       prefix_len,
                        blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes,
                        stream);
 }
@@ -537,8 +593,8 @@ rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void
   // completion counters (everything before the partials) before this call.
   cudaError_t e = cudaMemsetAsync(scratch, 0, plan.partials_off, s);
   if (e != cudaSuccess) return cuda_fail(e, "rswa_decode_noalloc: clearing the scratch counters");
-  st = decode_common(fn, false, dims, q, bf16_prefix(pk, pv), kNoBand, prefix_len, nullptr, nullptr, 0, ring_k, ring_v,
-                     wp,
+  st = decode_common(fn, false, dims, q, bf16_prefix(pk, pv), kNoBand, kNoAppend, prefix_len, nullptr, nullptr, 0,
+                     ring_k, ring_v, wp,
                      fill, scale, out, lse, scratch, kNoAllocScratchBytes, stream, kNoAllocScratchBytes);
   if (st != RSWA_OK) return st;
   if (status != nullptr) {

@@ -86,6 +86,13 @@ struct SeqView {
   int a0, len0, len1;  // ring slot ranges [a0, a0+len0) and [0, len1)
   int n_r0, n_r1;
   int blen, n_band;    // band rows and tiles (chunked prefill)
+  int n_new;           // fused append: 1 (this step's token, the last tile) or 0
+  const uint16_t* nk;  // fused append: this step's K / V row of (b, h)
+  const uint16_t* nv;
+  uint16_t* wk;        // fused append: ring slot wp[b] of (b, h), where the row is written
+  uint16_t* wv;
+  int32_t* slot_out;   // fused append: &slot_out[b] for head 0, else null
+  int wslot;
   int total;
 };
 
@@ -104,10 +111,12 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
     m = 0;
   }
   int w = 0, f = 0;
+  bool ring_ok = false;
   if (a.ring_k != nullptr) {
     w = a.wp[b];
     f = a.fill[b];
-    if (w < 0 || w >= a.n || f < 0 || f > a.n) {
+    ring_ok = w >= 0 && w < a.n && f >= 0 && f <= a.n;
+    if (!ring_ok) {
       if (report) set_status(a.status, RSWA_DEVICE_BAD_RING_STATE);
       w = 0;
       f = 0;
@@ -129,6 +138,11 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
   v.nb = (m + kBlock - 1) / kBlock;
   int cnt = f;  // ring slots read: the cnt most recently written, (w - cnt + i) mod n for i < cnt
   if (band) cnt = min(max(a.n - 1 - i, 0), f);
+  // fused append: the oldest slot of a full ring (slot w) is overwritten by this step's token,
+  // which is read from k_new / v_new as the last tile instead
+  // (a sequence with a bad ring state is left untouched, as rswa_append leaves it)
+  const bool app = a.k_new != nullptr && ring_ok;
+  if (app && f == a.n) cnt = a.n - 1;
   // a full ring is read as [0, n)
   int a0 = cnt == a.n ? 0 : (w - cnt) % a.n;
   if (a0 < 0) a0 += a.n;
@@ -147,7 +161,19 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
     v.bk = a.k_out + (bh * a.T + start) * kHeadDim;
     v.bv = a.v_out + (bh * a.T + start) * kHeadDim;
   }
-  v.total = v.n_first + v.n_r0 + v.n_r1 + v.n_band;
+  v.n_new = app ? 1 : 0;
+  v.wslot = w;
+  v.nk = v.nv = nullptr;
+  v.wk = v.wv = nullptr;
+  v.slot_out = nullptr;
+  if (app) {
+    v.nk = a.k_new + bh * kHeadDim;
+    v.nv = a.v_new + bh * kHeadDim;
+    v.wk = a.ring_k_w + (bh * a.n + w) * kHeadDim;
+    v.wv = a.ring_v_w + (bh * a.n + w) * kHeadDim;
+    if (h == 0 && a.slot_out) v.slot_out = a.slot_out + b;
+  }
+  v.total = v.n_first + v.n_r0 + v.n_r1 + v.n_band + v.n_new;
   return v;
 }
 
@@ -192,6 +218,13 @@ __device__ __forceinline__ TileRef tile_at(const SeqView& v, int t, int c, float
     return r;
   }
   t -= v.n_first;
+  if (v.n_new && t == v.n_r0 + v.n_r1 + v.n_band) {  // fused append: this step's token (no bias)
+    r.rows = 1;
+    r.k = reinterpret_cast<const uint8_t*>(v.nk);
+    r.v = reinterpret_cast<const uint8_t*>(v.nv);
+    r.blk = -2;
+    return r;
+  }
   if (t >= v.n_r0 + v.n_r1) {  // the causal band of a chunked-prefill query
     t -= v.n_r0 + v.n_r1;
     r.rows = min(kBlock, v.blen - t * kBlock);
@@ -270,6 +303,12 @@ __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& 
   const int c = __shfl_sync(0xffffffffu, iv.c, tile & 31);
   const float lp = __shfl_sync(0xffffffffu, iv.lp, tile & 31);
   const TileRef r = tile_at<kSparse, kFp8>(iv.v, tile, c, lp, lane == 0 ? a.status : nullptr);
+  if (r.blk == -2) {  // fused append: the warp writes this step's row into its ring slot
+    const uint4* src = reinterpret_cast<const uint4*>(lane < 16 ? iv.v.nk : iv.v.nv);
+    uint4* dst = reinterpret_cast<uint4*>(lane < 16 ? iv.v.wk : iv.v.wv);
+    dst[lane & 15] = src[lane & 15];
+    if (lane == 0 && iv.v.slot_out) *iv.v.slot_out = iv.v.wslot;
+  }
   f.rows = r.rows;
   f.bias = r.bias;
   f.fp8 = kFp8 && r.blk >= 0;
@@ -569,6 +608,27 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
       mbar_wait(&sm.full[warp * kStagesPerWarp + j], (phase >> j) & 1u);
       phase ^= 1u << j;
     }
+  if (a.k_new != nullptr) {
+    // fused append: every CTA has read wp / fill once it gets here; the last one to arrive
+    // advances them (sequences with a bad ring state stay untouched) and rearms the counter
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      sm.is_last = atomicAdd(a.grid_counter, 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (sm.is_last) {
+      __threadfence();
+      for (int b = tid; b < a.B; b += kDecodeThreads) {
+        const int w = a.wp_w[b], f = a.fill_w[b];
+        if (w >= 0 && w < a.n && f >= 0 && f <= a.n) {
+          a.wp_w[b] = (w + 1 == a.n) ? 0 : w + 1;
+          a.fill_w[b] = min(f + 1, a.n);
+        }
+      }
+      if (tid == 0) *a.grid_counter = 0;
+    }
+  }
 }
 
 }  // namespace

@@ -43,6 +43,17 @@ struct DecodeArgs {
   int T;
   const uint16_t* k_out;
   const uint16_t* v_out;
+  // fused ring append (decode only): this step's K/V [B][H][D] join the key set as one extra
+  // row, the warp that issues that row writes it into ring slot wp[b], and the launch's last
+  // CTA advances wp / fill (grid_counter: a zeroed int32 in the workspace); null otherwise
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* ring_k_w;
+  uint16_t* ring_v_w;
+  int32_t* wp_w;
+  int32_t* fill_w;
+  int32_t* slot_out;
+  int32_t* grid_counter;
 };
 
 // Workspace layout shared by every op: [status: 256 B][counters][partials].
