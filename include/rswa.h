@@ -265,7 +265,7 @@ RSWA_API rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, c
  * Arguments: those of rswa_append and rswa_decode (srswa_decode), with the ring, wp and
  * fill writable. workspace: rswa_workspace_bytes(dims, RSWA_OP_DECODE) (resp.
  * RSWA_OP_SRSWA_DECODE), zero-initialised; bytes 128..131 of its status area hold the
- * launch's completion counter, which every launch leaves at zero.
+ * launch's completion counter (its last CTA advances wp / fill), left at zero.
  * A sequence whose wp / fill are out of range is flagged (RSWA_DEVICE_BAD_RING_STATE)
  * and left untouched, its ring read as empty and its new token not attended.
  */

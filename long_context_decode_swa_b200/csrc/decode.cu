@@ -70,6 +70,12 @@ struct DecodeSmem {
 constexpr int kDecodeMinBlocks =
     (227 * 1024) / (int)sizeof(DecodeSmem) > 0 ? (227 * 1024) / (int)sizeof(DecodeSmem) : 1;
 
+// What a launch computes besides plain decode: nothing, the fused ring append, or the
+// chunked-prefill band. A compile-time mode, so each kernel carries only its own state.
+constexpr int kModeDecode = 0;
+constexpr int kModeAppend = 1;
+constexpr int kModeBand = 2;
+
 // What a warp needs to enumerate a (sequence, head)'s tiles.
 struct SeqView {
   const uint8_t* pk;  // prefix rows of this (b, h): bf16 rows, or E4M3 code rows (FP8 prefix)
@@ -93,6 +99,7 @@ struct SeqView {
   uint16_t* wv;
   int32_t* slot_out;   // fused append: &slot_out[b] for head 0, else null
   int wslot;
+  int skip_slot;       // fused append on a full ring: slot wp[b], read but masked (-1: none)
   int total;
 };
 
@@ -100,11 +107,11 @@ struct SeqView {
 // blocks) and the ring's valid slots. Chunked prefill: the routed blocks, the outputs
 // j with i - n < j <= i of the chunk (the band) and, for j < 0, the previous chunk's
 // last outputs from the ring: the min(n - 1 - i, fill) most recently written slots.
-template <bool kSparse, bool kFp8>
+template <bool kSparse, bool kFp8, int kMode>
 __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, int i, bool report) {
   SeqView v;
   const int64_t bh = (int64_t)b * a.H + h;
-  const bool band = a.k_out != nullptr;
+  const bool band = kMode == kModeBand;
   int m = a.prefix_len[b];
   if (m < 0 || m > a.cap) {
     if (report) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
@@ -140,9 +147,9 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
   if (band) cnt = min(max(a.n - 1 - i, 0), f);
   // fused append: the oldest slot of a full ring (slot w) is overwritten by this step's token,
   // which is read from k_new / v_new as the last tile instead
-  // (a sequence with a bad ring state is left untouched, as rswa_append leaves it)
-  const bool app = a.k_new != nullptr && ring_ok;
-  if (app && f == a.n) cnt = a.n - 1;
+  // (a sequence with a bad ring state is left untouched, as rswa_append leaves it). A full
+  // ring is still read as [0, n) in aligned tiles, with the overwritten slot masked.
+  const bool app = kMode == kModeAppend && ring_ok;
   // a full ring is read as [0, n)
   int a0 = cnt == a.n ? 0 : (w - cnt) % a.n;
   if (a0 < 0) a0 += a.n;
@@ -163,6 +170,7 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
   }
   v.n_new = app ? 1 : 0;
   v.wslot = w;
+  v.skip_slot = (app && f == a.n) ? w : -1;
   v.nk = v.nv = nullptr;
   v.wk = v.wv = nullptr;
   v.slot_out = nullptr;
@@ -178,24 +186,37 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
 }
 
 // Tile t of a (b, h): where its K and V rows start, how many rows (0 = empty tile), the
-// log2 bias, and the prefix block it covers (-1 for a ring tile). For SR-SWA, (c, lp) is
-// route entry t when t < topk.
+// log2 bias, and the prefix block it covers (-1 for a ring tile, -2 for the fused append's
+// token). For SR-SWA, (c, lp) is the route entry of the tile. Order: [the fused append's
+// token] [prefix tiles or routed blocks] [ring ranges] [chunked-prefill band].
 struct TileRef {
   const uint8_t* k;
   const uint8_t* v;
   int rows;
   float bias;
   int blk;
+  int skip;  // a row of the tile to leave out (-1: none)
 };
 
-template <bool kSparse, bool kFp8>
+template <bool kSparse, bool kFp8, int kMode>
 __device__ __forceinline__ TileRef tile_at(const SeqView& v, int t, int c, float lp, int32_t* status) {
   TileRef r;
   r.bias = 0.f;
   r.k = r.v = v.pk;
   r.rows = 0;
   r.blk = -1;
+  r.skip = -1;
   if (t >= v.total) return r;
+  if (kMode == kModeAppend && v.n_new) {  // fused append: this step's token comes first (no bias)
+    if (t == 0) {
+      r.rows = 1;
+      r.k = reinterpret_cast<const uint8_t*>(v.nk);
+      r.v = reinterpret_cast<const uint8_t*>(v.nv);
+      r.blk = -2;
+      return r;
+    }
+    t -= 1;
+  }
   if (t < v.n_first) {
     int blk;
     if (kSparse) {
@@ -218,13 +239,6 @@ __device__ __forceinline__ TileRef tile_at(const SeqView& v, int t, int c, float
     return r;
   }
   t -= v.n_first;
-  if (v.n_new && t == v.n_r0 + v.n_r1 + v.n_band) {  // fused append: this step's token (no bias)
-    r.rows = 1;
-    r.k = reinterpret_cast<const uint8_t*>(v.nk);
-    r.v = reinterpret_cast<const uint8_t*>(v.nv);
-    r.blk = -2;
-    return r;
-  }
   if (t >= v.n_r0 + v.n_r1) {  // the causal band of a chunked-prefill query
     t -= v.n_r0 + v.n_r1;
     r.rows = min(kBlock, v.blen - t * kBlock);
@@ -244,6 +258,7 @@ __device__ __forceinline__ TileRef tile_at(const SeqView& v, int t, int c, float
   r.rows = min(kBlock, len);
   r.k = reinterpret_cast<const uint8_t*>(v.rk + (int64_t)start * kHeadDim);
   r.v = reinterpret_cast<const uint8_t*>(v.rv + (int64_t)start * kHeadDim);
+  if (v.skip_slot >= start && v.skip_slot < start + r.rows) r.skip = v.skip_slot - start;
   return r;
 }
 
@@ -258,14 +273,14 @@ struct ItemView {
 };
 
 // Items are (query, split) with query vq = (b * H + h) * T + i.
-template <bool kSparse, bool kFp8>
+template <bool kSparse, bool kFp8, int kMode>
 __device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lane, ItemView& iv) {
   const int vq = item / a.splits, split = item - vq * a.splits;
   const int bh = vq / a.T, i = vq - bh * a.T;
   const int b = bh / a.H, h = bh - b * a.H;
   iv.item = item;
   iv.t0 = split * a.tiles_per_item;
-  iv.v = make_view<kSparse, kFp8>(a, b, h, i, lane == 0 && split == 0 && h == 0 && i == 0);
+  iv.v = make_view<kSparse, kFp8, kMode>(a, b, h, i, lane == 0 && split == 0 && h == 0 && i == 0);
   iv.c = -1;
   iv.lp = -INFINITY;
   if (kSparse && lane < a.topk) {
@@ -279,6 +294,7 @@ __device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lan
 // its K / V block scales (loaded at issue time, used at consume time).
 struct InFlight {
   int rows;
+  int skip;
   float bias;
   bool fp8;
   float ks, vs;
@@ -286,7 +302,7 @@ struct InFlight {
 
 // Issues CTA-local tile li (if it exists) into stage s: one bulk copy of its K rows and
 // one of its V rows on full[s]. Warp-collective.
-template <bool kSparse, bool kFp8>
+template <bool kSparse, bool kFp8, int kMode>
 __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& sm, int li, int s, int lane,
                                                ItemView& iv) {
   const int P = a.tiles_per_item;
@@ -294,15 +310,18 @@ __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& 
   const int64_t item = (int64_t)blockIdx.x + (int64_t)it * gridDim.x;
   InFlight f;
   f.rows = 0;
+  f.skip = -1;
   f.bias = 0.f;
   f.fp8 = false;
   f.ks = f.vs = 1.f;
   if (item >= a.items) return f;
-  if (iv.item != (int)item) load_item<kSparse, kFp8>(a, (int)item, lane, iv);
+  if (iv.item != (int)item) load_item<kSparse, kFp8, kMode>(a, (int)item, lane, iv);
   const int tile = iv.t0 + (li - it * P);
-  const int c = __shfl_sync(0xffffffffu, iv.c, tile & 31);
-  const float lp = __shfl_sync(0xffffffffu, iv.lp, tile & 31);
-  const TileRef r = tile_at<kSparse, kFp8>(iv.v, tile, c, lp, lane == 0 ? a.status : nullptr);
+  // route entry of the tile (the fused append's token tile comes before the routed blocks)
+  const int ridx = (kMode == kModeAppend && iv.v.n_new) ? tile - 1 : tile;
+  const int c = __shfl_sync(0xffffffffu, iv.c, ridx & 31);
+  const float lp = __shfl_sync(0xffffffffu, iv.lp, ridx & 31);
+  const TileRef r = tile_at<kSparse, kFp8, kMode>(iv.v, tile, c, lp, lane == 0 ? a.status : nullptr);
   if (r.blk == -2) {  // fused append: the warp writes this step's row into its ring slot
     const uint4* src = reinterpret_cast<const uint4*>(lane < 16 ? iv.v.nk : iv.v.nv);
     uint4* dst = reinterpret_cast<uint4*>(lane < 16 ? iv.v.wk : iv.v.wv);
@@ -310,6 +329,7 @@ __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& 
     if (lane == 0 && iv.v.slot_out) *iv.v.slot_out = iv.v.wslot;
   }
   f.rows = r.rows;
+  f.skip = r.skip;
   f.bias = r.bias;
   f.fp8 = kFp8 && r.blk >= 0;
   if (f.fp8 && r.rows > 0) {
@@ -348,8 +368,8 @@ __device__ __forceinline__ float2 bf16x2_f2(uint32_t w) { return make_float2(bf1
 // (128 B) of one prefix block with scales (ks, vs), folded into the score and into the
 // row weight of P.V; otherwise bf16 rows (256 B) and ks = vs = 1.
 template <bool kFull, bool kFp8>
-__device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* vt, int rows, float bias, float ks,
-                                             float vs, const float2 (&q2)[4], int g, int c, float& m_run,
+__device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* vt, int rows, int skip, float bias,
+                                             float ks, float vs, const float2 (&q2)[4], int g, int c, float& m_run,
                                              float& l_lane, float2 (&acc)[4]) {
   float pd[16];
 #pragma unroll
@@ -399,7 +419,8 @@ __device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* v
     pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
   }
   // this lane now holds the score of tile row 2c + g
-  const float sc = (kFull || 2 * c + g < rows) ? (kFp8 ? fmaf(pd[0], ks, bias) : pd[0] + bias) : -INFINITY;
+  const float sc = (kFull || (2 * c + g < rows && 2 * c + g != skip)) ? (kFp8 ? fmaf(pd[0], ks, bias) : pd[0] + bias)
+                                                                    : -INFINITY;
   const float m_new = fmaxf(m_run, warp_max(sc));
   const float alpha = exp2f(m_run - m_new);
   const float p = exp2f(sc - m_new);
@@ -412,7 +433,7 @@ __device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* v
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float pj = __shfl_sync(0xffffffffu, pw, (g << 4) | j);
-    if (kFull || 2 * j + g < rows) {
+    if (kFull || (2 * j + g < rows && 2 * j + g != skip)) {
       const float2 p2 = make_float2(pj, pj);
       if (kFp8) {
         const uint2 w = *reinterpret_cast<const uint2*>(vt + (2 * j + g) * kHeadDim + c * 8);
@@ -431,7 +452,7 @@ __device__ __forceinline__ void consume_tile(const uint8_t* kt, const uint8_t* v
   }
 }
 
-template <bool kSparse, bool kFp8>
+template <bool kSparse, bool kFp8, int kMode>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
@@ -453,7 +474,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
   InFlight fl[kStagesPerWarp];
 #pragma unroll
   for (int j = 0; j < kStagesPerWarp; ++j)
-    fl[j] = issue_tile<kSparse, kFp8>(a, sm, warp + j * kWarps, warp * kStagesPerWarp + j, lane, iv);
+    fl[j] = issue_tile<kSparse, kFp8, kMode>(a, sm, warp + j * kWarps, warp * kStagesPerWarp + j, lane, iv);
   uint32_t phase = 0;  // bit j: parity of the next completion of this warp's stage j
   int k = 0;           // tiles of this warp consumed so far
   bool ok = true;
@@ -497,22 +518,24 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
         phase ^= 1u << j;
         const uint8_t* kt = sm.stage[s][0];
         const uint8_t* vt = sm.stage[s][1];
+        const bool full = rows == kBlock && cur.skip < 0;
         if (kFp8 && cur.fp8) {
-          if (rows == kBlock)
-            consume_tile<true, true>(kt, vt, rows, cur.bias, cur.ks, cur.vs, q2, g, c, m_run, l_lane, acc);
+          if (full)
+            consume_tile<true, true>(kt, vt, rows, -1, cur.bias, cur.ks, cur.vs, q2, g, c, m_run, l_lane, acc);
           else
-            consume_tile<false, true>(kt, vt, rows, cur.bias, cur.ks, cur.vs, q2, g, c, m_run, l_lane, acc);
+            consume_tile<false, true>(kt, vt, rows, cur.skip, cur.bias, cur.ks, cur.vs, q2, g, c, m_run, l_lane,
+                                      acc);
         } else {
-          if (rows == kBlock)
-            consume_tile<true, false>(kt, vt, rows, cur.bias, 1.f, 1.f, q2, g, c, m_run, l_lane, acc);
+          if (full)
+            consume_tile<true, false>(kt, vt, rows, -1, cur.bias, 1.f, 1.f, q2, g, c, m_run, l_lane, acc);
           else
-            consume_tile<false, false>(kt, vt, rows, cur.bias, 1.f, 1.f, q2, g, c, m_run, l_lane, acc);
+            consume_tile<false, false>(kt, vt, rows, cur.skip, cur.bias, 1.f, 1.f, q2, g, c, m_run, l_lane, acc);
         }
       }
       __syncwarp();  // every lane has read the stage before it is refilled
 #pragma unroll
       for (int i = 0; i + 1 < kStagesPerWarp; ++i) fl[i] = fl[i + 1];
-      fl[kStagesPerWarp - 1] = issue_tile<kSparse, kFp8>(a, sm, li + kWarps * kStagesPerWarp, s, lane, iv);
+      fl[kStagesPerWarp - 1] = issue_tile<kSparse, kFp8, kMode>(a, sm, li + kWarps * kStagesPerWarp, s, lane, iv);
       ++k;
     }
     // fold the two half-warps (same dims, different rows) and the lanes' sums
@@ -608,9 +631,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
       mbar_wait(&sm.full[warp * kStagesPerWarp + j], (phase >> j) & 1u);
       phase ^= 1u << j;
     }
-  if (a.k_new != nullptr) {
+  if (kMode == kModeAppend) {
     // fused append: every CTA has read wp / fill once it gets here; the last one to arrive
-    // advances them (sequences with a bad ring state stay untouched) and rearms the counter
+    // advances them (sequences with a bad ring state stay untouched) and rearms the counter.
+    // (Advancing per sequence as its last item finishes put a fence and an atomic at every
+    // item boundary and measured slower.)
     __syncthreads();
     if (tid == 0) {
       __threadfence();
@@ -677,10 +702,27 @@ WorkspacePlan plan_decode_workspace(int B, int H, int64_t max_tiles, int sm_coun
 
 cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem);
-  static unsigned long long done[4] = {0, 0, 0, 0};
-  auto kernel = sparse ? (a.fp8 ? decode_kernel<true, true> : decode_kernel<true, false>)
-                       : (a.fp8 ? decode_kernel<false, true> : decode_kernel<false, false>);
-  cudaError_t e = ensure_smem_limit(kernel, smem, &done[(sparse ? 2 : 0) + (a.fp8 ? 1 : 0)]);
+  // the instantiations in use: plain decode for every prefix format; the fused append and the
+  // chunked-prefill band over a bf16 prefix
+  const int mode = a.k_out != nullptr ? kModeBand : (a.k_new != nullptr ? kModeAppend : kModeDecode);
+  void (*kernel)(const DecodeArgs) = nullptr;
+  int slot = 0;
+  if (mode == kModeDecode) {
+    kernel = sparse ? (a.fp8 ? decode_kernel<true, true, kModeDecode> : decode_kernel<true, false, kModeDecode>)
+                    : (a.fp8 ? decode_kernel<false, true, kModeDecode> : decode_kernel<false, false, kModeDecode>);
+    slot = (sparse ? 2 : 0) + (a.fp8 ? 1 : 0);
+  } else if (a.fp8) {
+    return cudaErrorNotSupported;
+  } else if (mode == kModeAppend) {
+    kernel = sparse ? decode_kernel<true, false, kModeAppend> : decode_kernel<false, false, kModeAppend>;
+    slot = sparse ? 5 : 4;
+  } else {
+    if (!sparse) return cudaErrorNotSupported;
+    kernel = decode_kernel<true, false, kModeBand>;
+    slot = 6;
+  }
+  static unsigned long long done[7] = {0, 0, 0, 0, 0, 0, 0};
+  cudaError_t e = ensure_smem_limit(kernel, smem, &done[slot]);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
