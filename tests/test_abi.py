@@ -107,3 +107,48 @@ def test_python_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         rswa.rswa_append(t, t, t[:, :, 0], t[:, :, 0], torch.zeros(1, dtype=torch.int32),
                          torch.zeros(1, dtype=torch.int32))
+
+
+def test_fp8_entry_points_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64)
+    st = ctypes.c_void_p(0x30000)
+    q = [ctypes.byref(d), A, A, A, A, A, A, A, st, None]           # valid: never called as is (it would launch)
+    bad = list(q)
+    bad[4] = None                                                      # pk8
+    assert lib.rswa_quantize_prefix(*bad) == INVALID and "pk8" in _err()
+    bad = list(q)
+    bad[6] = MIS                                                       # k_scale
+    assert lib.rswa_quantize_prefix(*bad) == INVALID and "aligned" in _err()
+    ws = lib.rswa_workspace_bytes(ctypes.byref(d), 1)
+    dec = [ctypes.byref(d), A, A, A, None, A, A, A, A, A, A, ctypes.c_float(0.088), A, None, A, ctypes.c_size_t(ws),
+           None]
+    assert lib.rswa_decode_fp8(*dec) == INVALID and "k_scale" in _err()
+
+
+def test_chunked_prefill_entry_points_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64)
+    route = lambda T, dims=d: lib.srswa_route_tokens(ctypes.byref(dims), T, A, A, A, ctypes.c_float(1.0), 16, A, A, A,
+                                                     ctypes.c_size_t(256), None)
+    assert route(0) == INVALID and "T must be" in _err()
+    assert route(40000) == UNSUPPORTED and "65535" in _err()
+    pf = lambda T=8, k_out=A, ring_k=None, ring_v=None: lib.srswa_prefill(
+        ctypes.byref(d), T, A, k_out, A, A, A, A, A, A, 16, ring_k, ring_v, None, None, ctypes.c_float(0.088), A, None,
+        A, ctypes.c_size_t(256), None)
+    assert pf(T=0) == INVALID and "T must be" in _err()
+    assert pf(k_out=MIS) == INVALID and "aligned" in _err()
+    assert pf(ring_k=A) == INVALID and "both" in _err()
+    assert pf(ring_k=A, ring_v=A2) == INVALID and "wp and fill" in _err()
+
+
+def test_fused_step_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64)
+    ws = lib.rswa_workspace_bytes(ctypes.byref(d), 1)
+    call = lambda k_new=A, ws_bytes=ws: lib.rswa_decode_append(
+        ctypes.byref(d), A, k_new, A, A, A, A, A, A, A, A, None, ctypes.c_float(0.088), A, None, A,
+        ctypes.c_size_t(ws_bytes), None)
+    assert call(k_new=None) == INVALID and "k_new" in _err()
+    assert call(k_new=MIS) == INVALID and "aligned" in _err()
+    assert call(ws_bytes=255) == INVALID and "workspace" in _err()
