@@ -372,6 +372,8 @@ rswa_status rswa_decode_append(const rswa_dims* dims, const void* q, const void*
                                const void* pk, const void* pv, const int32_t* prefix_len, void* ring_k, void* ring_v,
                                int32_t* wp, int32_t* fill, int32_t* slot_out, float scale, float* out, float* lse,
                                void* workspace, size_t ws_bytes, void* stream) {
+  if (k_new == nullptr || v_new == nullptr)
+    return fail(RSWA_ERR_INVALID, "rswa_decode_append: k_new and v_new must not be NULL");
   return decode_common("rswa_decode_append", false, dims, q, bf16_prefix(pk, pv), kNoBand,
                        AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, nullptr, nullptr, 0,
                        ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
@@ -382,6 +384,8 @@ rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, const void
                                 const float* blk_logp, int32_t topk, void* ring_k, void* ring_v, int32_t* wp,
                                 int32_t* fill, int32_t* slot_out, float scale, float* out, float* lse,
                                 void* workspace, size_t ws_bytes, void* stream) {
+  if (k_new == nullptr || v_new == nullptr)
+    return fail(RSWA_ERR_INVALID, "srswa_decode_append: k_new and v_new must not be NULL");
   return decode_common("srswa_decode_append", true, dims, q, bf16_prefix(pk, pv), kNoBand,
                        AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, blk_idx, blk_logp,
                        topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
