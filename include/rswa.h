@@ -76,15 +76,17 @@ typedef struct {
 } rswa_dims;
 
 /* Operation codes for rswa_workspace_bytes. */
-#define RSWA_OP_DECODE 1        /* rswa_decode                       */
-#define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode (any topk in 1..32)  */
-#define RSWA_OP_ROUTE 3         /* srswa_route                       */
-#define RSWA_OP_PREFILL 4       /* rswa_prefill                      */
+#define RSWA_OP_DECODE 1        /* rswa_decode, rswa_decode_fp8, rswa_decode_append          */
+#define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode, srswa_decode_fp8, srswa_decode_append
+                                   (any topk in 1..32)                                      */
+#define RSWA_OP_ROUTE 3         /* srswa_route, srswa_route_tokens (256 bytes)               */
+#define RSWA_OP_PREFILL 4       /* rswa_prefill, srswa_prefill (256 bytes)                   */
 
 /* Message of the last failed call on this host thread ("" if none). */
 RSWA_API const char* rswa_last_error(void);
 
-/* Library ABI version (incremented on any signature change). */
+/* Library ABI version (incremented when entry points are added or changed): 2 adds the
+ * FP8 prefix, the fused decode step and the SR-SWA chunked prefill to version 1. */
 RSWA_API int32_t rswa_version(void);
 
 /*

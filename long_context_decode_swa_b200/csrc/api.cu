@@ -75,7 +75,7 @@ extern "C" {
 
 const char* rswa_last_error(void) { return g_last_error; }
 
-int32_t rswa_version(void) { return 1; }
+int32_t rswa_version(void) { return 2; }
 
 size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
   const char* fn = "rswa_workspace_bytes";

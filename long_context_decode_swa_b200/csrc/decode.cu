@@ -28,6 +28,12 @@
 //    of a (sequence, head) to finish (atomic counter) merges the partials by
 //    log-sum-exp and resets the counter.
 // The split count is chosen per launch to minimise the busiest CTA's tile count.
+//
+// The same kernel serves, as compile-time variants: an FP8 (E4M3) prefix with block
+// scales (a prefix tile is 128-byte code rows); the fused decode step (this step's token
+// is read as a one-row tile and written into its ring slot inside the launch, whose last
+// CTA advances wp / fill); and the SR-SWA chunked prefill (items are single queries of a
+// chunk, whose key sets end with their causal band of the chunk's outputs).
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 

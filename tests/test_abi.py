@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     lib = rswa.load()
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.rswa_version() == 1
+    assert lib.rswa_version() == 2
 
 
 def _err():
