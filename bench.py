@@ -228,11 +228,16 @@ def measured_peak():
 
 
 def kernel_source_hash(kind: str) -> str:
-    """Hash of the sources the measured kernel is built from (kind: dense, sparse or prefill)."""
-    files = ["prefill.cu" if kind == "prefill" else "decode.cu", "common.cuh", "internal.h"]
+    """Hash of the code the measured kernel is built from (kind: dense, sparse or prefill), with
+    comments and blank lines removed: a traffic record stays valid across comment edits only."""
+    import re
+    files = ["prefill.cu", "common.cuh"] if kind == "prefill" else ["decode.cu", "common.cuh", "internal.h"]
     h = hashlib.sha256()
     for f in files:
-        h.update(open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", f), encoding="utf-8").read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("\n".join(line.rstrip() for line in src.splitlines() if line.strip()).encode())
     h.update(kind.encode())
     return h.hexdigest()[:16]
 
