@@ -283,7 +283,7 @@ RSWA_API rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, c
                                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * SR-SWA chunked prefill (the survey's next row 1). The pages size prefill memory by a
+ * SR-SWA chunked prefill. The pages size prefill memory by a
  * per-token router score tensor of about [tokens, context/32] (serving notes,
  * --max-prefill-tokens), i.e. every output-side token of a chunk is routed by itself;
  * the rule is the decode router's (srswa_route). Reading adopted: query i of a chunk of

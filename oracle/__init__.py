@@ -76,6 +76,10 @@ def _L():
             lib.oracle_rswa_decode_fp8.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, P, P, Dbl, P, P]
             lib.oracle_srswa_decode_fp8.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, I, P, P, P, P, Dbl,
                                                     P, P]
+            lib.oracle_bf16_round.argtypes = [Dbl]
+            lib.oracle_bf16_round.restype = ctypes.c_uint16
+            lib.oracle_bf16_round_array.argtypes = [I64, P, P]
+            lib.oracle_rope_page2d.argtypes = [I64, I, I, P, P, P, Dbl, I, P]
             _lib = lib
     return _lib
 
@@ -363,6 +367,39 @@ def srswa_decode_fp8(q, pk8, pv8, kscale, vscale, prefix_len, blk_idx, blk_logp,
                                  _p(prefix_len), _p(blk_idx), _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp),
                                  _p(fill), float(scale), _p(out), _p(lse))
     return out, lse
+
+
+# ---------------------------------------------------------------- page2d rotary encoding
+
+def bf16_round(x) -> np.ndarray:
+    """Nearest bf16 bit patterns (uint16) of fp64 values, ties to even."""
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.zeros(x.shape, np.uint16)
+    _L().oracle_bf16_round_array(x.size, _p(x), _p(out))
+    return out
+
+
+def rope_page2d(x, tok_pos, page, base: float = 10000.0, page_mod: int = 2) -> np.ndarray:
+    """page2d rotary encoding of bf16 rows x uint16 [..., H, D]; tok_pos / page int32 with the
+    shape of x's leading dims (one token-axis and one page-axis position per row).
+    Returns the exact rotation in fp64, shaped like x (readings: oracle_rope_page2d)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16 or x.ndim < 2:
+        raise TypeError("x: expected bf16 bit patterns as uint16 [..., H, D]")
+    H, D = x.shape[-2:]
+    if D % 2:
+        raise ValueError("D must be even")
+    lead = x.shape[:-2]
+    tok_pos = _i32(np.asarray(tok_pos, np.int32), "tok_pos")
+    page = _i32(np.asarray(page, np.int32), "page")
+    if tok_pos.shape != lead or page.shape != lead:
+        raise ValueError(f"positions must have shape {lead}")
+    if page_mod < 0:
+        raise ValueError("page_mod must be >= 0")
+    rows = int(np.prod(lead)) if lead else 1
+    out = np.zeros(x.shape, np.float64)
+    _L().oracle_rope_page2d(rows, H, D, _p(x), _p(tok_pos), _p(page), float(base), int(page_mod), _p(out))
+    return out
 
 
 def kv_cache_bytes(ref_tokens: int, T: int, heads: int, head_dim: int, layers: int, bytes_per_elem: int,

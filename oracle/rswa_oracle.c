@@ -713,7 +713,7 @@ void oracle_e4m3_encode_array(int64_t count, const float* x, uint8_t* out) {
 }
 
 /* ------------------------------------------------------------------ */
-/* next row: SR-SWA chunked prefill                                    */
+/* SR-SWA chunked prefill                                              */
 /* ------------------------------------------------------------------ */
 
 /*
@@ -792,5 +792,85 @@ void oracle_srswa_prefill(int B, int H, int D, int n, int64_t cap, int T, int bl
       attend(&L, q + (bh * T + i) * D, D, scale, out + (bh * nrows + r) * D, lse + bh * nrows + r);
     }
     keylist_free(&L);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* page2d rotary position encoding                                     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Nearest bf16 to x, ties to the even pattern, as its bit pattern. The bf16
+ * grid in the binade [2^e, 2^(e+1)) has spacing 2^(e-7) (2^-133 below 2^-126);
+ * magnitudes that round past the largest finite value give infinity.
+ * Pinned by: torch's float32 -> bfloat16 conversion (round to nearest even) on
+ * float32-representable inputs, exact round trips of bf16 values, and the
+ * tie cases 1 + 2^-8 -> 1 and 1 + 3 * 2^-8 -> 1 + 2^-6.
+ */
+uint16_t oracle_bf16_round(double x) {
+  if (isnan(x)) return 0x7fc0;
+  uint16_t sign = signbit(x) ? 0x8000 : 0;
+  double a = fabs(x), spacing;
+  if (a < ldexp(1.0, -126)) {
+    spacing = ldexp(1.0, -133);
+  } else {
+    int e;
+    frexp(a, &e);
+    spacing = ldexp(1.0, e - 1 - 7); /* a in [2^(e-1), 2^e) */
+  }
+  double r = round_half_even(a / spacing) * spacing;
+  if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7f80);
+  float f = (float)r; /* exact: r is on the bf16 grid */
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  return (uint16_t)(sign | (u >> 16));
+}
+
+void oracle_bf16_round_array(int64_t count, const double* x, uint16_t* out) {
+  for (int64_t i = 0; i < count; ++i) out[i] = oracle_bf16_round(x[i]);
+}
+
+/*
+ * page2d rotary position encoding of rows x [rows][H][D] (bf16), each row with
+ * a token-axis position tok_pos[r] (the in-page offset) and a page-axis position
+ * page[r] (the page number)
+ *   [SR-SWA explainer, 2D 位置编码: two rotary axes, sparse_rope_mode page2d,
+ *    the token axis orders tokens inside a page, the page axis (page_mod: 2)
+ *    tells pages apart].
+ * Readings where the page is silent (constants and layout are not given):
+ *   - the head dimension is rotated in the half-split pairing of the LLaMA
+ *     family the model's attention derives from: pair i couples dims i and
+ *     i + D/2, for i < D/2, rotated by angle a:
+ *       out_i = x_i cos a - x_{i+D/2} sin a,  out_{i+D/2} = x_{i+D/2} cos a + x_i sin a;
+ *   - pair i has frequency theta_i = base^(-2i/D) (base 10000 in the model
+ *     family; a parameter here);
+ *   - page_mod interleaves the axes: pair i follows the page axis when
+ *     i mod page_mod = page_mod - 1, the token axis otherwise (page_mod 2: odd
+ *     pairs on the page axis, even pairs on the token axis); page_mod 0 puts
+ *     every pair on the token axis (plain 1-D rotary encoding);
+ *   - a = position of the pair's axis * theta_i.
+ * out [rows][H][D] in fp64 (the exact rotation of the bf16 inputs).
+ * Pinned by: the LLaMA rotary routine of the transformers library (page_mod 0;
+ * page_mod 2 with page = tok_pos), axis separation (page 0 leaves the page-axis
+ * pairs unchanged and the token-axis pairs equal the library's encoding, and
+ * the converse), relative-position invariance of q.k, per-pair norms.
+ */
+void oracle_rope_page2d(int64_t rows, int H, int D, const uint16_t* x, const int32_t* tok_pos, const int32_t* page,
+                        double base, int page_mod, double* out) {
+  const int half = D / 2;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int i = 0; i < half; ++i) {
+      int on_page = page_mod > 0 && i % page_mod == page_mod - 1;
+      double pos = on_page ? (double)page[r] : (double)tok_pos[r];
+      double theta = pow(base, -2.0 * i / D);
+      double c = cos(pos * theta), s = sin(pos * theta);
+      for (int h = 0; h < H; ++h) {
+        int64_t off = (r * H + h) * (int64_t)D;
+        double lo = bf16_to_double(x[off + i]), hi = bf16_to_double(x[off + i + half]);
+        out[off + i] = lo * c - hi * s;
+        out[off + i + half] = hi * c + lo * s;
+      }
+    }
   }
 }

@@ -1,4 +1,4 @@
-"""Pins of the oracle's SR-SWA chunked prefill (the survey's next row 1).
+"""Pins of the oracle's SR-SWA chunked prefill.
 
 - per-token routes: with planted router keys every token recovers its planted
   top-16 in order (the construction of synth.plant_router_keys).
