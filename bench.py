@@ -10,6 +10,9 @@ A step is one decode step of the whole batch through the C ABI:
                           once before timing: rswa_append + rswa_decode_fp8
                           (+ srswa_route + srswa_decode_fp8)
   config 8 (SR-SWA chunked prefill): srswa_route_tokens + srswa_prefill
+  config 9 (page2d rotary encoding of a prefill chunk's q and k): rswa_rope_page2d
+  config 10:              config 4 with the page2d encoding: rswa_append_rope +
+                          srswa_route + srswa_decode
 (the router's block index keys are pooled once per prefix, before timing).
 The default workload is the batched R-SWA decode: 512 sequences, 16 heads,
 head_dim 128, a 10-page prefix (2560 visual + 32 prompt tokens) and a full
@@ -86,6 +89,15 @@ def workload(cfg: int) -> dict:
                     name="SR-SWA chunked prefill, 4 sequences, 16 heads, head_dim 128, 32768-token history (1024 "
                          "blocks), 4096 output-side queries each routed to its own top-16 blocks (planted, 32 "
                          "directions cycled over the tokens) + causal band 128")
+    if cfg == 9:
+        return dict(kind="rope", B=4, H=16, D=128, n=128, plen=[0] * 4, cap=0, T=4096, wp0=None,
+                    name="page2d rotary encoding of a prefill chunk, 4 sequences x 4096 tokens, 16 heads, head_dim "
+                         "128, q and k (bf16 in, bf16 out), tokens on pages of 200-2000 tokens, base 10000, page_mod 2")
+    if cfg == 10:
+        w = workload(4)
+        w["rope"] = True
+        w["name"] += "; page2d rotary encoding of q and the new key fused into the ring append (rswa_append_rope)"
+        return w
     if cfg in (6, 7):  # the batched R-SWA and the 32K-history SR-SWA workloads over an FP8 (E4M3) prefix
         w = workload(2 if cfg == 6 else 4)
         w["fp8"] = True
@@ -228,10 +240,11 @@ def measured_peak():
 
 
 def kernel_source_hash(kind: str) -> str:
-    """Hash of the code the measured kernel is built from (kind: dense, sparse or prefill), with
+    """Hash of the code the measured kernel is built from (kind: dense, sparse, prefill or rope), with
     comments and blank lines removed: a traffic record stays valid across comment edits only."""
     import re
-    files = ["prefill.cu", "common.cuh"] if kind == "prefill" else ["decode.cu", "common.cuh", "internal.h"]
+    files = {"prefill": ["prefill.cu", "common.cuh"], "rope": ["rope.cu", "common.cuh"]}.get(
+        kind, ["decode.cu", "common.cuh", "internal.h"])
     h = hashlib.sha256()
     for f in files:
         src = open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", f), encoding="utf-8").read()
@@ -307,6 +320,12 @@ class Problem:
             self.k8, self.v8, self.ks, self.vs = rswa.fp8_prefix_buffers(self.c.pk)
             rswa.rswa_quantize_prefix(self.c.pk, self.c.pv, self.c.prefix_len, self.k8, self.v8, self.ks, self.vs,
                                       status=self.ws)
+        self.rope = bool(w.get("rope"))
+        if self.rope:  # this step's token positions ([steps][B]) and the encoded query
+            tok, page = synth.page_positions(B, steps_total, seed=seed + 2)
+            self.tok = tok.t().contiguous().to("cuda")
+            self.page = page.t().contiguous().to("cuda")
+            self.q_rot = torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda")
         if self.sparse:
             n_dirs = 32
             pl = synth.plant_router_keys(w["plen"], w["cap"], n_dirs=n_dirs, seed=seed + 1, device="cuda")
@@ -338,7 +357,15 @@ class Problem:
             if ev is not None:
                 ev[1].record()
             return 1
-        r.rswa_append(c.ring_k, c.ring_v, k_new, v_new, c.wp, c.fill, status=self.ws)
+        if self.rope:
+            if ev is not None:
+                ev[4].record()
+            q = r.rswa_append_rope(c.ring_k, c.ring_v, k_new, v_new, c.wp, c.fill, q, self.tok[i % self.tok.shape[0]],
+                                   self.page[i % self.page.shape[0]], q_out=self.q_rot, status=self.ws)
+            if ev is not None:
+                ev[5].record()
+        else:
+            r.rswa_append(c.ring_k, c.ring_v, k_new, v_new, c.wp, c.fill, status=self.ws)
         if not self.sparse:
             if ev is not None:
                 ev[0].record()
@@ -462,6 +489,8 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     K, W = args.steps, args.warmup
     if w["kind"] in ("prefill", "srswa_prefill"):
         return run_prefill(args, w, world, rank, local)
+    if w["kind"] == "rope":
+        return run_rope(args, w, world, rank, local)
     prob = Problem(w, K + W, seed=1000 * args.config + rank)
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
@@ -473,7 +502,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     # every EVENT_EVERY-th step (an event node costs several microseconds of step time, so bracketing
     # every step would slow the step it measures)
     sampled = list(range(0, K, EVENT_EVERY))
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in sampled]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)] for _ in sampled]
     graph = torch.cuda.CUDAGraph()
     launches = 0
     with torch.cuda.graph(graph, stream=stream):
@@ -503,6 +532,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     ms_total = start.elapsed_time(end)
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     route_ms = [e[2].elapsed_time(e[3]) for e in evs] if prob.sparse else []
+    rope_ms = [e[4].elapsed_time(e[5]) for e in evs] if prob.rope else []
     ms_max = max_over_ranks(world, ms_total)
     del graph
 
@@ -562,7 +592,8 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
                      "fallback 6650 GB/s", "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes["attn"], "avg_launch_us": attn_avg_s * 1e6},
         "kernels_us": {"attention": attn_avg_s * 1e6,
-                       **({"route": statistics.mean(route_ms) * 1e3} if route_ms else {})},
+                       **({"route": statistics.mean(route_ms) * 1e3} if route_ms else {}),
+                       **({"append_rope": statistics.mean(rope_ms) * 1e3} if rope_ms else {})},
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "steps/s", "h2d_bytes_per_step": e2e["h2d"],
@@ -650,6 +681,139 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
         "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "prefill chunks/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
     }
+
+
+class RopeProblem:
+    """A prefill chunk's q and k (bf16 [B][T][H][D]) with their page positions; a step is one
+    rswa_rope_page2d launch encoding both into separate outputs."""
+
+    def __init__(self, w: dict, seed: int):
+        import torch
+
+        import long_context_decode_swa_b200 as rswa
+        from long_context_decode_swa_b200 import synth
+        self.rswa = rswa
+        self.w = w
+        B, T, H, D = w["B"], w["T"], w["H"], w["D"]
+        g = synth._gen(seed, "cuda")
+        self.q = synth.randn_bf16((B, T, H, D), g, "cuda")
+        self.k = synth.randn_bf16((B, T, H, D), g, "cuda")
+        tok, page = synth.page_positions(B, T, seed=seed + 1)
+        self.tok, self.page = tok.to("cuda"), page.to("cuda")
+        self.q_out, self.k_out = torch.empty_like(self.q), torch.empty_like(self.k)
+        torch.cuda.synchronize()
+
+    def step(self, i: int, q=None, k=None, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.rswa.rswa_rope_page2d(self.q if q is None else q, self.tok, self.page, q_out=self.q_out,
+                                   k=self.k if k is None else k, k_out=self.k_out, base=10000.0, page_mod=2)
+        if ev is not None:
+            ev[1].record()
+        return 1
+
+
+def rope_bytes(w: dict) -> float:
+    """Bytes the encoding must move per launch: q and k read and written once (2 B per element)
+    and the two int32 positions of every token."""
+    elems = w["B"] * w["T"] * w["H"] * w["D"]
+    return float(2 * 2 * 2 * elems + 2 * 4 * w["B"] * w["T"])
+
+
+def run_rope(args, w: dict, world: int, rank: int, local: int) -> dict:
+    import torch
+    K, W = args.steps, args.warmup
+    prob = RopeProblem(w, seed=1000 * args.config + rank)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            prob.step(i)
+    stream.synchronize()
+    sampled = list(range(0, K, EVENT_EVERY))
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in sampled]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            prob.step(i, ev=evs[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
+    graph.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record()
+        graph.replay()
+        end.record()
+    end.synchronize()
+    t1 = time.time()
+    barrier(world)
+    clk = clocks.stop(t0, t1)
+    ms_max = max_over_ranks(world, start.elapsed_time(end))
+    kern_s = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    del graph
+    nbytes = rope_bytes(w)
+    achieved = nbytes / kern_s / 1e9
+    peak, peak_src = measured_peak()
+    e2e = run_rope_e2e(prob, K, W) if not args.no_e2e else {"ms": float("nan"), "h2d": 0, "d2h": 0}
+    e2e_ms = max_over_ranks(world, e2e["ms"])
+    B, H, T = w["B"], w["H"], w["T"]
+    value = world * K / (ms_max / 1e3)
+    return {
+        "metric": METRIC, "value": value, "unit": "encoded chunks/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "heads": H,
+                   "head_dim": w["D"], "chunk": T, "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: each step streams {nbytes / 1e9:.2f} GB through L2 ({nbytes / 2e9:.2f} GB read, "
+                         "as much written), twice its 126 MB, in the same order every step",
+                   "timing": "K launches in one CUDA graph replay, CUDA events; kernel durations from "
+                             f"event brackets in every {EVENT_EVERY}th step"},
+        "tok_per_s": value * B * T,
+        "roofline": {"bound": "hbm", "kernel": "rope_kernel (page2d, q and k)", "achieved": achieved, "peak": peak,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
+                     "fallback 6650 GB/s", "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": committed_traffic(f"rope_config{args.config}", kernel_source_hash("rope")),
+                     "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": kern_s * 1e6},
+        "kernels_us": {"rope": kern_s * 1e6},
+        "gpu_launches": K,
+        "clocks": clk,
+        "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "encoded chunks/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
+    }
+
+
+def run_rope_e2e(prob: RopeProblem, K: int, W: int) -> dict:
+    """Pinned host q and k -> device -> rswa_rope_page2d -> encoded q and k back to the host."""
+    import torch
+    hq, hk = prob.q.cpu().pin_memory(), prob.k.cpu().pin_memory()
+    dq, dk = torch.empty_like(prob.q), torch.empty_like(prob.k)
+    oq = torch.empty(prob.q.shape, dtype=torch.bfloat16, pin_memory=True)
+    ok = torch.empty(prob.k.shape, dtype=torch.bfloat16, pin_memory=True)
+    stream = torch.cuda.Stream()
+
+    def one(i):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        prob.step(i, q=dq, k=dk)
+        oq.copy_(prob.q_out, non_blocking=True)
+        ok.copy_(prob.k_out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            one(i)
+    stream.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record()
+        for i in range(K):
+            one(i)
+        e.record()
+    e.synchronize()
+    return {"ms": s.elapsed_time(e), "h2d": 2 * hq.numel() * 2, "d2h": 2 * oq.numel() * 2}
 
 
 def run_prefill_e2e(prob: PrefillProblem, K: int, W: int) -> dict:
@@ -744,6 +908,9 @@ def oracle_sample_step(w: dict, sample: int, seed: int):
         import oracle
         st["k8"], st["ks"] = oracle.quantize_prefix(st["pk"], st["plen"])
         st["v8"], st["vs"] = oracle.quantize_prefix(st["pv"], st["plen"])
+    if w.get("rope"):
+        tok, page = synth.page_positions(sample, 1, seed=seed + 2)
+        st["tok"], st["page"] = tok[:, 0].numpy().copy(), page[:, 0].numpy().copy()
     if w["kind"] == "srswa":
         pl = synth.plant_router_keys(plen, cap, n_dirs=1, seed=seed + 1)
         st["k_idx"] = u(pl.k_idx)
@@ -753,7 +920,12 @@ def oracle_sample_step(w: dict, sample: int, seed: int):
 
 def oracle_step(st: dict, w: dict):
     import oracle
-    oracle.append(st["rk"], st["rv"], st["k"], st["v"], st["wp"], st["fill"])
+    if w.get("rope"):  # the page2d encoding of this step's query and key, rounded to bf16
+        st = dict(st, q=oracle.bf16_round(oracle.rope_page2d(st["q"], st["tok"], st["page"])))
+        k = oracle.bf16_round(oracle.rope_page2d(st["k"], st["tok"], st["page"]))
+    else:
+        k = st["k"]
+    oracle.append(st["rk"], st["rv"], k, st["v"], st["wp"], st["fill"])
     if w["kind"] == "rswa":
         if w.get("fp8"):
             return oracle.rswa_decode_fp8(st["q"], st["k8"], st["v8"], st["ks"], st["vs"], st["plen"], st["rk"],
@@ -810,8 +982,40 @@ def oracle_prefill_step(st: dict, w: dict):
                                w["n"])
 
 
+ROPE_ORACLE_TOKENS = 512  # tokens of one sequence per oracle step of the encoding config
+
+
+def oracle_rope_case(w: dict, seed: int):
+    """Host q, k and positions of ROPE_ORACLE_TOKENS tokens of one sequence, and the work
+    fraction of a chunk they stand for."""
+    from long_context_decode_swa_b200 import synth
+    g = synth._gen(seed, "cpu")
+    shape = (ROPE_ORACLE_TOKENS, w["H"], w["D"])
+    q, k = synth.randn_bf16(shape, g, "cpu"), synth.randn_bf16(shape, g, "cpu")
+    tok, page = synth.page_positions(1, ROPE_ORACLE_TOKENS, seed=seed + 1)
+    st = dict(q=synth.to_u16(q), k=synth.to_u16(k), tok=tok[0].numpy().copy(), page=page[0].numpy().copy())
+    return st, ROPE_ORACLE_TOKENS / (w["B"] * w["T"])
+
+
+def oracle_rope_step(st: dict):
+    import oracle
+    return (oracle.bf16_round(oracle.rope_page2d(st["q"], st["tok"], st["page"])),
+            oracle.bf16_round(oracle.rope_page2d(st["k"], st["tok"], st["page"])))
+
+
 def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
     import oracle
+    if w["kind"] == "rope":
+        st, frac = oracle_rope_case(w, seed=77)
+        oracle_rope_step(st)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 2 or (time.perf_counter() - t0 < budget_s and reps < 200):
+            oracle_rope_step(st)
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+        return {"value": frac / dt, "unit": "encoded chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
+                "sample": f"{ROPE_ORACLE_TOKENS} of {w['B'] * w['T']} tokens (all heads, q and k), {reps} steps "
+                          f"timed; chunks/s extrapolated by the sample fraction; fp64 C oracle + bf16 rounding"}
     if w["kind"] in ("prefill", "srswa_prefill"):
         st, frac = oracle_prefill_case(w, 1, seed=77)
         oracle_prefill_step(st, w)
@@ -847,6 +1051,24 @@ def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
 def run_reference(args, w: dict) -> dict:
     """The oracle as the reference arm, on the host cores, K timed steps of a bounded sample."""
     import oracle
+    if w["kind"] == "rope":
+        st, frac = oracle_rope_case(w, seed=99)
+        for _ in range(args.warmup):
+            oracle_rope_step(st)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_rope_step(st)
+        value = frac / ((time.perf_counter() - t0) / args.steps)
+        cb = {"value": value, "unit": "encoded chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
+              "sample": f"{ROPE_ORACLE_TOKENS} of {w['B'] * w['T']} tokens per step (all heads, q and k); chunks/s "
+                        f"extrapolated by the sample fraction; fp64 C oracle on the host cores"}
+        return {"metric": METRIC, "value": value, "unit": "encoded chunks/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": w["B"]},
+                "cpu_baseline": cb,
+                "e2e": {"value": value, "unit": "encoded chunks/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     if w["kind"] in ("prefill", "srswa_prefill"):
         st, frac = oracle_prefill_case(w, 1, seed=99)
         for _ in range(args.warmup):
@@ -865,7 +1087,7 @@ def run_reference(args, w: dict) -> dict:
                 "cpu_baseline": cb,
                 "e2e": {"value": value, "unit": "prefill chunks/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
-    sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2}.get(args.config, 1))
+    sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2, 10: 2}.get(args.config, 1))
     st = oracle_sample_step(w, sample, seed=99)
     for _ in range(args.warmup):
         oracle_step(st, w)
@@ -920,7 +1142,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8, 9, 10])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")

@@ -86,7 +86,8 @@ typedef struct {
 RSWA_API const char* rswa_last_error(void);
 
 /* Library ABI version (incremented when entry points are added or changed): 2 adds the
- * FP8 prefix, the fused decode step and the SR-SWA chunked prefill to version 1. */
+ * FP8 prefix, the fused decode step and the SR-SWA chunked prefill to version 1; 3 adds
+ * the page2d rotary encoding (rswa_rope_page2d, rswa_append_rope). */
 RSWA_API int32_t rswa_version(void);
 
 /*
@@ -359,6 +360,47 @@ RSWA_API rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, cons
                                       const int32_t* blk_idx, const float* blk_logp, int32_t topk, const void* ring_k,
                                       const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
                                       float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * page2d rotary position encoding (Unlimited-OCR-2 SR-SWA explainer, 2D 位置编码: two
+ * rotary axes, sparse_rope_mode page2d; the token axis carries the token's offset inside
+ * its page, the page axis (page_mod: 2) the page number). The pages give no constants;
+ * this library's reading:
+ *   - pair i (i < D/2) couples dims i and i + D/2 (the LLaMA family's half split) and is
+ *     turned by angle a_i:  y_i = x_i cos a_i - x_{i+D/2} sin a_i,
+ *                           y_{i+D/2} = x_{i+D/2} cos a_i + x_i sin a_i;
+ *   - a_i = pos * base^(-2i/D), pos = page[r] when i mod page_mod == page_mod - 1 (the
+ *     page axis), else tok_pos[r] (the token axis); page_mod 0 = token axis only (plain
+ *     1-D rotary encoding); base = 10000 in the model family;
+ *   - computed in fp64 and rounded once to bf16 (round to nearest even).
+ * Keys are stored encoded (the prefix and the ring hold encoded keys); values and the
+ * router's index keys are not encoded.
+ *
+ * rswa_rope_page2d: encodes `rows` tokens of q (and of k) in one launch.
+ *   rows       : R >= 0 (R = 0 launches nothing); one token per row
+ *   q, q_out   : bf16 [R][heads][head_dim]; q_out may be q (in place)
+ *   k, k_out   : bf16 [R][heads][head_dim], or both NULL; k_out may be k
+ *   tok_pos, page : int32 [R] device arrays, any values
+ *   heads 1..128; head_dim a multiple of 16 in [16, 256]; base finite > 0; page_mod >= 0
+ *   No device-side checks; nothing is launched on a host-side error.
+ *
+ * rswa_append_rope: rswa_append of this step's token with its key encoded on the way
+ * into the ring, and its query encoded into q_out, in one launch (head_dim 128).
+ *   Arguments of rswa_append, plus q, q_out : bf16 [B][H][D] (q_out may be q) and
+ *   tok_pos, page : int32 [B] (this step's token positions), base, page_mod. q_out is
+ *   written whatever the ring state; a sequence with wp / fill out of range is flagged
+ *   and its ring left untouched, as in rswa_append.
+ * A decode step with the encoding: rswa_append_rope, then srswa_route + srswa_decode (or
+ * rswa_decode) on q_out; or rswa_rope_page2d on q and k_new, then rswa_decode_append.
+ */
+RSWA_API rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, const void* q, void* q_out,
+                                      const void* k, void* k_out, const int32_t* tok_pos, const int32_t* page,
+                                      double base, int32_t page_mod, void* stream);
+
+RSWA_API rswa_status rswa_append_rope(const rswa_dims* dims, void* ring_k, void* ring_v, const void* k_new,
+                                      const void* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, const void* q,
+                                      void* q_out, const int32_t* tok_pos, const int32_t* page, double base,
+                                      int32_t page_mod, int32_t* status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -6,8 +6,8 @@ seeded synthetic-input generators. There is no CPU fallback.
 """
 from .binding import (  # noqa: F401
     EXPORTED, LIB_PATH, OP_DECODE, OP_PREFILL, OP_ROUTE, OP_SRSWA_DECODE, Dims, RswaError, check_status, dims_of,
-    fp8_prefix_buffers, load, new_workspace, route_workspace, rswa_append, rswa_decode, rswa_decode_append,
-    rswa_decode_fp8, rswa_prefill,
+    fp8_prefix_buffers, load, new_workspace, route_workspace, rswa_append, rswa_append_rope, rswa_decode,
+    rswa_decode_append, rswa_decode_fp8, rswa_prefill, rswa_rope_page2d,
     rswa_quantize_prefix, srswa_decode, srswa_decode_append, srswa_decode_fp8, srswa_index_pool, srswa_prefill,
     srswa_route,
     srswa_route_tokens, workspace_bytes,
@@ -16,4 +16,5 @@ from .binding import (  # noqa: F401
 __all__ = ["load", "Dims", "RswaError", "rswa_append", "rswa_decode", "rswa_prefill", "srswa_index_pool", "srswa_route",
            "srswa_decode", "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "fp8_prefix_buffers",
            "srswa_route_tokens", "srswa_prefill", "rswa_decode_append", "srswa_decode_append",
+           "rswa_rope_page2d", "rswa_append_rope",
            "workspace_bytes", "new_workspace", "route_workspace", "check_status", "dims_of"]

@@ -37,7 +37,7 @@ DEVICE_PIPELINE = 0x10
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
             "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill",
             "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill",
-            "rswa_decode_append", "srswa_decode_append")
+            "rswa_decode_append", "srswa_decode_append", "rswa_rope_page2d", "rswa_append_rope")
 
 
 class RswaError(RuntimeError):
@@ -99,6 +99,8 @@ def load(path: str | None = None):
             "rswa_decode_append": ([DP, P, P, P, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_decode_append": ([DP, P, P, P, P, P, P, P, P, I32, P, P, P, P, P, F32, P, P, P, SZ, P],
                                     ctypes.c_int),
+            "rswa_rope_page2d": ([I64, I32, I32, P, P, P, P, P, P, ctypes.c_double, I32, P], ctypes.c_int),
+            "rswa_append_rope": ([DP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_double, I32, P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -184,6 +186,58 @@ def rswa_append(ring_k, ring_v, k_new, v_new, wp, fill, slot_out=None, status=No
     dims = Dims(B, H, D, n, 0)
     _check("rswa_append", load().rswa_append(ctypes.byref(dims), _ptr(ring_k), _ptr(ring_v), _ptr(k_new), _ptr(v_new),
                                              _ptr(wp), _ptr(fill), _ptr(slot_out), _ptr(status), _stream(stream)))
+
+
+def rswa_rope_page2d(q, tok_pos, page, q_out=None, k=None, k_out=None, base: float = 10000.0, page_mod: int = 2,
+                     stream=None):
+    """page2d rotary encoding of q (and k) bf16 [..., H, D], one token per leading index with
+    positions tok_pos / page (int32, shaped like the leading dims). q_out / k_out default to
+    in place. Returns (q_out, k_out)."""
+    if q.dim() < 2:
+        raise ValueError("q: expected [..., H, D]")
+    H, D = q.shape[-2:]
+    lead = tuple(q.shape[:-2])
+    _want(q, "q", torch.bfloat16)
+    q_out = q if q_out is None else _want(q_out, "q_out", torch.bfloat16, q.shape)
+    if k is not None:
+        _want(k, "k", torch.bfloat16, q.shape)
+        k_out = k if k_out is None else _want(k_out, "k_out", torch.bfloat16, q.shape)
+    elif k_out is not None:
+        raise ValueError("k_out given without k")
+    _want(tok_pos, "tok_pos", torch.int32, lead)
+    _want(page, "page", torch.int32, lead)
+    rows = q.numel() // (H * D) if q.numel() else 0
+    _check("rswa_rope_page2d", load().rswa_rope_page2d(rows, H, D, _ptr(q), _ptr(q_out), _ptr(k), _ptr(k_out),
+                                                       _ptr(tok_pos), _ptr(page), float(base), int(page_mod),
+                                                       _stream(stream)))
+    return q_out, k_out
+
+
+def rswa_append_rope(ring_k, ring_v, k_new, v_new, wp, fill, q, tok_pos, page, q_out=None, base: float = 10000.0,
+                     page_mod: int = 2, slot_out=None, status=None, stream=None):
+    """rswa_append with k_new page2d-encoded on its way into the ring and q encoded into q_out
+    (default: in place), one launch. Returns q_out."""
+    B, H, n, D = ring_k.shape
+    _want(ring_k, "ring_k", torch.bfloat16)
+    _want(ring_v, "ring_v", torch.bfloat16, ring_k.shape)
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    q_out = q if q_out is None else _want(q_out, "q_out", torch.bfloat16, (B, H, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(tok_pos, "tok_pos", torch.int32, (B,))
+    _want(page, "page", torch.int32, (B,))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    if status is not None:
+        _want(status, "status", status.dtype)
+    dims = Dims(B, H, D, n, 0)
+    _check("rswa_append_rope", load().rswa_append_rope(ctypes.byref(dims), _ptr(ring_k), _ptr(ring_v), _ptr(k_new),
+                                                       _ptr(v_new), _ptr(wp), _ptr(fill), _ptr(slot_out), _ptr(q),
+                                                       _ptr(q_out), _ptr(tok_pos), _ptr(page), float(base),
+                                                       int(page_mod), _ptr(status), _stream(stream)))
+    return q_out
 
 
 def rswa_decode(q, pk, pv, prefix_len, ring_k, ring_v, wp, fill, out, workspace, lse=None, scale=None, stream=None):

@@ -75,7 +75,7 @@ extern "C" {
 
 const char* rswa_last_error(void) { return g_last_error; }
 
-int32_t rswa_version(void) { return 2; }
+int32_t rswa_version(void) { return 3; }
 
 size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
   const char* fn = "rswa_workspace_bytes";
@@ -355,6 +355,63 @@ rswa_status rswa_quantize_prefix(const rswa_dims* dims, const void* pk, const vo
                                                static_cast<const uint16_t*>(pk), static_cast<const uint16_t*>(pv),
                                                prefix_len, pk8, pv8, k_scale, v_scale, status,
                                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+// page2d rotary encoding: the checks shared by both entry points.
+static rswa_status check_rope_params(const char* fn, const int32_t* tok_pos, const int32_t* page, double base,
+                                     int32_t page_mod) {
+  if (tok_pos == nullptr || page == nullptr) return fail(RSWA_ERR_INVALID, "%s: tok_pos and page must not be NULL", fn);
+  if (!(base > 0.0) || !std::isfinite(base)) return fail(RSWA_ERR_INVALID, "%s: base must be finite and > 0", fn);
+  if (page_mod < 0) return fail(RSWA_ERR_INVALID, "%s: page_mod must be >= 0 (got %d)", fn, page_mod);
+  return RSWA_OK;
+}
+
+rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, const void* q, void* q_out, const void* k,
+                             void* k_out, const int32_t* tok_pos, const int32_t* page, double base, int32_t page_mod,
+                             void* stream) {
+  const char* fn = "rswa_rope_page2d";
+  if (rows < 0) return fail(RSWA_ERR_INVALID, "%s: rows must be >= 0 (got %lld)", fn, (long long)rows);
+  if (heads < 1 || heads > 128) return fail(RSWA_ERR_INVALID, "%s: heads must be in [1, 128] (got %d)", fn, heads);
+  if (head_dim < 16 || head_dim > 256 || head_dim % 16 != 0)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: head_dim must be a multiple of 16 in [16, 256] (got %d)", fn, head_dim);
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(q_out);
+  if ((k == nullptr) != (k_out == nullptr)) return fail(RSWA_ERR_INVALID, "%s: k and k_out must both be given or both NULL", fn);
+  REQUIRE_PTR_OR_NULL(k);
+  REQUIRE_PTR_OR_NULL(k_out);
+  rswa_status st = check_rope_params(fn, tok_pos, page, base, page_mod);
+  if (st != RSWA_OK) return st;
+  if (rows == 0) return ok();
+  cudaError_t e = rswa::launch_rope(rows, heads, head_dim, static_cast<const uint16_t*>(q), static_cast<uint16_t*>(q_out),
+                                    static_cast<const uint16_t*>(k), static_cast<uint16_t*>(k_out), tok_pos, page, base,
+                                    page_mod, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+rswa_status rswa_append_rope(const rswa_dims* dims, void* ring_k, void* ring_v, const void* k_new, const void* v_new,
+                             int32_t* wp, int32_t* fill, int32_t* slot_out, const void* q, void* q_out,
+                             const int32_t* tok_pos, const int32_t* page, double base, int32_t page_mod, int32_t* status,
+                             void* stream) {
+  const char* fn = "rswa_append_rope";
+  rswa_status st = check_dims(fn, dims, false);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(ring_k);
+  REQUIRE_PTR(ring_v);
+  REQUIRE_PTR(k_new);
+  REQUIRE_PTR(v_new);
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(q_out);
+  if (wp == nullptr || fill == nullptr) return fail(RSWA_ERR_INVALID, "%s: wp and fill must not be NULL", fn);
+  st = check_rope_params(fn, tok_pos, page, base, page_mod);
+  if (st != RSWA_OK) return st;
+  cudaError_t e = rswa::launch_append_rope(
+      dims->batch, dims->heads, dims->ring, static_cast<uint16_t*>(ring_k), static_cast<uint16_t*>(ring_v),
+      static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), static_cast<const uint16_t*>(q),
+      static_cast<uint16_t*>(q_out), tok_pos, page, base, page_mod, wp, fill, slot_out, status,
+      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
 }

@@ -74,6 +74,15 @@ cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_
                           const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status,
                           cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream);
+// page2d rotary encoding of rows x [H][D] of q (and k when not NULL); outputs may alias inputs.
+cudaError_t launch_rope(int64_t rows, int H, int D, const uint16_t* q, uint16_t* q_out, const uint16_t* k,
+                        uint16_t* k_out, const int32_t* tok_pos, const int32_t* page, double base, int page_mod,
+                        cudaStream_t stream);
+// launch_append with the new key rotated (page2d) before it is written and the query rotated into q_out.
+cudaError_t launch_append_rope(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_v, const uint16_t* k_new,
+                               const uint16_t* v_new, const uint16_t* q, uint16_t* q_out, const int32_t* tok_pos,
+                               const int32_t* page, double base, int page_mod, int32_t* wp, int32_t* fill,
+                               int32_t* slot_out, int32_t* status, cudaStream_t stream);
 cudaError_t launch_quantize_prefix(int B, int H, int64_t cap, const uint16_t* pk, const uint16_t* pv,
                                    const int32_t* prefix_len, uint8_t* pk8, uint8_t* pv8, float* k_scale,
                                    float* v_scale, int32_t* status, cudaStream_t stream);

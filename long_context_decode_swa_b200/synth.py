@@ -18,6 +18,9 @@ page plus a 32-token prompt as the reference prefix, a 128-slot output ring):
 * An FP8 prefix drawn directly (``fp8_prefix``): uniformly random finite E4M3
   code bytes (the two NaN codes excluded) and log-uniform positive block
   scales, a valid stored cache without going through any quantiser.
+* Token positions for the page2d encoding (``page_positions``): consecutive
+  output tokens walk through pages of 200-2000 tokens from a random start page
+  below 400 and a random offset in it.
 """
 from __future__ import annotations
 
@@ -237,6 +240,31 @@ def log_uniform_pages(B: int, lo: int, hi: int, seed: int) -> list[int]:
     u = torch.rand(B, generator=g, dtype=torch.float64)
     pages = torch.exp(math.log(lo) + u * (math.log(hi + 1) - math.log(lo))).floor().clamp(lo, hi)
     return [int(p) for p in pages]
+
+
+def page_positions(B: int, T: int, seed: int, page_len=(200, 2000), first_page=(0, 400), device="cpu"):
+    """Page layout of T consecutive output tokens per sequence, for the page2d encoding:
+    (tok_pos, page), int32 [B][T]. Each sequence starts on a page drawn from
+    [first_page[0], first_page[1]) at an offset inside it; pages hold a number of tokens
+    drawn from [page_len[0], page_len[1]] (a per-page output length, below the pages'
+    20000-token per-page cap); tok_pos is the token's offset inside its page and restarts
+    at 0 on each new page. CPU generator, device independent."""
+    g = _gen(seed, "cpu")
+    lo, hi = page_len
+    n_pages = T // lo + 2
+    tok = torch.empty((B, T), dtype=torch.int32)
+    pg = torch.empty((B, T), dtype=torch.int32)
+    for b in range(B):
+        lens = torch.randint(lo, hi + 1, (n_pages,), generator=g)
+        start_off = int(torch.randint(0, int(lens[0]), (1,), generator=g))
+        p0 = int(torch.randint(first_page[0], first_page[1], (1,), generator=g))
+        ends = torch.cumsum(lens, 0) - start_off                       # first token index past each page
+        t = torch.arange(T)
+        j = torch.searchsorted(ends, t, right=True)                   # page (relative) of token t
+        begin = torch.where(j > 0, ends[(j - 1).clamp(min=0)], torch.full_like(t, -start_off))
+        tok[b] = (t - begin).to(torch.int32)
+        pg[b] = (p0 + j).to(torch.int32)
+    return tok.to(device), pg.to(device)
 
 
 def to_u16(t: torch.Tensor):

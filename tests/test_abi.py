@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     lib = rswa.load()
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.rswa_version() == 2
+    assert lib.rswa_version() == 3
 
 
 def _err():
@@ -152,3 +152,39 @@ def test_fused_step_validation():
     assert call(k_new=None) == INVALID and "k_new" in _err()
     assert call(k_new=MIS) == INVALID and "aligned" in _err()
     assert call(ws_bytes=255) == INVALID and "workspace" in _err()
+
+
+def test_rope_entry_points_validation():
+    lib = rswa.load()
+    D64 = ctypes.c_double
+
+    def rope(rows=8, heads=4, head_dim=128, q=A, q_out=A, k=None, k_out=None, tok=A, page=A2, base=1e4, page_mod=2):
+        return lib.rswa_rope_page2d(rows, heads, head_dim, q, q_out, k, k_out, tok, page, D64(base), page_mod, None)
+
+    assert rope(rows=-1) == INVALID and "rows" in _err()
+    assert rope(heads=0) == INVALID and "heads" in _err()
+    assert rope(head_dim=100) == UNSUPPORTED and "head_dim" in _err()
+    assert rope(head_dim=272) == UNSUPPORTED
+    assert rope(q=None) == INVALID and "q must not be NULL" in _err()
+    assert rope(q_out=MIS) == INVALID and "aligned" in _err()
+    assert rope(k=A) == INVALID and "both" in _err()
+    assert rope(k=MIS, k_out=A) == INVALID and "aligned" in _err()
+    assert rope(tok=None) == INVALID and "tok_pos" in _err()
+    assert rope(base=0.0) == INVALID and "base" in _err()
+    assert rope(base=float("inf")) == INVALID
+    assert rope(page_mod=-1) == INVALID and "page_mod" in _err()
+    assert rope(rows=0) == 0 and _err() == ""          # nothing to encode: no launch
+
+    d = Dims(2, 4, 128, 128, 0)
+
+    def app(dims=d, q=A, q_out=A, wp=A, page=A2, base=1e4, page_mod=2):
+        return lib.rswa_append_rope(ctypes.byref(dims), A, A, A, A, wp, A, None, q, q_out, A, page, D64(base),
+                                    page_mod, None, None)
+
+    assert app(dims=Dims(2, 4, 64, 128, 0)) == UNSUPPORTED and "head_dim" in _err()
+    assert app(q=None) == INVALID and "q must not be NULL" in _err()
+    assert app(q_out=MIS) == INVALID and "aligned" in _err()
+    assert app(wp=None) == INVALID and "wp and fill" in _err()
+    assert app(page=None) == INVALID and "page" in _err()
+    assert app(base=float("nan")) == INVALID and "base" in _err()
+    assert app(page_mod=-2) == INVALID and "page_mod" in _err()
