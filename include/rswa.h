@@ -377,7 +377,8 @@ RSWA_API rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, cons
  * router's index keys are not encoded.
  *
  * rswa_rope_page2d: encodes `rows` tokens of q (and of k) in one launch.
- *   rows       : R >= 0 (R = 0 launches nothing); one token per row
+ *   rows       : R >= 0; one token per row. R = 0 launches nothing and accepts NULL
+ *                buffers (after the checks of heads, head_dim, base and page_mod)
  *   q, q_out   : bf16 [R][heads][head_dim]; q_out may be q (in place)
  *   k, k_out   : bf16 [R][heads][head_dim], or both NULL; k_out may be k
  *   tok_pos, page : int32 [R] device arrays, any values

@@ -376,6 +376,9 @@ rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, cons
   if (heads < 1 || heads > 128) return fail(RSWA_ERR_INVALID, "%s: heads must be in [1, 128] (got %d)", fn, heads);
   if (head_dim < 16 || head_dim > 256 || head_dim % 16 != 0)
     return fail(RSWA_ERR_UNSUPPORTED, "%s: head_dim must be a multiple of 16 in [16, 256] (got %d)", fn, head_dim);
+  if (!(base > 0.0) || !std::isfinite(base)) return fail(RSWA_ERR_INVALID, "%s: base must be finite and > 0", fn);
+  if (page_mod < 0) return fail(RSWA_ERR_INVALID, "%s: page_mod must be >= 0 (got %d)", fn, page_mod);
+  if (rows == 0) return ok();  // nothing to encode; the (empty) buffers may be NULL
   REQUIRE_PTR(q);
   REQUIRE_PTR(q_out);
   if ((k == nullptr) != (k_out == nullptr)) return fail(RSWA_ERR_INVALID, "%s: k and k_out must both be given or both NULL", fn);
@@ -383,7 +386,6 @@ rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, cons
   REQUIRE_PTR_OR_NULL(k_out);
   rswa_status st = check_rope_params(fn, tok_pos, page, base, page_mod);
   if (st != RSWA_OK) return st;
-  if (rows == 0) return ok();
   cudaError_t e = rswa::launch_rope(rows, heads, head_dim, static_cast<const uint16_t*>(q), static_cast<uint16_t*>(q_out),
                                     static_cast<const uint16_t*>(k), static_cast<uint16_t*>(k_out), tok_pos, page, base,
                                     page_mod, static_cast<cudaStream_t>(stream));

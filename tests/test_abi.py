@@ -174,6 +174,8 @@ def test_rope_entry_points_validation():
     assert rope(base=float("inf")) == INVALID
     assert rope(page_mod=-1) == INVALID and "page_mod" in _err()
     assert rope(rows=0) == 0 and _err() == ""          # nothing to encode: no launch
+    assert rope(rows=0, q=None, q_out=None, tok=None, page=None) == 0     # empty tensors have NULL data
+    assert rope(rows=0, head_dim=100) == UNSUPPORTED and rope(rows=0, base=-1.0) == INVALID
 
     d = Dims(2, 4, 128, 128, 0)
 
