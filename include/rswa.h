@@ -372,7 +372,9 @@ RSWA_API rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, cons
  *   - a_i = pos * base^(-2i/D), pos = page[r] when i mod page_mod == page_mod - 1 (the
  *     page axis), else tok_pos[r] (the token axis); page_mod 0 = token axis only (plain
  *     1-D rotary encoding); base = 10000 in the model family;
- *   - computed in fp64 and rounded once to bf16 (round to nearest even).
+ *   - angles and their cos / sin in fp64, cos / sin rounded to f32, the rotation in f32
+ *     (one product and one FMA per output), the result rounded to bf16 (nearest even):
+ *     within 2^-22 (|x_i| + |x_{i+D/2}|) plus half a bf16 step of the exact rotation.
  * Keys are stored encoded (the prefix and the ring hold encoded keys); values and the
  * router's index keys are not encoded.
  *

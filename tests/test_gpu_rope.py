@@ -1,10 +1,15 @@
 """GPU parity of the page2d rotary encoding (rswa_rope_page2d, rswa_append_rope) against
-the oracle's fp64 rotation rounded to bf16 (oracle.bf16_round).
+the oracle's fp64 rotation (oracle.rope_page2d).
 
-Both sides rotate the same bf16 inputs by the same angles in fp64 and round once, so
-the bf16 outputs agree bit for bit except where the exact result lies within the last
-bits of an fp64 angle of a rounding tie; the bar is: every element within 1 bf16 ulp
-and at most 1 in 10^5 elements (or 1) not bit-identical. The ring append around the
+Tolerance, from the kernel's arithmetic: it takes each angle in fp64, rounds cos and sin
+to fp32 and forms x_i cos - x_{i+D/2} sin (and the partner) with one fp32 product and one
+fp32 FMA. Each of those four roundings errs by at most 2^-24 of a term no larger than
+|x_i| + |x_{i+D/2}|, so before its final rounding an output is within
+E = 2^-22 (|x_i| + |x_{i+D/2}|) of the exact rotation (the fp64 angles differ from the
+oracle's by ~1e-16 relative, negligible). Rounding to bf16 adds at most half a bf16 step
+of the result. The test asserts |got - exact| <= E + half a step for every element, and
+that at most 1 in 1000 elements differ from the correctly rounded value (oracle.bf16_round
+of the exact rotation; the expected share is about 1e-4). The ring append around the
 encoding is bit-exact (slot, wp, fill, untouched slots, the value row)."""
 import numpy as np
 import pytest
@@ -17,20 +22,27 @@ from tests.gpu_util import LSE_ABS, assert_attention_close, to_np
 pytestmark = pytest.mark.gpu
 
 
-def _bf16_ulps(a: np.ndarray, b: np.ndarray) -> np.ndarray:
-    """Distance in bf16 steps between two arrays of finite bf16 patterns."""
-    def ordered(x):
-        x = x.astype(np.int32)
-        return np.where(x & 0x8000, 0x8000 - x, x)       # monotone map of the sign-magnitude patterns
-    return np.abs(ordered(a) - ordered(b))
+def _step(v: np.ndarray) -> np.ndarray:
+    """Spacing of the bf16 grid at |v| (2^-133 at zero and in the subnormal range)."""
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(np.maximum(e - 7, -133)), 2.0 ** -133)
 
 
-def assert_rope_match(got_bits: np.ndarray, want_bits: np.ndarray, what: str):
-    assert got_bits.shape == want_bits.shape, what
-    d = _bf16_ulps(got_bits, want_bits)
-    bad = int((d != 0).sum())
-    assert d.max() <= 1, f"{what}: {d.max()} bf16 ulps off"
-    assert bad <= max(1, d.size // 100000), f"{what}: {bad} of {d.size} elements not bit-identical"
+def assert_rope_close(got_bits: np.ndarray, x_bits: np.ndarray, tok, page, base, page_mod, what: str):
+    """got_bits: the kernel's bf16 output for the bf16 input rows x_bits [..., H, D]."""
+    exact = oracle.rope_page2d(x_bits, tok, page, base=base, page_mod=page_mod)
+    assert got_bits.shape == exact.shape, what
+    got = oracle.bf16_bits_to_f64(got_bits)
+    x = np.abs(oracle.bf16_bits_to_f64(x_bits))
+    h = x.shape[-1] // 2
+    pair = x[..., :h] + x[..., h:]
+    bound = 2.0 ** -22 * np.concatenate([pair, pair], axis=-1) + 0.5 * _step(got)
+    err = np.abs(got - exact)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert (err <= bound).all(), f"{what}: error {err[worst]:.3e} above bound {bound[worst]:.3e} at {worst}"
+    off = int((got_bits != oracle.bf16_round(exact)).sum())
+    assert off <= max(1, got_bits.size // 1000), f"{what}: {off} of {got_bits.size} not correctly rounded"
 
 
 def _positions(rows, seed, neg=False):
@@ -38,10 +50,6 @@ def _positions(rows, seed, neg=False):
     tok = rng.integers(-50 if neg else 0, 20000, rows).astype(np.int32)
     page = rng.integers(-5 if neg else 0, 400, rows).astype(np.int32)
     return tok, page
-
-
-def _oracle_bits(x_bits, tok, page, base, page_mod):
-    return oracle.bf16_round(oracle.rope_page2d(x_bits, tok, page, base=base, page_mod=page_mod))
 
 
 @pytest.mark.parametrize("rows,H,D,page_mod,base", [
@@ -60,18 +68,18 @@ def test_rope_page2d_matches_oracle(cuda_lib, rows, H, D, page_mod, base):
     cuda_lib.rswa_rope_page2d(q, torch.from_numpy(tok).cuda(), torch.from_numpy(page).cuda(), q_out=q_out, k=k,
                               k_out=k_out, base=base, page_mod=page_mod)
     torch.cuda.synchronize()
-    assert_rope_match(to_np(q_out), _oracle_bits(to_np(q), tok, page, base, page_mod), "q")
-    assert_rope_match(to_np(k_out), _oracle_bits(to_np(k), tok, page, base, page_mod), "k")
+    assert_rope_close(to_np(q_out), to_np(q), tok, page, base, page_mod, "q")
+    assert_rope_close(to_np(k_out), to_np(k), tok, page, base, page_mod, "k")
 
 
 def test_rope_page2d_in_place_q_only_and_empty(cuda_lib):
     g = synth._gen(910, "cuda")
     x = synth.randn_bf16((4, 7, 9, 128), g, "cuda")          # leading dims [4][7] = 28 tokens
     tok, page = synth.page_positions(4, 7, seed=911)
-    want = _oracle_bits(to_np(x), tok.numpy(), page.numpy(), 10000.0, 2)
+    x_in = to_np(x).copy()
     cuda_lib.rswa_rope_page2d(x, tok.cuda(), page.cuda())    # in place, no k
     torch.cuda.synchronize()
-    assert_rope_match(to_np(x), want, "in place")
+    assert_rope_close(to_np(x), x_in, tok.numpy(), page.numpy(), 10000.0, 2, "in place")
     empty = torch.empty((0, 4, 128), dtype=torch.bfloat16, device="cuda")
     z = torch.empty(0, dtype=torch.int32, device="cuda")
     cuda_lib.rswa_rope_page2d(empty, z, z)                    # nothing launched, no error
@@ -87,8 +95,8 @@ def test_rope_page2d_prefill_chunk_full_size(cuda_lib):
     q_out, k_out = torch.empty_like(q), torch.empty_like(k)
     cuda_lib.rswa_rope_page2d(q, tok.cuda(), page.cuda(), q_out=q_out, k=k, k_out=k_out)
     torch.cuda.synchronize()
-    assert_rope_match(to_np(q_out), _oracle_bits(to_np(q), tok.numpy(), page.numpy(), 10000.0, 2), "q chunk")
-    assert_rope_match(to_np(k_out), _oracle_bits(to_np(k), tok.numpy(), page.numpy(), 10000.0, 2), "k chunk")
+    assert_rope_close(to_np(q_out), to_np(q), tok.numpy(), page.numpy(), 10000.0, 2, "q chunk")
+    assert_rope_close(to_np(k_out), to_np(k), tok.numpy(), page.numpy(), 10000.0, 2, "k chunk")
 
 
 @pytest.mark.parametrize("B,H,n", [(6, 16, 128), (3, 20, 40), (2, 40, 7)])
@@ -105,8 +113,9 @@ def test_append_rope_matches_oracle(cuda_lib, B, H, n):
     wp[-1] = -1                                                   # a bad ring state: flagged, ring untouched
     tok, page = _positions(B, seed=H + 1)
     o_rk, o_rv = to_np(ring_k).copy(), to_np(ring_v).copy()
-    want_q = _oracle_bits(to_np(q), tok, page, 10000.0, 2)
-    want_k = _oracle_bits(to_np(k_new), tok, page, 10000.0, 2)
+    k_bits = to_np(k_new)
+    # the ring holds the kernel's encoded key; the oracle's append takes the correctly rounded one
+    want_k = oracle.bf16_round(oracle.rope_page2d(k_bits, tok, page))
     t_wp, t_fill = torch.from_numpy(wp).cuda(), torch.from_numpy(fill).cuda()
     slot = torch.full((B,), -7, dtype=torch.int32, device="cuda")
     status = torch.zeros(64, dtype=torch.int32, device="cuda")
@@ -114,7 +123,7 @@ def test_append_rope_matches_oracle(cuda_lib, B, H, n):
     cuda_lib.rswa_append_rope(ring_k, ring_v, k_new, v_new, t_wp, t_fill, q, torch.from_numpy(tok).cuda(),
                               torch.from_numpy(page).cuda(), q_out=q_out, slot_out=slot, status=status)
     assert cuda_lib.check_status(status) == 0x2                     # RSWA_DEVICE_BAD_RING_STATE
-    assert_rope_match(to_np(q_out), want_q, "q_out")
+    assert_rope_close(to_np(q_out), to_np(q), tok, page, 10000.0, 2, "q_out")
     # the oracle's append of the encoded key for the sequences with a valid ring
     ok = slice(0, B - 1)
     o_wp, o_fill = wp[ok].copy(), fill[ok].copy()
@@ -126,7 +135,8 @@ def test_append_rope_matches_oracle(cuda_lib, B, H, n):
     got_rk, got_rv = to_np(ring_k), to_np(ring_v)
     for b in range(B - 1):
         s = o_slot[b]
-        assert_rope_match(got_rk[b, :, s], o_rk_ok[b, :, s], f"ring_k slot b={b}")
+        assert_rope_close(got_rk[b, :, s][None], k_bits[b][None], tok[b:b + 1], page[b:b + 1], 10000.0, 2,
+                          f"ring_k slot b={b}")
         others = np.arange(n) != s
         np.testing.assert_array_equal(got_rk[b][:, others], o_rk_ok[b][:, others])
         np.testing.assert_array_equal(got_rv[b], o_rv_ok[b])
@@ -160,8 +170,8 @@ def test_srswa_step_with_page2d_encoding(cuda_lib):
         cuda_lib.srswa_decode(q_rot, case.pk, case.pv, case.prefix_len, torch.from_numpy(blk).cuda(),
                               torch.from_numpy(logp).cuda(), ring_k, ring_v, wp, fill, out, ws, lse=lse,
                               scale=case.scale)
-        qo = _oracle_bits(to_np(case.q[s]), t_s.numpy(), p_s.numpy(), 10000.0, 2)
-        ko = _oracle_bits(to_np(case.k_new[s]), t_s.numpy(), p_s.numpy(), 10000.0, 2)
+        qo = oracle.bf16_round(oracle.rope_page2d(to_np(case.q[s]), t_s.numpy(), p_s.numpy()))
+        ko = oracle.bf16_round(oracle.rope_page2d(to_np(case.k_new[s]), t_s.numpy(), p_s.numpy()))
         oracle.append(o_rk, o_rv, ko, to_np(case.v_new[s]), o_wp, o_fill)
         ref, ref_lse = oracle.srswa_decode(qo, to_np(case.pk), to_np(case.pv), to_np(case.prefix_len), blk,
                                            logp.astype(np.float64), o_rk, o_rv, o_wp, o_fill, case.scale)
