@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kRopeThreads = 256;
 constexpr int kRopeMaxHalf = 128;  // D <= 256
-constexpr int kRopeCtasPerSm = 8;
+constexpr int kRopeCtasPerSm = 4;   // resident CTAs per SM (64 registers a thread)
 constexpr int kRopeMaxGroup = 8;    // tokens per CTA iteration
 constexpr int kRopeUnits = 4;       // chunk pairs a thread holds per pass
 
@@ -63,7 +63,7 @@ __device__ __forceinline__ void rotate8(uint4& lo, uint4& hi, const float2* cs) 
 }
 
 // rows x [H][D] of q (and k): one row per token with positions tok_pos[r], page[r].
-__global__ void __launch_bounds__(kRopeThreads) rope_kernel(int64_t rows, int H, int D, int group, const uint16_t* q,
+__global__ void __launch_bounds__(kRopeThreads, kRopeCtasPerSm) rope_kernel(int64_t rows, int H, int D, int group, const uint16_t* q,
                                                            uint16_t* q_out, const uint16_t* k, uint16_t* k_out,
                                                            const int32_t* __restrict__ tok_pos,
                                                            const int32_t* __restrict__ page, double log2_base,
