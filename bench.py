@@ -1003,7 +1003,34 @@ def oracle_rope_step(st: dict):
             oracle.bf16_round(oracle.rope_page2d(st["k"], st["tok"], st["page"])))
 
 
-def cpu_baseline(w: dict, budget_s: float = 12.0) -> dict:
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo", encoding="utf-8"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(w: dict, budget_s: float = 12.0, budget_1thread_s: float = 3.0) -> dict:
+    """The oracle on all host threads (the reported value), plus a shorter 1-thread figure."""
+    import oracle
+    res = _cpu_baseline_run(w, budget_s)
+    threads = oracle.get_threads()
+    try:
+        oracle.set_threads(1)
+        one = _cpu_baseline_run(w, budget_1thread_s)
+    finally:
+        oracle.set_threads(threads)
+    res["value_1thread"] = one["value"]
+    res["sample_1thread"] = one["sample"]
+    res["host_cpus"] = os.cpu_count()
+    res["cpu_model"] = cpu_model()
+    return res
+
+
+def _cpu_baseline_run(w: dict, budget_s: float) -> dict:
     import oracle
     if w["kind"] == "rope":
         st, frac = oracle_rope_case(w, seed=77)

@@ -827,6 +827,7 @@ uint16_t oracle_bf16_round(double x) {
 }
 
 void oracle_bf16_round_array(int64_t count, const double* x, uint16_t* out) {
+#pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < count; ++i) out[i] = oracle_bf16_round(x[i]);
 }
 
