@@ -1014,46 +1014,45 @@ def cpu_model() -> str:
 
 
 def cpu_baseline(w: dict, budget_s: float = 12.0, budget_1thread_s: float = 3.0) -> dict:
-    """The oracle on all host threads (the reported value), plus a shorter 1-thread figure."""
+    """The oracle as it stands, on all host threads (the reported value) and, over the same
+    sample for a shorter time, on one thread."""
     import oracle
-    res = _cpu_baseline_run(w, budget_s)
+    step, frac, unit, what, lo, hi = _cpu_baseline_case(w, budget_s)
     threads = oracle.get_threads()
+    dt, reps = _time_steps(step, budget_s, lo, hi)
     try:
         oracle.set_threads(1)
-        one = _cpu_baseline_run(w, budget_1thread_s)
+        dt1, reps1 = _time_steps(step, budget_1thread_s, 1, hi)
     finally:
         oracle.set_threads(threads)
-    res["value_1thread"] = one["value"]
-    res["sample_1thread"] = one["sample"]
-    res["host_cpus"] = os.cpu_count()
-    res["cpu_model"] = cpu_model()
-    return res
+    return {"value": frac / dt, "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": f"{what}, {reps} steps timed; {unit} extrapolated by the sample fraction; fp64 C oracle "
+                      f"(OpenMP over independent problems)",
+            "value_1thread": frac / dt1, "steps_1thread": reps1, "host_cpus": os.cpu_count(),
+            "cpu_model": cpu_model()}
 
 
-def _cpu_baseline_run(w: dict, budget_s: float) -> dict:
-    import oracle
+def _time_steps(step, budget_s: float, min_reps: int, max_reps: int):
+    reps, t0 = 0, time.perf_counter()
+    while reps < min_reps or (time.perf_counter() - t0 < budget_s and reps < max_reps):
+        step()
+        reps += 1
+    return (time.perf_counter() - t0) / reps, reps
+
+
+def _cpu_baseline_case(w: dict, budget_s: float):
+    """(step function, work fraction of one full step, unit, sample description, min / max
+    timed steps) of a bounded oracle sample of the workload, warmed up once."""
     if w["kind"] == "rope":
         st, frac = oracle_rope_case(w, seed=77)
         oracle_rope_step(st)
-        reps, t0 = 0, time.perf_counter()
-        while reps < 2 or (time.perf_counter() - t0 < budget_s and reps < 200):
-            oracle_rope_step(st)
-            reps += 1
-        dt = (time.perf_counter() - t0) / reps
-        return {"value": frac / dt, "unit": "encoded chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
-                "sample": f"{ROPE_ORACLE_TOKENS} of {w['B'] * w['T']} tokens (all heads, q and k), {reps} steps "
-                          f"timed; chunks/s extrapolated by the sample fraction; fp64 C oracle + bf16 rounding"}
+        return (lambda: oracle_rope_step(st)), frac, "encoded chunks/s", \
+            f"{ROPE_ORACLE_TOKENS} of {w['B'] * w['T']} tokens (all heads, q and k)", 2, 200
     if w["kind"] in ("prefill", "srswa_prefill"):
         st, frac = oracle_prefill_case(w, 1, seed=77)
         oracle_prefill_step(st, w)
-        reps, t0 = 0, time.perf_counter()
-        while reps < 1 or (time.perf_counter() - t0 < budget_s and reps < 20):
-            oracle_prefill_step(st, w)
-            reps += 1
-        dt = (time.perf_counter() - t0) / reps
-        return {"value": frac / dt, "unit": "prefill chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
-                "sample": f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows (all heads), "
-                          f"{reps} steps timed; chunks/s extrapolated by the sample fraction; fp64 C oracle"}
+        return (lambda: oracle_prefill_step(st, w)), frac, "prefill chunks/s", \
+            f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows (all heads)", 1, 20
     sample = min(w["B"], 2)
     st = oracle_sample_step(w, sample, seed=77)
     oracle_step(st, w)                               # warm (and pool the router keys)
@@ -1064,15 +1063,8 @@ def _cpu_baseline_run(w: dict, budget_s: float) -> dict:
     sample = int(max(1, min(w["B"], sample * budget_s / max(one, 1e-3) / 3)))
     st = oracle_sample_step(w, sample, seed=78)
     oracle_step(st, w)
-    reps, t0 = 0, time.perf_counter()
-    while reps < 2 or (time.perf_counter() - t0 < budget_s and reps < 50):
-        oracle_step(st, w)
-        reps += 1
-    dt = (time.perf_counter() - t0) / reps
-    frac = sample / w["B"]
-    return {"value": frac / dt, "unit": "steps/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": f"{sample} of {w['B']} sequences per step (all heads), {reps} steps timed; "
-                      f"steps/s extrapolated by the sample fraction; fp64 C oracle, OpenMP"}
+    return (lambda: oracle_step(st, w)), sample / w["B"], "steps/s", \
+        f"{sample} of {w['B']} sequences per step (all heads)", 2, 50
 
 
 def run_reference(args, w: dict) -> dict:
