@@ -8,10 +8,21 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace {
+
+// An NVTX range named after the entry point around each call that launches work (it shows
+// in Nsight timelines; without an attached tool the calls are no-ops).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 thread_local char g_last_error[512] = "";
 
@@ -135,6 +146,7 @@ rswa_status rswa_check_status(void* workspace, size_t ws_bytes, int32_t* device_
 rswa_status rswa_append(const rswa_dims* dims, void* ring_k, void* ring_v, const void* k_new, const void* v_new,
                         int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status, void* stream) {
   const char* fn = "rswa_append";
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, false);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(ring_k);
@@ -189,6 +201,7 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
                                  const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                                  const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0) {
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q);
@@ -340,6 +353,7 @@ rswa_status rswa_quantize_prefix(const rswa_dims* dims, const void* pk, const vo
                                  uint8_t* pk8, uint8_t* pv8, float* k_scale, float* v_scale, int32_t* status,
                                  void* stream) {
   const char* fn = "rswa_quantize_prefix";
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(pk);
@@ -372,6 +386,7 @@ rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, cons
                              void* k_out, const int32_t* tok_pos, const int32_t* page, double base, int32_t page_mod,
                              void* stream) {
   const char* fn = "rswa_rope_page2d";
+  const NvtxRange nvtx_range(fn);
   if (rows < 0) return fail(RSWA_ERR_INVALID, "%s: rows must be >= 0 (got %lld)", fn, (long long)rows);
   if (heads < 1 || heads > 128) return fail(RSWA_ERR_INVALID, "%s: heads must be in [1, 128] (got %d)", fn, heads);
   if (head_dim < 16 || head_dim > 256 || head_dim % 16 != 0)
@@ -398,6 +413,7 @@ rswa_status rswa_append_rope(const rswa_dims* dims, void* ring_k, void* ring_v, 
                              const int32_t* tok_pos, const int32_t* page, double base, int32_t page_mod, int32_t* status,
                              void* stream) {
   const char* fn = "rswa_append_rope";
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, false);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(ring_k);
@@ -455,6 +471,7 @@ rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const 
                          int32_t* wp, int32_t* fill, float scale, float* out, float* lse, int32_t write_ring,
                          void* workspace, size_t ws_bytes, void* stream) {
   const char* fn = "rswa_prefill";
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   if (T < 1) return fail(RSWA_ERR_INVALID, "%s: T must be >= 1 (got %d)", fn, T);
@@ -516,6 +533,7 @@ rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const 
 rswa_status srswa_index_pool(const rswa_dims* dims, const void* k_idx, const int32_t* prefix_len, float* kbar,
                              void* stream) {
   const char* fn = "srswa_index_pool";
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(k_idx);
@@ -532,6 +550,7 @@ static rswa_status route_common(const char* fn, const rswa_dims* dims, int token
                                 const float* kbar, const int32_t* prefix_len, float idx_scale, int32_t topk,
                                 int32_t* blk_idx, float* blk_logp, float* probs, float* tau, void* workspace,
                                 size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q_idx);
@@ -628,6 +647,7 @@ rswa_status rswa_decode_noalloc(const rswa_dims* dims, const void* q, const void
                                 const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                                 int32_t* status, void* stream) {
   const char* fn = "rswa_decode_noalloc";
+  const NvtxRange nvtx_range(fn);
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q);
