@@ -190,3 +190,13 @@ def test_rope_entry_points_validation():
     assert app(page=None) == INVALID and "page" in _err()
     assert app(base=float("nan")) == INVALID and "base" in _err()
     assert app(page_mod=-2) == INVALID and "page_mod" in _err()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # no CPU fallback: without the library every call path raises
+    import subprocess
+    import sys
+    env = dict(os.environ, RSWA_LIBRARY=str(tmp_path / "absent" / "librswa.so"))
+    code = "import long_context_decode_swa_b200 as r\nr.load()"
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT, timeout=300)
+    assert out.returncode != 0 and "not found" in out.stderr
