@@ -316,9 +316,10 @@ RSWA_API rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void*
                                    float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * FP8 prefix cache (the pages name quantised KV-cache compression as a next step,
- * "百度 Unlimited OCR 深度实战" tutorial, future directions, KV缓存压缩, without fixing a
- * format; the format below is this library's reading). The prefix K and V are stored
+ * FP8 prefix cache (the Unlimited-OCR technical analysis page, "Unlimited-OCR：突破32768
+ * 上下文限制的视觉语言模型技术解析", lists quantised KV-cache compression among its memory
+ * measures, 内存使用效率 / KV缓存压缩, without fixing a format; the format below is this
+ * library's reading). The prefix K and V are stored
  * as OCP FP8 E4M3 codes (bias 7, 3 mantissa bits, subnormals, largest finite 448, no
  * infinities) with one f32 scale per (sequence, head, 32-token block) for K and one
  * for V; an element is code value * scale. The ring stays bf16.

@@ -1,7 +1,8 @@
 // quant.cu -- FP8 (E4M3) prefix quantisation with per-(sequence, head, block) scales.
 //
-// The pages name quantised KV-cache compression as a next step (tutorial, future
-// directions, KV缓存压缩) without a format; this library's reading: E4M3 codes with one
+// The Unlimited-OCR technical analysis page lists quantised KV-cache compression among
+// its memory measures (内存使用效率, KV缓存压缩) without a format; this library's
+// reading: E4M3 codes with one
 // f32 scale per (sequence, head, 32-token block) for K and one for V, scale = amax / 448
 // over the block's valid rows, code = E4M3(x / scale) rounded to nearest even and
 // saturating at +-448, both steps in f32 (IEEE division, as written). Rows of a partial

@@ -80,6 +80,11 @@ def _L():
             lib.oracle_bf16_round.restype = ctypes.c_uint16
             lib.oracle_bf16_round_array.argtypes = [I64, P, P]
             lib.oracle_rope_page2d.argtypes = [I64, I, I, P, P, P, Dbl, I, P]
+            lib.oracle_append_fp8.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, P]
+            lib.oracle_rswa_decode_fp8kv.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, P, P, P, P, Dbl,
+                                                     P, P]
+            lib.oracle_srswa_decode_fp8kv.argtypes = [I, I, I, I, I64, I, P, P, P, P, P, P, P, P, I, P, P, P, P, P,
+                                                      P, Dbl, P, P]
             _lib = lib
     return _lib
 
@@ -366,6 +371,71 @@ def srswa_decode_fp8(q, pk8, pv8, kscale, vscale, prefix_len, blk_idx, blk_logp,
     _L().oracle_srswa_decode_fp8(B, H, D, n, cap, blk, _p(q), _p(pk8), _p(pv8), _p(kscale), _p(vscale),
                                  _p(prefix_len), _p(blk_idx), _p(blk_logp), topk, _p(ring_k), _p(ring_v), _p(wp),
                                  _p(fill), float(scale), _p(out), _p(lse))
+    return out, lse
+
+
+# ---------------------------------------------------------------- FP8 ring
+
+def fp8_ring(B: int, H: int, n: int, D: int = 128):
+    """An empty FP8 ring: codes (K, V) uint8 [B][H][n][D] and row scales (K, V) f32 [B][H][n]."""
+    return (np.zeros((B, H, n, D), np.uint8), np.zeros((B, H, n, D), np.uint8), np.ones((B, H, n), np.float32),
+            np.ones((B, H, n), np.float32))
+
+
+def append_fp8(rk8, rv8, rks, rvs, k_new, v_new, wp, fill):
+    """Ring append into an FP8 ring (each written row quantised with its own scale), in place on
+    the codes, scales, wp and fill. Returns slot_out [B]."""
+    for name, a in (("rk8", rk8), ("rv8", rv8), ("rks", rks), ("rvs", rvs), ("wp", wp), ("fill", fill)):
+        if not (isinstance(a, np.ndarray) and a.flags.c_contiguous):
+            raise ValueError(f"{name} must be a C-contiguous numpy array (updated in place)")
+    if rk8.dtype != np.uint8 or rks.dtype != np.float32 or wp.dtype != np.int32:
+        raise TypeError("codes uint8, scales float32, wp / fill int32")
+    B, H, n, D = rk8.shape
+    k_new, v_new = _u16(k_new, 3, "k_new"), _u16(v_new, 3, "v_new")
+    slot = np.zeros(B, np.int32)
+    _L().oracle_append_fp8(B, H, n, D, _p(rk8), _p(rv8), _p(rks), _p(rvs), _p(k_new), _p(v_new), _p(wp), _p(fill),
+                           _p(slot))
+    return slot
+
+
+def rswa_decode_fp8kv(q, pk8, pv8, kscale, vscale, prefix_len, rk8, rv8, rks, rvs, wp, fill, scale,
+                      blk: int = BLOCK):
+    """R-SWA decode over an E4M3 prefix (block scales) and an E4M3 ring (row scales).
+    Returns (out fp64 [B][H][D], lse fp64 [B][H])."""
+    q = _u16(q, 3, "q")
+    pk8, pv8, rk8, rv8 = _u8(pk8, 4, "pk8"), _u8(pv8, 4, "pv8"), _u8(rk8, 4, "rk8"), _u8(rv8, 4, "rv8")
+    kscale, vscale = np.ascontiguousarray(kscale, np.float32), np.ascontiguousarray(vscale, np.float32)
+    rks, rvs = np.ascontiguousarray(rks, np.float32), np.ascontiguousarray(rvs, np.float32)
+    prefix_len, wp, fill = _i32(prefix_len, "prefix_len"), _i32(wp, "wp"), _i32(fill, "fill")
+    B, H, D = q.shape
+    cap, n = pk8.shape[2], rk8.shape[2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _L().oracle_rswa_decode_fp8kv(B, H, D, n, cap, blk, _p(q), _p(pk8), _p(pv8), _p(kscale), _p(vscale),
+                                  _p(prefix_len), _p(rk8), _p(rv8), _p(rks), _p(rvs), _p(wp), _p(fill), float(scale),
+                                  _p(out), _p(lse))
+    return out, lse
+
+
+def srswa_decode_fp8kv(q, pk8, pv8, kscale, vscale, prefix_len, blk_idx, blk_logp, rk8, rv8, rks, rvs, wp, fill,
+                       scale, blk: int = BLOCK):
+    """SR-SWA gathered-block decode over an E4M3 prefix and an E4M3 ring.
+    Returns (out fp64 [B][H][D], lse fp64 [B][H])."""
+    q = _u16(q, 3, "q")
+    pk8, pv8, rk8, rv8 = _u8(pk8, 4, "pk8"), _u8(pv8, 4, "pv8"), _u8(rk8, 4, "rk8"), _u8(rv8, 4, "rv8")
+    kscale, vscale = np.ascontiguousarray(kscale, np.float32), np.ascontiguousarray(vscale, np.float32)
+    rks, rvs = np.ascontiguousarray(rks, np.float32), np.ascontiguousarray(rvs, np.float32)
+    prefix_len, wp, fill = _i32(prefix_len, "prefix_len"), _i32(wp, "wp"), _i32(fill, "fill")
+    blk_idx = _i32(blk_idx, "blk_idx")
+    blk_logp = np.ascontiguousarray(blk_logp, np.float64)
+    B, H, D = q.shape
+    topk = blk_idx.shape[1]
+    cap, n = pk8.shape[2], rk8.shape[2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _L().oracle_srswa_decode_fp8kv(B, H, D, n, cap, blk, _p(q), _p(pk8), _p(pv8), _p(kscale), _p(vscale),
+                                   _p(prefix_len), _p(blk_idx), _p(blk_logp), topk, _p(rk8), _p(rv8), _p(rks),
+                                   _p(rvs), _p(wp), _p(fill), float(scale), _p(out), _p(lse))
     return out, lse
 
 

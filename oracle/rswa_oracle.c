@@ -15,6 +15,7 @@
  *   [R-SWA summary]   "百度Unlimited OCR" paper summary, lshu.cn/news/33052
  *   [R-SWA tutorial]  "百度 Unlimited OCR 深度实战 ... R-SWA注意力革命", chenxutan.com/d/4055.html
  *   [SR-SWA explainer] Unlimited-OCR-2 SR-SWA explainer, nxmr.cn/news/162408
+ *   [tech analysis]   "Unlimited-OCR：突破32768上下文限制的视觉语言模型技术解析", pnsm.cn
  *
  * Layouts (row-major, all little-endian):
  *   bf16 tensors are passed as their raw 16-bit patterns (uint16_t).
@@ -540,9 +541,8 @@ void oracle_srswa_decode(int B, int H, int D, int n, int64_t cap, int blk, const
 /* ------------------------------------------------------------------ */
 
 /*
- * The pages list quantised KV-cache compression as the next step after the
- * window itself (Tutorial, "KV缓存压缩" under future directions) without fixing
- * a format. Reading adopted: the prefix K and V are stored as OCP FP8 E4M3
+ * The pages list quantised KV-cache compression among the memory measures
+ * ([tech analysis] 内存使用效率, "KV缓存压缩") without fixing a format. Reading adopted: the prefix K and V are stored as OCP FP8 E4M3
  * codes (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0
  * holds the subnormals m/8 * 2^-6; S.1111.111 is NaN; no infinities; largest
  * finite value 448), one fp32 scale per (sequence, head, 32-token block) for K
@@ -873,5 +873,126 @@ void oracle_rope_page2d(int64_t rows, int H, int D, const uint16_t* x, const int
         out[off + i + half] = hi * c + lo * s;
       }
     }
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 ring                                                            */
+/* ------------------------------------------------------------------ */
+
+/*
+ * One row quantised on its own: scale = the largest |x| over its D dims / 448
+ * in fp32 (1 when that is 0), code = E4M3(x / scale) with the quotient in fp32
+ * (the prefix quantiser's rule with a single row as the block).
+ */
+static void quantize_row(int D, const uint16_t* x, uint8_t* codes, float* scale) {
+  float amax = 0.0f;
+  for (int d = 0; d < D; ++d) {
+    float v = fabsf((float)bf16_to_double(x[d]));
+    if (v > amax) amax = v;
+  }
+  float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+  *scale = sc;
+  for (int d = 0; d < D; ++d) codes[d] = oracle_e4m3_encode((float)bf16_to_double(x[d]) / sc);
+}
+
+/*
+ * Ring append into an FP8 ring (KV-cache quantisation, [tech analysis]
+ * 内存使用效率, extended from the prefix to the ring; the format is this
+ * library's reading): the new token's K and V rows of every head are quantised
+ * one row at a time, since the ring is written one token at a time and a row is
+ * the unit that is complete when written. Codes [B][H][n][D], scales [B][H][n]
+ * for K and for V; wp / fill / slot_out advance as in oracle_append.
+ * Pinned by: slots, wp and fill equal oracle_append's; every written row equals
+ * the prefix quantiser (separately pinned) applied to that row as a one-row block.
+ */
+void oracle_append_fp8(int B, int H, int n, int D, uint8_t* rk8, uint8_t* rv8, float* rks, float* rvs,
+                       const uint16_t* k_new, const uint16_t* v_new, int32_t* wp, int32_t* fill,
+                       int32_t* slot_out) {
+  for (int b = 0; b < B; ++b) {
+    int32_t slot = wp[b];
+    for (int h = 0; h < H; ++h) {
+      int64_t row = ((int64_t)b * H + h) * n + slot;
+      int64_t src = ((int64_t)b * H + h) * D;
+      quantize_row(D, k_new + src, rk8 + row * D, rks + row);
+      quantize_row(D, v_new + src, rv8 + row * D, rvs + row);
+    }
+    wp[b] = (slot + 1 == n) ? 0 : slot + 1;
+    if (fill[b] < n) fill[b] = fill[b] + 1;
+    if (slot_out) slot_out[b] = slot;
+  }
+}
+
+/* The FP8 ring's valid slots (as push_ring), each row with its own scales. */
+static void push_ring8(keylist* L, const uint8_t* rk8, const uint8_t* rv8, const float* rks, const float* rvs,
+                       int64_t bh, int n, int D, int32_t wp, int32_t fill) {
+  for (int32_t i = 0; i < fill; ++i) {
+    int64_t row = bh * n + pos_mod((int64_t)wp - fill + i, n);
+    keylist_push8(L, rk8 + row * D, rv8 + row * D, rks[row], rvs[row], 0.0);
+  }
+}
+
+/*
+ * R-SWA decode over an FP8 prefix (block scales) and an FP8 ring (row scales):
+ * oracle_rswa_decode with every element read as code value * its scale.
+ * Pinned by: on data on the E4M3 grid whose every block and row holds a 448
+ * (unit scales) it equals oracle_rswa_decode of the same values exactly.
+ */
+void oracle_rswa_decode_fp8kv(int B, int H, int D, int n, int64_t cap, int blk, const uint16_t* q,
+                              const uint8_t* pk8, const uint8_t* pv8, const float* kscale, const float* vscale,
+                              const int32_t* prefix_len, const uint8_t* rk8, const uint8_t* rv8, const float* rks,
+                              const float* rvs, const int32_t* wp, const int32_t* fill, double scale, double* out,
+                              double* lse) {
+  int64_t BH = (int64_t)B * H, nb_cap = (cap + blk - 1) / blk;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, cap + n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+      int64_t b = bh / H;
+      L.count = 0;
+      for (int64_t j = 0; j < prefix_len[b]; ++j) {
+        int64_t off = (bh * cap + j) * D, sc = bh * nb_cap + j / blk;
+        keylist_push8(&L, pk8 + off, pv8 + off, kscale[sc], vscale[sc], 0.0);
+      }
+      push_ring8(&L, rk8, rv8, rks, rvs, bh, n, D, wp[b], fill[b]);
+      attend(&L, q + bh * D, D, scale, out + bh * D, lse + bh);
+    }
+    keylist_free(&L);
+  }
+}
+
+/* SR-SWA gathered decode over an FP8 prefix and an FP8 ring (same pins, against
+ * oracle_srswa_decode). */
+void oracle_srswa_decode_fp8kv(int B, int H, int D, int n, int64_t cap, int blk, const uint16_t* q,
+                               const uint8_t* pk8, const uint8_t* pv8, const float* kscale, const float* vscale,
+                               const int32_t* prefix_len, const int32_t* blk_idx, const double* blk_logp, int topk,
+                               const uint8_t* rk8, const uint8_t* rv8, const float* rks, const float* rvs,
+                               const int32_t* wp, const int32_t* fill, double scale, double* out, double* lse) {
+  int64_t BH = (int64_t)B * H, nb_cap = (cap + blk - 1) / blk;
+#pragma omp parallel
+  {
+    keylist L;
+    keylist_init(&L, (int64_t)topk * blk + n);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+      int64_t b = bh / H;
+      int64_t m = prefix_len[b];
+      L.count = 0;
+      for (int k = 0; k < topk; ++k) {
+        int64_t c = blk_idx[b * topk + k];
+        double bias = blk_logp[b * topk + k];
+        if (c < 0 || bias == -INFINITY) continue;
+        int64_t t1 = (c + 1) * blk < m ? (c + 1) * blk : m;
+        for (int64_t t = c * blk; t < t1; ++t) {
+          int64_t off = (bh * cap + t) * D, sc = bh * nb_cap + c;
+          keylist_push8(&L, pk8 + off, pv8 + off, kscale[sc], vscale[sc], bias);
+        }
+      }
+      push_ring8(&L, rk8, rv8, rks, rvs, bh, n, D, wp[b], fill[b]);
+      attend(&L, q + bh * D, D, scale, out + bh * D, lse + bh);
+    }
+    keylist_free(&L);
   }
 }

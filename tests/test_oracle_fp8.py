@@ -8,9 +8,10 @@
 - quantiser: per (sequence, head, 32-token block) scale = amax / 448 in fp32;
   the block's largest element lands on +-448; every element is within half a
   grid step of its dequantised value; rows past the prefix are zero codes.
-- FP8 decodes: data that already lie on the E4M3 grid with a 448 in every
-  block get unit scales, so the FP8 decode must equal the (pinned) bf16 decode
-  of the same values exactly, for R-SWA and for SR-SWA.
+- FP8 decodes: data on the E4M3 grid with a 448 in every block, each block then
+  times its own power of two (small enough that the softmax is not saturated),
+  get exactly that power of two as scale, so the FP8 decode must equal the
+  (pinned) bf16 decode of the same values exactly, for R-SWA and for SR-SWA.
 """
 import numpy as np
 import pytest
@@ -98,26 +99,39 @@ def test_quantize_prefix_properties(plen):
             assert (scales[b, h, (m + 31) // 32:] == 0).all()
 
 
+GRID_POW2 = (-10, -6)   # block / row factors 2^e: keeps q.k moderate, so the softmax is not saturated
+
+
 def _grid_prefix(B, H, cap, D, seed):
-    """bf16 prefix whose values are E4M3 values with a 448 in every 32-row block (unit scales)."""
+    """bf16 prefix on the E4M3 grid with a 448 in every 32-row block, each block then times its
+    own 2^e, e in GRID_POW2: every block scale is exactly 2^e and every element exactly its
+    code value times that scale. Returns (prefix, e [B][H][blocks])."""
     rng = np.random.default_rng(seed)
     t = _table()
     sign = (rng.integers(0, 2, (B, H, cap, D)) << 7).astype(np.uint8)
     codes = rng.integers(0, 0x7f, (B, H, cap, D)).astype(np.uint8) | sign   # finite codes only
     codes[:, :, ::32, 0] = 0x7e                                             # amax = 448 in every block
-    return torch.from_numpy(t[codes].astype(np.float32)).bfloat16()          # exact: E4M3 values fit bf16
+    e = rng.integers(GRID_POW2[0], GRID_POW2[1] + 1, (B, H, (cap + 31) // 32))
+    f = np.repeat(np.exp2(e), 32, axis=2)[:, :, :cap, None]
+    return torch.from_numpy((t[codes] * f).astype(np.float32)).bfloat16(), e   # exact: E4M3 x 2^e fits bf16
+
+
+def _check_grid_scales(scales, e, plen):
+    for b, m in enumerate(plen):
+        nb = (m + 31) // 32
+        np.testing.assert_array_equal(scales[b, :, :nb], np.exp2(e[b, :, :nb]).astype(np.float32))
 
 
 def test_rswa_decode_fp8_equals_bf16_on_grid_data():
     B, H, D, n, cap = 2, 2, 128, 8, 96
     c = synth.decode_case(B, H, D, [96, 70], cap, n, 1, seed=21, wp0=3, fill0=8)
-    pk = _grid_prefix(B, H, cap, D, 1)
-    pv = _grid_prefix(B, H, cap, D, 2)
+    pk, ek = _grid_prefix(B, H, cap, D, 1)
+    pv, ev = _grid_prefix(B, H, cap, D, 2)
     plen = c.prefix_len.numpy()
     k8, ks = oracle.quantize_prefix(synth.to_u16(pk), plen)
     v8, vs = oracle.quantize_prefix(synth.to_u16(pv), plen)
-    for b, m in enumerate(plen):
-        assert (ks[b, :, :(m + 31) // 32] == 1.0).all() and (vs[b, :, :(m + 31) // 32] == 1.0).all()
+    _check_grid_scales(ks, ek, plen)
+    _check_grid_scales(vs, ev, plen)
     args = (synth.to_u16(c.ring_k), synth.to_u16(c.ring_v), c.wp.numpy(), c.fill.numpy(), c.scale)
     ref, ref_lse = oracle.rswa_decode(synth.to_u16(c.q[0]), synth.to_u16(pk), synth.to_u16(pv), plen, *args)
     got, got_lse = oracle.rswa_decode_fp8(synth.to_u16(c.q[0]), k8, v8, ks, vs, plen, *args)
@@ -128,11 +142,13 @@ def test_rswa_decode_fp8_equals_bf16_on_grid_data():
 def test_srswa_decode_fp8_equals_bf16_on_grid_data():
     B, H, D, n, cap = 2, 2, 128, 8, 160
     c = synth.decode_case(B, H, D, [160, 100], cap, n, 1, seed=22, wp0=5, fill0=8)
-    pk = _grid_prefix(B, H, cap, D, 3)
-    pv = _grid_prefix(B, H, cap, D, 4)
+    pk, ek = _grid_prefix(B, H, cap, D, 3)
+    pv, ev = _grid_prefix(B, H, cap, D, 4)
     plen = c.prefix_len.numpy()
     k8, ks = oracle.quantize_prefix(synth.to_u16(pk), plen)
     v8, vs = oracle.quantize_prefix(synth.to_u16(pv), plen)
+    _check_grid_scales(ks, ek, plen)
+    _check_grid_scales(vs, ev, plen)
     blk = np.array([[4, 0, 2, -1], [3, 1, 0, 2]], np.int32)
     logp = np.log(np.array([[0.5, 0.3, 0.2, 1.0], [0.4, 0.3, 0.2, 0.1]]))
     args = (synth.to_u16(c.ring_k), synth.to_u16(c.ring_v), c.wp.numpy(), c.fill.numpy(), c.scale)
