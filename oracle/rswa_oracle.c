@@ -542,7 +542,8 @@ void oracle_srswa_decode(int B, int H, int D, int n, int64_t cap, int blk, const
 
 /*
  * The pages list quantised KV-cache compression among the memory measures
- * ([tech analysis] 内存使用效率, "KV缓存压缩") without fixing a format. Reading adopted: the prefix K and V are stored as OCP FP8 E4M3
+ * ([tech analysis] 内存使用效率, "KV缓存压缩") without fixing a format.
+ * Reading adopted: the prefix K and V are stored as OCP FP8 E4M3
  * codes (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0
  * holds the subnormals m/8 * 2^-6; S.1111.111 is NaN; no infinities; largest
  * finite value 448), one fp32 scale per (sequence, head, 32-token block) for K
