@@ -5,7 +5,8 @@
 
 A step is one decode step of the whole batch through the C ABI:
   configs 1, 2 (R-SWA):   rswa_decode_append (ring append fused into the decode)
-  configs 4, 5 (SR-SWA):  rswa_append + srswa_route + srswa_decode
+  configs 4, 5 (SR-SWA):  srswa_step (ring append, router and gathered attention in
+                          one launch; --unfused: rswa_append + srswa_route + srswa_decode)
   configs 6, 7:           configs 2 and 4 over an FP8 (E4M3) prefix, quantised
                           once before timing: rswa_append + rswa_decode_fp8
                           (+ srswa_route + srswa_decode_fp8)
@@ -13,6 +14,8 @@ A step is one decode step of the whole batch through the C ABI:
   config 9 (page2d rotary encoding of a prefill chunk's q and k): rswa_rope_page2d
   config 10:              config 4 with the page2d encoding: rswa_append_rope +
                           srswa_route + srswa_decode
+  configs 11, 12:         configs 6 and 7 with an FP8 ring as well: rswa_append_fp8 +
+                          rswa_decode_fp8kv (+ srswa_route + srswa_decode_fp8kv)
 (the router's block index keys are pooled once per prefix, before timing).
 The default workload is the batched R-SWA decode: 512 sequences, 16 heads,
 head_dim 128, a 10-page prefix (2560 visual + 32 prompt tokens) and a full
@@ -44,6 +47,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +57,10 @@ if ROOT not in sys.path:
 METRIC = "decode attn steps/s & achieved HBM GB/s (fraction of peak) on 1 B200"
 FALLBACK_HBM_GBS = 6650.0
 EVENT_EVERY = 8  # kernel durations are bracketed with CUDA events in every 8th timed step
+TIMING_NOTE = (f"K steps in one CUDA graph replay timed by CUDA events (ms_per_step); kernel durations from event "
+               f"brackets around the kernels of every {EVENT_EVERY}th step (avg_launch_us): an event node between "
+               "two kernels also ends programmatic dependent launch there, so a bracket includes the launch gap "
+               "that the un-bracketed steps hide, and a one-kernel step's bracket can exceed ms_per_step")
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -98,6 +106,11 @@ def workload(cfg: int) -> dict:
         w["rope"] = True
         w["name"] += "; page2d rotary encoding of q and the new key fused into the ring append (rswa_append_rope)"
         return w
+    if cfg in (11, 12):  # configs 6 and 7 with the ring in FP8 too (row scales)
+        w = workload(6 if cfg == 11 else 7)
+        w["fp8_ring"] = True
+        w["name"] += "; ring K/V stored as E4M3 codes with one f32 scale per row"
+        return w
     if cfg in (6, 7):  # the batched R-SWA and the 32K-history SR-SWA workloads over an FP8 (E4M3) prefix
         w = workload(2 if cfg == 6 else 4)
         w["fp8"] = True
@@ -141,14 +154,15 @@ def algorithmic_bytes(w: dict, blk_rows=None) -> dict:
     """
     H, n = w["H"], w["n"]
     per_q = 256 + 512 + 4
+    ring_row = 264 if w.get("fp8_ring") else 512  # FP8 ring: 128 + 128 B of codes + two 4-byte row scales
     # an FP8 prefix row is 128 + 128 B of codes, plus 8 B of scales per 32-row block
     row = 256 if w.get("fp8") else 512
     if w["kind"] == "rswa":
-        attn = sum(m * row + (8 * ((m + 31) // 32) if w.get("fp8") else 0) + n * 512 + per_q
+        attn = sum(m * row + (8 * ((m + 31) // 32) if w.get("fp8") else 0) + n * ring_row + per_q
                    for m in w["plen"]) * H
         return dict(attn=attn, route=0)
     rows = blk_rows if blk_rows is not None else [16 * 32] * w["B"]
-    attn = sum(r * row + (8 * ((r + 31) // 32) if w.get("fp8") else 0) + n * 512 + per_q for r in rows) * H
+    attn = sum(r * row + (8 * ((r + 31) // 32) if w.get("fp8") else 0) + n * ring_row + per_q for r in rows) * H
     route = sum(((m + 31) // 32) * 128 + 128 + 16 * 8 for m in w["plen"])
     return dict(attn=attn, route=route)
 
@@ -181,12 +195,12 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+        self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
+            fd, self.path = tempfile.mkstemp(prefix="rswa_clocks_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
                                          stderr=subprocess.DEVNULL)
@@ -248,6 +262,10 @@ def kernel_source_hash(kind: str) -> str:
     h = hashlib.sha256()
     for f in files:
         src = open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", f), encoding="utf-8").read()
+        if f == "internal.h":  # only the argument and workspace structs the decode kernel is built from
+            a = src.index("struct DecodeArgs")
+            b = src.index("};", src.index("struct WorkspacePlan")) + 2
+            src = src[a:b]
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
         h.update("\n".join(line.rstrip() for line in src.splitlines() if line.strip()).encode())
@@ -316,10 +334,22 @@ class Problem:
         self.lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
         self.sparse = w["kind"] == "srswa"
         self.fp8 = bool(w.get("fp8"))
+        # SR-SWA over a bf16 prefix and ring: the whole step (append + router + attention) in one
+        # launch (srswa_step), unless unfused is asked for
+        self.fused_route = self.sparse and not self.fp8 and not w.get("rope") and not w.get("fp8_ring") and \
+            not w.get("unfused")
         if self.fp8:  # the stored cache: the bf16 prefix quantised once, by the library
             self.k8, self.v8, self.ks, self.vs = rswa.fp8_prefix_buffers(self.c.pk)
             rswa.rswa_quantize_prefix(self.c.pk, self.c.pv, self.c.prefix_len, self.k8, self.v8, self.ks, self.vs,
                                       status=self.ws)
+        self.fp8_ring = bool(w.get("fp8_ring"))
+        if self.fp8_ring:  # a full FP8 ring: n appends of random rows before timing
+            self.ring8 = rswa.fp8_ring_buffers(self.c.ring_k.shape)
+            g = synth._gen(seed + 3, "cuda")
+            for _ in range(n):
+                kk = synth.randn_bf16((B, H, D), g, "cuda")
+                vv = synth.randn_bf16((B, H, D), g, "cuda")
+                rswa.rswa_append_fp8(*self.ring8, kk, vv, self.c.wp, self.c.fill, status=self.ws)
         self.rope = bool(w.get("rope"))
         if self.rope:  # this step's token positions ([steps][B]) and the encoded query
             tok, page = synth.page_positions(B, steps_total, seed=seed + 2)
@@ -337,7 +367,8 @@ class Problem:
             self.blk = torch.empty((B, 16), dtype=torch.int32, device="cuda")
             self.logp = torch.empty((B, 16), dtype=torch.float32, device="cuda")
             self.ws_route = rswa.new_workspace(self.dims, rswa.OP_ROUTE)
-            self.ws = rswa.new_workspace(self.dims, rswa.OP_SRSWA_DECODE)
+            self.ws = rswa.new_workspace(self.dims, rswa.OP_SRSWA_ROUTED if self.fused_route else
+                                         rswa.OP_SRSWA_DECODE)
             del pl
         torch.cuda.synchronize()
 
@@ -347,6 +378,14 @@ class Problem:
         q = c.q[i] if q is None else q
         k_new = c.k_new[i] if k_new is None else k_new
         v_new = c.v_new[i] if v_new is None else v_new
+        if self.fused_route:
+            if ev is not None:
+                ev[0].record()
+            r.srswa_step(q, k_new, v_new, self.q_idx[i % self.n_dirs], self.kbar, c.pk, c.pv, c.prefix_len, c.ring_k,
+                         c.ring_v, c.wp, c.fill, self.blk, self.logp, self.out, self.ws, lse=self.lse, scale=c.scale)
+            if ev is not None:
+                ev[1].record()
+            return 1
         if not self.fp8 and not self.sparse:
             # R-SWA over a bf16 prefix: the fused step (ring append inside the decode launch),
             # measured faster there; the SR-SWA steps keep append + route + decode
@@ -357,6 +396,26 @@ class Problem:
             if ev is not None:
                 ev[1].record()
             return 1
+        if self.fp8_ring:
+            r.rswa_append_fp8(*self.ring8, k_new, v_new, c.wp, c.fill, status=self.ws)
+            if self.sparse:
+                if ev is not None:
+                    ev[2].record()
+                r.srswa_route(self.q_idx[i % self.n_dirs], self.kbar, c.prefix_len, self.blk, self.logp,
+                              self.ws_route, prefix_cap=self.w["cap"])
+                if ev is not None:
+                    ev[3].record()
+            if ev is not None:
+                ev[0].record()
+            if self.sparse:
+                r.srswa_decode_fp8kv(q, self.k8, self.v8, self.ks, self.vs, c.prefix_len, self.blk, self.logp,
+                                     *self.ring8, c.wp, c.fill, self.out, self.ws, lse=self.lse, scale=c.scale)
+            else:
+                r.rswa_decode_fp8kv(q, self.k8, self.v8, self.ks, self.vs, c.prefix_len, *self.ring8, c.wp, c.fill,
+                                    self.out, self.ws, lse=self.lse, scale=c.scale)
+            if ev is not None:
+                ev[1].record()
+            return 3 if self.sparse else 2
         if self.rope:
             if ev is not None:
                 ev[4].record()
@@ -531,7 +590,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     clk = clocks.stop(t_wall0, t_wall1)
     ms_total = start.elapsed_time(end)
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    route_ms = [e[2].elapsed_time(e[3]) for e in evs] if prob.sparse else []
+    route_ms = [e[2].elapsed_time(e[3]) for e in evs] if prob.sparse and not prob.fused_route else []
     rope_ms = [e[4].elapsed_time(e[5]) for e in evs] if prob.rope else []
     ms_max = max_over_ranks(world, ms_total)
     del graph
@@ -546,12 +605,15 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
             m = w["plen"][b]
             blk_rows.append(sum(min(32, m - 32 * c) for c, l in zip(blk[b], lp[b]) if c >= 0 and l > -math.inf))
     nbytes = algorithmic_bytes(w, blk_rows)
-    if not prob.fp8 and not prob.sparse:  # the fused step also writes this step's K and V row into the ring
+    if not prob.fp8 and (not prob.sparse or prob.fused_route):
+        # the fused step also writes this step's K and V row into the ring
         nbytes["attn"] += w["B"] * w["H"] * 512
+    if prob.fused_route:  # one kernel moves the router's bytes too
+        nbytes = dict(attn=nbytes["attn"] + nbytes["route"], route=0)
     attn_avg_s = statistics.mean(attn_ms) / 1e3
     achieved = nbytes["attn"] / attn_avg_s / 1e9
     peak, peak_src = measured_peak()
-    key = f"{'srswa' if prob.sparse else 'rswa'}_decode_config{args.config}"
+    key = f"{'srswa_step' if prob.fused_route else ('srswa' if prob.sparse else 'rswa')}_decode_config{args.config}"
     traffic = committed_traffic(key, kernel_source_hash("sparse" if prob.sparse else "dense"))
 
     # ---- e2e through the public API: pinned host inputs -> device -> append/decode -> host result ----
@@ -571,21 +633,21 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
-        "storage_dtype": "e4m3 prefix (f32 block scales) + bf16 ring" if prob.fp8 else "bf16",
+        "storage_dtype": ("e4m3 prefix (f32 block scales) + " + ("e4m3 ring (f32 row scales)" if prob.fp8_ring
+                                                                  else "bf16 ring")) if prob.fp8 else "bf16",
         "data": "synthetic",
         "impl": "ours",
-        "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "global_batch": B * world,
-                   "heads": H, "head_dim": D, "ring": w["n"],
-                   "prefix_tokens_mean": statistics.mean(w["plen"]), "parallelism": f"replicas x{world}",
-                   "l2": l2_note(w, nbytes),
-                   "timing": "K steps in one CUDA graph replay, CUDA events; kernel durations from "
-                             f"event brackets in every {EVENT_EVERY}th step"},
+        "config": config_of(w, args, world),
+        "timing": TIMING_NOTE,
         "qtok_per_s": steps_per_s * B * H,
         "seq_tok_per_s": steps_per_s * B,
         "hbm_gbs_step": world * K * (nbytes["attn"] + nbytes["route"]) / (ms_max / 1e3) / 1e9,
         "bytes_per_step": {"attn": nbytes["attn"], "route": nbytes["route"]},
-        "roofline": {"bound": "hbm", "kernel": ("srswa decode_kernel<true" if prob.sparse else "rswa decode_kernel<false")
-                     + (", fp8>" if prob.fp8 else (", bf16>" if prob.sparse else ", bf16> with the fused ring append")),
+        "roofline": {"bound": "hbm", "kernel": ("srswa step kernel: decode_kernel<true, bf16> with the ring append and "
+                                                "the router fused" if prob.fused_route else
+                                                ("srswa decode_kernel<true" if prob.sparse else "rswa decode_kernel<false")
+                                                + (", fp8>" if prob.fp8 else (", bf16>" if prob.sparse else
+                                                                              ", bf16> with the fused ring append"))),
                      "achieved": achieved,
                      "peak": peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
@@ -658,10 +720,8 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
         "metric": METRIC, "value": value, "unit": "prefill chunks/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if sparse else "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
-        "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "heads": H,
-                   "head_dim": w["D"], "ring": w["n"], "chunk": T, "prefix_tokens_mean": statistics.mean(w["plen"]),
-                   "parallelism": f"replicas x{world}", "timing": "K launches in one CUDA graph replay, CUDA events; kernel durations from "
-                             f"event brackets in every {EVENT_EVERY}th step"},
+        "config": config_of(w, args, world),
+        "timing": TIMING_NOTE,
         "qtok_per_s": value * B * H * T,
         "roofline": ({"bound": "alu", "kernel": "srswa decode_kernel<true, bf16> (chunked-prefill queries)",
                       "achieved": achieved, "peak": peak,
@@ -766,12 +826,8 @@ def run_rope(args, w: dict, world: int, rank: int, local: int) -> dict:
         "metric": METRIC, "value": value, "unit": "encoded chunks/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
-        "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "heads": H,
-                   "head_dim": w["D"], "chunk": T, "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: each step streams {nbytes / 1e9:.2f} GB through L2 ({nbytes / 2e9:.2f} GB read, "
-                         "as much written), twice its 126 MB, in the same order every step",
-                   "timing": "K launches in one CUDA graph replay, CUDA events; kernel durations from "
-                             f"event brackets in every {EVENT_EVERY}th step"},
+        "config": config_of(w, args, world),
+        "timing": TIMING_NOTE,
         "tok_per_s": value * B * T,
         "roofline": {"bound": "hbm", "kernel": "rope_kernel (page2d, q and k)", "achieved": achieved, "peak": peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
@@ -904,10 +960,18 @@ def oracle_sample_step(w: dict, sample: int, seed: int):
     st = dict(q=u(c.q[0]), k=u(c.k_new[0]), v=u(c.v_new[0]), pk=u(c.pk), pv=u(c.pv), plen=c.prefix_len.numpy(),
               rk=u(c.ring_k).copy(), rv=u(c.ring_v).copy(), wp=c.wp.numpy().copy(), fill=c.fill.numpy().copy(),
               scale=c.scale)
+    import oracle
     if w.get("fp8"):
-        import oracle
         st["k8"], st["ks"] = oracle.quantize_prefix(st["pk"], st["plen"])
         st["v8"], st["vs"] = oracle.quantize_prefix(st["pv"], st["plen"])
+    if w.get("fp8_ring"):  # a full FP8 ring: n appends of random rows
+        import numpy as np
+        st["ring8"] = list(oracle.fp8_ring(sample, w["H"], w["n"], w["D"]))
+        rng = np.random.default_rng(seed + 3)
+        for _ in range(w["n"]):
+            kk = oracle.bf16_round(rng.standard_normal((sample, w["H"], w["D"])))
+            vv = oracle.bf16_round(rng.standard_normal((sample, w["H"], w["D"])))
+            oracle.append_fp8(*st["ring8"], kk, vv, st["wp"], st["fill"])
     if w.get("rope"):
         tok, page = synth.page_positions(sample, 1, seed=seed + 2)
         st["tok"], st["page"] = tok[:, 0].numpy().copy(), page[:, 0].numpy().copy()
@@ -925,6 +989,17 @@ def oracle_step(st: dict, w: dict):
         k = oracle.bf16_round(oracle.rope_page2d(st["k"], st["tok"], st["page"]))
     else:
         k = st["k"]
+    if w.get("fp8_ring"):
+        oracle.append_fp8(*st["ring8"], k, st["v"], st["wp"], st["fill"])
+        if w["kind"] == "rswa":
+            return oracle.rswa_decode_fp8kv(st["q"], st["k8"], st["v8"], st["ks"], st["vs"], st["plen"], *st["ring8"],
+                                            st["wp"], st["fill"], st["scale"])
+        kbar = st.get("kbar")
+        if kbar is None:
+            kbar = st["kbar"] = oracle.index_pool(st["k_idx"], st["plen"])
+        r = oracle.route(st["q_idx"], kbar, st["plen"])
+        return oracle.srswa_decode_fp8kv(st["q"], st["k8"], st["v8"], st["ks"], st["vs"], st["plen"], r["blk_idx"],
+                                         r["blk_logp"], *st["ring8"], st["wp"], st["fill"], st["scale"])
     oracle.append(st["rk"], st["rv"], k, st["v"], st["wp"], st["fill"])
     if w["kind"] == "rswa":
         if w.get("fp8"):
@@ -1067,80 +1142,85 @@ def _cpu_baseline_case(w: dict, budget_s: float):
         f"{sample} of {w['B']} sequences per step (all heads)", 2, 50
 
 
+def config_of(w: dict, args, world: int) -> dict:
+    """The `config` object of a workload, the same for both arms."""
+    B = w["B"]
+    c = {"workload": w["name"], "config_index": args.config, "batch_per_gpu": B, "global_batch": B * world,
+         "heads": w["H"], "head_dim": w["D"], "ring": w["n"], "parallelism": f"replicas x{world}"}
+    if w["kind"] == "rope":
+        nbytes = rope_bytes(w)
+        c.pop("ring")
+        c["chunk"] = w["T"]
+        c["l2"] = (f"no flush: each step streams {nbytes / 1e9:.2f} GB through L2 ({nbytes / 2e9:.2f} GB read, "
+                   "as much written), twice its 126 MB, in the same order every step")
+    elif w["kind"] in ("prefill", "srswa_prefill"):
+        c["chunk"] = w["T"]
+        c["prefix_tokens_mean"] = statistics.mean(w["plen"])
+        c["l2"] = "no flush: the prefix K/V of the chunk exceed L2; each step recomputes the same chunk"
+    else:
+        c["prefix_tokens_mean"] = statistics.mean(w["plen"])
+        c["l2"] = l2_note(w, algorithmic_bytes(w))
+    return c
+
+
 def run_reference(args, w: dict) -> dict:
-    """The oracle as the reference arm, on the host cores, K timed steps of a bounded sample."""
+    """The oracle as the reference arm, on the host cores, K timed steps of a bounded sample.
+
+    Each step runs the oracle on a sample of the workload; `value` is extrapolated to the
+    whole workload by the sample fraction, while `ms_per_step` is the measured time of one
+    sampled step (so steps x ms_per_step is the timed region's real length)."""
     import oracle
     if w["kind"] == "rope":
         st, frac = oracle_rope_case(w, seed=99)
-        for _ in range(args.warmup):
-            oracle_rope_step(st)
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
-            oracle_rope_step(st)
-        value = frac / ((time.perf_counter() - t0) / args.steps)
-        cb = {"value": value, "unit": "encoded chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
-              "sample": f"{ROPE_ORACLE_TOKENS} of {w['B'] * w['T']} tokens per step (all heads, q and k); chunks/s "
-                        f"extrapolated by the sample fraction; fp64 C oracle on the host cores"}
-        return {"metric": METRIC, "value": value, "unit": "encoded chunks/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": w["B"]},
-                "cpu_baseline": cb,
-                "e2e": {"value": value, "unit": "encoded chunks/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-    if w["kind"] in ("prefill", "srswa_prefill"):
+        step = lambda: oracle_rope_step(st)  # noqa: E731
+        unit = "encoded chunks/s"
+        what = f"{ROPE_ORACLE_TOKENS} of {w['B'] * w['T']} tokens per step (all heads, q and k)"
+    elif w["kind"] in ("prefill", "srswa_prefill"):
         st, frac = oracle_prefill_case(w, 1, seed=99)
-        for _ in range(args.warmup):
-            oracle_prefill_step(st, w)
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
-            oracle_prefill_step(st, w)
-        value = frac / ((time.perf_counter() - t0) / args.steps)
-        cb = {"value": value, "unit": "prefill chunks/s", "cores": oracle.get_threads(), "kind": "oracle",
-              "sample": f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows per step (all heads); "
-                        f"chunks/s extrapolated by the sample fraction; fp64 C oracle on the host cores"}
-        return {"metric": METRIC, "value": value, "unit": "prefill chunks/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": w["B"]},
-                "cpu_baseline": cb,
-                "e2e": {"value": value, "unit": "prefill chunks/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-    sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2, 10: 2}.get(args.config, 1))
-    st = oracle_sample_step(w, sample, seed=99)
+        step = lambda: oracle_prefill_step(st, w)  # noqa: E731
+        unit = "prefill chunks/s"
+        what = f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows per step (all heads)"
+    else:
+        sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2, 10: 2, 11: 8, 12: 2}.get(args.config, 1))
+        st = oracle_sample_step(w, sample, seed=99)
+        step = lambda: oracle_step(st, w)  # noqa: E731
+        frac = sample / w["B"]
+        unit = "steps/s"
+        what = f"{sample} of {w['B']} sequences per step (all heads)"
     for _ in range(args.warmup):
-        oracle_step(st, w)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(st, w)
+        step()
     dt = (time.perf_counter() - t0) / args.steps
-    value = (sample / w["B"]) / dt
-    cb = {"value": value, "unit": "steps/s", "cores": oracle.get_threads(), "kind": "oracle",
-          "sample": f"{sample} of {w['B']} sequences per step (all heads); steps/s extrapolated by the sample "
-                    f"fraction; fp64 C oracle on the host cores"}
-    return {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w["name"], "config_index": args.config, "batch_per_gpu": w["B"]},
-            "cpu_baseline": cb,
-            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    value = frac / dt
+    cb = {"value": value, "unit": unit, "cores": oracle.get_threads(), "kind": "oracle",
+          "sample": f"{what}; {unit} extrapolated by the sample fraction ({frac:.4g}); fp64 C oracle on the host "
+                    f"cores"}
+    return {"metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "ms_per_full_step_extrapolated": 1e3 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": config_of(w, args, 1), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 SWEEP_LENGTHS = (8192, 16384, 32768, 65536, 102400)
 
 
-def run_length_sweep(args, world: int, rank: int, local: int) -> dict:
+def run_length_sweep(args, world: int, rank: int, local: int, lengths=SWEEP_LENGTHS) -> dict:
     """The SR-SWA step at uniform history lengths (16 sequences, top-16 + 128-slot ring).
 
     The attention reads the same 640 rows per (sequence, head) at every length; only the
     router's block-key scan (128 B per 32-token block) grows with the history."""
     import torch
     rows = []
-    for m in SWEEP_LENGTHS:
+    for m in lengths:
         w = workload(5)
         w["plen"] = [m] * w["B"]
         w["cap"] = m
         w["name"] = f"SR-SWA decode, 16 sequences, 16 heads, head_dim 128, uniform history {m} tokens"
+        if getattr(args, "unfused", False):
+            w["unfused"] = True
         r = run_ours(args, w, world, rank, local)
         rows.append({"history": m, "ms_per_step": r["ms_per_step"], "steps_per_s": r["value"],
                      "kernels_us": r["kernels_us"], "attn_hbm_frac": r["roofline"]["frac"],
@@ -1154,6 +1234,47 @@ def run_length_sweep(args, world: int, rank: int, local: int) -> dict:
             "impl": "ours", "sweep": rows, "max_over_min": max(steps) / min(steps)}
 
 
+EXTRA_CONFIGS = (1, 3, 4, 5)
+EXTRA_SWEEP = (8192, 102400)
+
+
+def summary(r: dict) -> dict:
+    """The figures of one workload's run kept in the default line's `configs` object."""
+    rf = r["roofline"]
+    keep = ("bound", "kernel", "achieved", "peak", "peak_source", "unit", "frac", "traffic",
+            "algorithmic_bytes_per_launch", "algorithmic_flops_per_launch", "avg_launch_us")
+    return {"workload": r["config"]["workload"], "value": r["value"], "unit": r["unit"],
+            "ms_per_step": r["ms_per_step"], "steps": r["steps"], "warmup": r["warmup"],
+            **({"qtok_per_s": r["qtok_per_s"]} if "qtok_per_s" in r else {}),
+            **({"hbm_gbs_step": r["hbm_gbs_step"]} if "hbm_gbs_step" in r else {}),
+            "kernels_us": r["kernels_us"], "gpu_launches": r["gpu_launches"],
+            "roofline": {k: rf[k] for k in keep if k in rf}, "clocks": r["clocks"], "l2": r["config"].get("l2")}
+
+
+def run_extra_configs(args, world: int, rank: int, local: int) -> dict:
+    """Configs 1, 3, 4 and 5 and the two ends of the SR-SWA length sweep, each with its own
+    K timed steps, kernel brackets, roofline and clocks (no e2e or CPU legs)."""
+    import copy
+
+    import torch
+    out = {}
+    for cfg in EXTRA_CONFIGS:
+        a = copy.copy(args)
+        a.config = cfg
+        a.no_e2e = True
+        out[str(cfg)] = summary(run_ours(a, workload(cfg), world, rank, local))
+        torch.cuda.empty_cache()
+    a = copy.copy(args)
+    a.config = 5
+    a.no_e2e = True
+    sw = run_length_sweep(a, world, rank, local, EXTRA_SWEEP)
+    out["length_sweep"] = {"what": sw["metric"] + " (16 sequences, uniform histories)", "unit": sw["unit"],
+                           "points": [{"history": x["history"], "ms_per_step": x["ms_per_step"],
+                                       "kernels_us": x["kernels_us"], "clocks": x["clocks"]} for x in sw["sweep"]],
+                           "max_over_min": sw["max_over_min"]}
+    return out
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -1161,7 +1282,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8, 9, 10])
+    ap.add_argument("--config", type=int, default=None, choices=list(range(1, 13)),
+                    help="the workload (default 2, which also runs configs 1, 3, 4, 5 into `configs`)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
@@ -1169,18 +1291,28 @@ def main():
                     help="override the workload's batch (a smaller case, e.g. for an ncu capture)")
     ap.add_argument("--prefix", type=int, default=None,
                     help="override every sequence's prefix length (and the capacity) of the workload")
+    ap.add_argument("--unfused", action="store_true",
+                    help="SR-SWA workloads: append + srswa_route + srswa_decode (three launches) instead of srswa_step")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="with the default workload, skip the other configs' lines in `configs`")
     ap.add_argument("--length-sweep", action="store_true",
                     help="SR-SWA latency against history length: 16 sequences at uniform lengths "
                          f"{SWEEP_LENGTHS}, one JSON line with every length's step and kernel times")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    extras = args.config is None and not args.no_extra_configs and args.batch is None and args.prefix is None
+    if args.config is None:
+        args.config = 2
     w = workload(args.config)
     if args.batch is not None:
         reps = (args.batch + len(w["plen"]) - 1) // len(w["plen"])
         w["plen"] = (w["plen"] * reps)[:args.batch]
         w["name"] = w["name"].replace(f"{w['B']} sequences", f"{args.batch} sequences")
         w["B"] = args.batch
+    if args.unfused:
+        w["unfused"] = True
+        w["name"] += " [append, router and attention as three launches]"
     if args.prefix is not None:
         w["plen"] = [args.prefix] * w["B"]
         w["cap"] = args.prefix
@@ -1203,6 +1335,10 @@ def main():
         res = run_ours(args, w, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w)
+        if extras and world == 1:
+            import torch
+            torch.cuda.empty_cache()
+            res["configs"] = run_extra_configs(args, world, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

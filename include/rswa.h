@@ -81,13 +81,16 @@ typedef struct {
                                    (any topk in 1..32)                                      */
 #define RSWA_OP_ROUTE 3         /* srswa_route, srswa_route_tokens (256 bytes)               */
 #define RSWA_OP_PREFILL 4       /* rswa_prefill, srswa_prefill (256 bytes)                   */
+#define RSWA_OP_SRSWA_ROUTED 5  /* srswa_decode_routed, srswa_step (any topk in 1..32)       */
 
 /* Message of the last failed call on this host thread ("" if none). */
 RSWA_API const char* rswa_last_error(void);
 
 /* Library ABI version (incremented when entry points are added or changed): 2 adds the
  * FP8 prefix, the fused decode step and the SR-SWA chunked prefill to version 1; 3 adds
- * the page2d rotary encoding (rswa_rope_page2d, rswa_append_rope). */
+ * the page2d rotary encoding (rswa_rope_page2d, rswa_append_rope); 4 the FP8 ring
+ * (rswa_append_fp8, rswa_decode_fp8kv, srswa_decode_fp8kv), the fused router
+ * (srswa_decode_routed, srswa_step) and the wait-timeout test hook. */
 RSWA_API int32_t rswa_version(void);
 
 /*
@@ -104,9 +107,28 @@ RSWA_API size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op);
  * Synchronises `stream`, reads the workspace's device status word into
  * *device_status (may be NULL) and clears it. Returns RSWA_OK if it was zero,
  * RSWA_ERR_DEVICE_CHECK otherwise, RSWA_ERR_CUDA if the copy failed.
+ * If RSWA_DEVICE_WAIT_TIMEOUT is set, CTAs that gave up may have left completion
+ * counters behind, so all ws_bytes of the workspace are zero-filled again (its
+ * initial state) and it can be reused; otherwise only the status word is cleared.
  * Also accepts the `status` pointer given to rswa_append (ws_bytes >= 4).
  */
 RSWA_API rswa_status rswa_check_status(void* workspace, size_t ws_bytes, int32_t* device_status, void* stream);
+
+/*
+ * Test hook for the bounded-wait path (failure detection without a GPU fault; the
+ * pages have no counterpart). Every pipeline wait of the decode kernels gives up after
+ * a time limit (2 s by default), sets RSWA_DEVICE_WAIT_TIMEOUT, lets its CTA's copies
+ * in flight land (bounded by the same limit) and ends the CTA, so the call returns and
+ * the CUDA context stays usable. This call arms, for the NEXT decode-family call made
+ * by the calling host thread only (rswa_decode*, srswa_decode*, srswa_prefill,
+ * rswa_decode_noalloc; consumed by that call even if it fails validation):
+ *   drop_tile     : >= 0: CTA 0 neither arms nor fills the shared-memory stage of its
+ *                   CTA-local tile number drop_tile, so that tile's bounded wait runs
+ *                   out (no copy is in flight for it); -1: nothing dropped.
+ *   wait_limit_ns : the wait limit for that call, in [1e3, 1e10] ns.
+ * Returns RSWA_ERR_INVALID for values out of range. Not for production use.
+ */
+RSWA_API rswa_status rswa_test_arm_wait_timeout(int32_t drop_tile, int64_t wait_limit_ns);
 
 /*
  * Ring append (one generated token per sequence).
@@ -284,6 +306,45 @@ RSWA_API rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, c
                                          float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * SR-SWA decode with the router fused into the gathered-block attention: srswa_route
+ * followed by srswa_decode in ONE launch (SR-SWA explainer, 稀疏路由 steps 2-4 and
+ * "三者合起来": the router picks the remote blocks that the attention then reads).
+ * Same route as srswa_route (blk_idx, blk_logp, tau as there; probs is not produced) and
+ * the same attention output as srswa_decode over that route. Inside the launch every
+ * warp first scores slices of 64 blocks (z = idx_scale <q_idx, kbar_c>) and publishes
+ * each slice sorted; one CTA per sequence then merges the slices' candidates, solves the
+ * exact 1.5-entmax threshold and publishes the top-k; meanwhile the attention warps
+ * stream the ring (which needs no route) and wait, bounded, for their sequence's route
+ * before they read the routed blocks. The CTAs of the launch wait on one another, so the
+ * grid is sized to one resident wave of the kernel: do not run two of these launches
+ * concurrently on one GPU (their waits would run out: RSWA_DEVICE_WAIT_TIMEOUT).
+ * Arguments: srswa_decode's, with q_idx f32 [B][32], kbar f32 [B][ceil(prefix_cap/32)][32]
+ * (srswa_index_pool), idx_scale, and blk_idx int32 [B][topk], blk_logp f32 [B][topk],
+ * tau f32 [B] or NULL as OUTPUTS. workspace: rswa_workspace_bytes(dims,
+ * RSWA_OP_SRSWA_ROUTED) bytes, zero-initialised; each launch leaves its counters at zero.
+ * Unsupported: ceil(prefix_cap / 32) > 8192.
+ */
+RSWA_API rswa_status srswa_decode_routed(const rswa_dims* dims, const void* q, const float* q_idx, const float* kbar,
+                                         float idx_scale, int32_t topk, const void* pk, const void* pv,
+                                         const int32_t* prefix_len, const void* ring_k, const void* ring_v,
+                                         const int32_t* wp, const int32_t* fill, float scale, int32_t* blk_idx,
+                                         float* blk_logp, float* tau, float* out, float* lse, void* workspace,
+                                         size_t ws_bytes, void* stream);
+
+/*
+ * The whole SR-SWA decode step in one launch: the ring append of rswa_decode_append and
+ * the fused router + gathered attention of srswa_decode_routed. Results equal rswa_append,
+ * srswa_route and srswa_decode called in turn. Arguments: those of srswa_decode_routed
+ * plus k_new, v_new (bf16 [B][H][D]) and slot_out (int32 [B] or NULL), with ring_k,
+ * ring_v, wp and fill updated in place as by rswa_append.
+ */
+RSWA_API rswa_status srswa_step(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new,
+                                const float* q_idx, const float* kbar, float idx_scale, int32_t topk, const void* pk,
+                                const void* pv, const int32_t* prefix_len, void* ring_k, void* ring_v, int32_t* wp,
+                                int32_t* fill, int32_t* slot_out, float scale, int32_t* blk_idx, float* blk_logp,
+                                float* tau, float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * SR-SWA chunked prefill. The pages size prefill memory by a
  * per-token router score tensor of about [tokens, context/32] (serving notes,
  * --max-prefill-tokens), i.e. every output-side token of a chunk is routed by itself;
@@ -361,6 +422,34 @@ RSWA_API rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, cons
                                       const int32_t* blk_idx, const float* blk_logp, int32_t topk, const void* ring_k,
                                       const void* ring_v, const int32_t* wp, const int32_t* fill, float scale,
                                       float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * FP8 ring (the KV-cache quantisation above extended to the ring): the ring K and V are
+ * stored as E4M3 codes [B][H][n][D] with one f32 scale per row [B][H][n] for K and one
+ * for V. The ring is written one token at a time, so each written row is quantised on its
+ * own: scale = amax over its D dims / 448 (1 if 0), code = E4M3(x / scale), nearest even,
+ * saturating, both in f32 (the prefix rule with a one-row block).
+ *
+ * rswa_append_fp8: rswa_append into an FP8 ring (same wp / fill / slot_out / status rules).
+ * rswa_decode_fp8kv / srswa_decode_fp8kv: rswa_decode_fp8 / srswa_decode_fp8 reading the
+ *   ring as codes and row scales; workspace as rswa_decode (srswa_decode).
+ */
+RSWA_API rswa_status rswa_append_fp8(const rswa_dims* dims, uint8_t* ring_k8, uint8_t* ring_v8, float* ring_kscale,
+                                     float* ring_vscale, const void* k_new, const void* v_new, int32_t* wp,
+                                     int32_t* fill, int32_t* slot_out, int32_t* status, void* stream);
+
+RSWA_API rswa_status rswa_decode_fp8kv(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                                       const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                                       const uint8_t* ring_k8, const uint8_t* ring_v8, const float* ring_kscale,
+                                       const float* ring_vscale, const int32_t* wp, const int32_t* fill, float scale,
+                                       float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+RSWA_API rswa_status srswa_decode_fp8kv(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                                        const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                                        const int32_t* blk_idx, const float* blk_logp, int32_t topk,
+                                        const uint8_t* ring_k8, const uint8_t* ring_v8, const float* ring_kscale,
+                                        const float* ring_vscale, const int32_t* wp, const int32_t* fill, float scale,
+                                        float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * page2d rotary position encoding (Unlimited-OCR-2 SR-SWA explainer, 2D 位置编码: two

@@ -25,6 +25,7 @@ OP_DECODE = 1
 OP_SRSWA_DECODE = 2
 OP_ROUTE = 3
 OP_PREFILL = 4
+OP_SRSWA_ROUTED = 5
 
 STATUS_NAMES = {0: "RSWA_OK", 1: "RSWA_ERR_INVALID", 2: "RSWA_ERR_UNSUPPORTED", 3: "RSWA_ERR_CUDA",
                 5: "RSWA_ERR_DEVICE_CHECK"}
@@ -37,7 +38,9 @@ DEVICE_PIPELINE = 0x10
 EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_check_status", "rswa_append",
             "rswa_decode", "srswa_index_pool", "srswa_route", "srswa_decode", "rswa_decode_noalloc", "rswa_prefill",
             "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill",
-            "rswa_decode_append", "srswa_decode_append", "rswa_rope_page2d", "rswa_append_rope")
+            "rswa_decode_append", "srswa_decode_append", "rswa_rope_page2d", "rswa_append_rope", "rswa_append_fp8",
+            "rswa_decode_fp8kv", "srswa_decode_fp8kv", "rswa_test_arm_wait_timeout", "srswa_decode_routed",
+            "srswa_step")
 
 
 class RswaError(RuntimeError):
@@ -84,6 +87,11 @@ def load(path: str | None = None):
             "rswa_version": ([], I32),
             "rswa_workspace_bytes": ([DP, I32], SZ),
             "rswa_check_status": ([P, SZ, P, P], ctypes.c_int),
+            "rswa_test_arm_wait_timeout": ([I32, I64], ctypes.c_int),
+            "srswa_decode_routed": ([DP, P, P, P, F32, I32, P, P, P, P, P, P, P, F32, P, P, P, P, P, P, SZ, P],
+                                    ctypes.c_int),
+            "srswa_step": ([DP, P, P, P, P, P, F32, I32, P, P, P, P, P, P, P, P, F32, P, P, P, P, P, P, SZ, P],
+                           ctypes.c_int),
             "rswa_append": ([DP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "rswa_decode": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_index_pool": ([DP, P, P, P, P], ctypes.c_int),
@@ -101,6 +109,10 @@ def load(path: str | None = None):
                                     ctypes.c_int),
             "rswa_rope_page2d": ([I64, I32, I32, P, P, P, P, P, P, ctypes.c_double, I32, P], ctypes.c_int),
             "rswa_append_rope": ([DP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_double, I32, P, P], ctypes.c_int),
+            "rswa_append_fp8": ([DP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "rswa_decode_fp8kv": ([DP, P, P, P, P, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_decode_fp8kv": ([DP, P, P, P, P, P, P, P, P, I32, P, P, P, P, P, P, F32, P, P, P, SZ, P],
+                                   ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -159,6 +171,12 @@ def new_workspace(dims: Dims, op: int, device=None) -> torch.Tensor:
 def route_workspace(batch: int, prefix_cap: int, device=None) -> torch.Tensor:
     """A zero-filled workspace for srswa_route over `batch` sequences of capacity `prefix_cap`."""
     return new_workspace(Dims(batch, 1, 128, 1, prefix_cap), OP_ROUTE, device)
+
+
+def test_arm_wait_timeout(drop_tile: int, wait_limit_ns: int) -> None:
+    """Test hook: the next decode-family call of this thread drops CTA 0's tile `drop_tile`
+    (its bounded wait then runs out) and waits at most `wait_limit_ns` (see rswa.h)."""
+    _check("rswa_test_arm_wait_timeout", load().rswa_test_arm_wait_timeout(int(drop_tile), int(wait_limit_ns)))
 
 
 def check_status(workspace: torch.Tensor, stream=None) -> int:
@@ -384,6 +402,93 @@ def rswa_decode_fp8(q, pk8, pv8, k_scale, v_scale, prefix_len, ring_k, ring_v, w
                                                      _stream(stream)))
 
 
+def fp8_ring_buffers(ring_shape, device=None):
+    """An FP8 ring: E4M3 code tensors (uint8) [B][H][n][D] and f32 row-scale tensors [B][H][n] for K and V."""
+    B, H, n, D = ring_shape
+    dev = device or "cuda"
+    return (torch.zeros((B, H, n, D), dtype=torch.uint8, device=dev),
+            torch.zeros((B, H, n, D), dtype=torch.uint8, device=dev),
+            torch.ones((B, H, n), dtype=torch.float32, device=dev),
+            torch.ones((B, H, n), dtype=torch.float32, device=dev))
+
+
+def _want_fp8_ring(ring_k8, ring_v8, ring_kscale, ring_vscale):
+    B, H, n, D = ring_k8.shape
+    _want(ring_k8, "ring_k8", torch.uint8)
+    _want(ring_v8, "ring_v8", torch.uint8, (B, H, n, D))
+    _want(ring_kscale, "ring_kscale", torch.float32, (B, H, n))
+    _want(ring_vscale, "ring_vscale", torch.float32, (B, H, n))
+    return B, H, n, D
+
+
+def rswa_append_fp8(ring_k8, ring_v8, ring_kscale, ring_vscale, k_new, v_new, wp, fill, slot_out=None, status=None,
+                    stream=None):
+    """rswa_append into an FP8 ring (each written row quantised with its own scale)."""
+    B, H, n, D = _want_fp8_ring(ring_k8, ring_v8, ring_kscale, ring_vscale)
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    if status is not None:
+        _want(status, "status", status.dtype)
+    dims = Dims(B, H, D, n, 0)
+    _check("rswa_append_fp8", load().rswa_append_fp8(ctypes.byref(dims), _ptr(ring_k8), _ptr(ring_v8),
+                                                     _ptr(ring_kscale), _ptr(ring_vscale), _ptr(k_new), _ptr(v_new),
+                                                     _ptr(wp), _ptr(fill), _ptr(slot_out), _ptr(status),
+                                                     _stream(stream)))
+
+
+def rswa_decode_fp8kv(q, pk8, pv8, k_scale, v_scale, prefix_len, ring_k8, ring_v8, ring_kscale, ring_vscale, wp, fill,
+                      out, workspace, lse=None, scale=None, stream=None):
+    """rswa_decode_fp8 with the ring read as E4M3 codes and row scales."""
+    B, H, cap, D = _want_fp8_prefix(pk8, pv8, k_scale, v_scale)
+    n = _want_fp8_ring(ring_k8, ring_v8, ring_kscale, ring_vscale)[2]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("rswa_decode_fp8kv", load().rswa_decode_fp8kv(ctypes.byref(dims), _ptr(q), _ptr(pk8), _ptr(pv8),
+                                                         _ptr(k_scale), _ptr(v_scale), _ptr(prefix_len),
+                                                         _ptr(ring_k8), _ptr(ring_v8), _ptr(ring_kscale),
+                                                         _ptr(ring_vscale), _ptr(wp), _ptr(fill), scale, _ptr(out),
+                                                         _ptr(lse), _ptr(workspace), workspace.numel(),
+                                                         _stream(stream)))
+
+
+def srswa_decode_fp8kv(q, pk8, pv8, k_scale, v_scale, prefix_len, blk_idx, blk_logp, ring_k8, ring_v8, ring_kscale,
+                       ring_vscale, wp, fill, out, workspace, lse=None, scale=None, stream=None):
+    """srswa_decode_fp8 with the ring read as E4M3 codes and row scales."""
+    B, H, cap, D = _want_fp8_prefix(pk8, pv8, k_scale, v_scale)
+    n = _want_fp8_ring(ring_k8, ring_v8, ring_kscale, ring_vscale)[2]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32)
+    topk = blk_idx.shape[1]
+    _want(blk_logp, "blk_logp", torch.float32, (B, topk))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_decode_fp8kv", load().srswa_decode_fp8kv(ctypes.byref(dims), _ptr(q), _ptr(pk8), _ptr(pv8),
+                                                           _ptr(k_scale), _ptr(v_scale), _ptr(prefix_len),
+                                                           _ptr(blk_idx), _ptr(blk_logp), topk, _ptr(ring_k8),
+                                                           _ptr(ring_v8), _ptr(ring_kscale), _ptr(ring_vscale),
+                                                           _ptr(wp), _ptr(fill), scale, _ptr(out), _ptr(lse),
+                                                           _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
 def srswa_decode_fp8(q, pk8, pv8, k_scale, v_scale, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, out,
                      workspace, lse=None, scale=None, stream=None):
     B, H, cap, D = _want_fp8_prefix(pk8, pv8, k_scale, v_scale)
@@ -559,3 +664,63 @@ def rswa_prefill(q, k_out, v_out, pk, pv, prefix_len, out, workspace, lse=None, 
                                                _ptr(pv), _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp),
                                                _ptr(fill), scale, _ptr(out), _ptr(lse), 1 if write_ring else 0,
                                                _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def _want_routed(q, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, blk_idx, blk_logp, tau, out, lse,
+                 workspace):
+    B, H, cap, D = pk.shape
+    n = ring_k.shape[2]
+    topk = blk_idx.shape[1]
+    nb_cap = (cap + 31) // 32
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(q_idx, "q_idx", torch.float32, (B, 32))
+    _want(kbar, "kbar", torch.float32, (B, nb_cap, 32))
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    _want(blk_idx, "blk_idx", torch.int32, (B, topk))
+    _want(blk_logp, "blk_logp", torch.float32, (B, topk))
+    if tau is not None:
+        _want(tau, "tau", torch.float32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    return B, H, cap, D, n, topk
+
+
+def srswa_decode_routed(q, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, blk_idx, blk_logp, out,
+                        workspace, lse=None, tau=None, idx_scale=1.0, scale=None, stream=None):
+    """srswa_route + srswa_decode in one launch: the route (blk_idx, blk_logp, tau) is an output.
+    workspace: new_workspace(dims, OP_SRSWA_ROUTED)."""
+    B, H, cap, D, n, topk = _want_routed(q, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, blk_idx,
+                                         blk_logp, tau, out, lse, workspace)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_decode_routed", load().srswa_decode_routed(
+        ctypes.byref(dims), _ptr(q), _ptr(q_idx), _ptr(kbar), float(idx_scale), topk, _ptr(pk), _ptr(pv),
+        _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp), _ptr(fill), scale, _ptr(blk_idx), _ptr(blk_logp),
+        _ptr(tau), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def srswa_step(q, k_new, v_new, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, blk_idx, blk_logp, out,
+               workspace, lse=None, tau=None, slot_out=None, idx_scale=1.0, scale=None, stream=None):
+    """The whole SR-SWA decode step in one launch: rswa_append + srswa_route + srswa_decode.
+    workspace: new_workspace(dims, OP_SRSWA_ROUTED)."""
+    B, H, cap, D, n, topk = _want_routed(q, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, blk_idx,
+                                         blk_logp, tau, out, lse, workspace)
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_step", load().srswa_step(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_idx), _ptr(kbar), float(idx_scale), topk,
+        _ptr(pk), _ptr(pv), _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp), _ptr(fill), _ptr(slot_out), scale,
+        _ptr(blk_idx), _ptr(blk_logp), _ptr(tau), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))

@@ -72,6 +72,12 @@ rswa_status check_dims(const char* fn, const rswa_dims* d, bool need_prefix) {
 
 int32_t* ws_status(void* ws) { return reinterpret_cast<int32_t*>(ws); }
 
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Set by rswa_test_arm_wait_timeout for the next decode launch of this host thread only.
+thread_local int g_test_drop_tile = -1;
+thread_local uint64_t g_test_wait_ns = 0;
+
 }  // namespace
 
 namespace rswa {
@@ -86,7 +92,7 @@ extern "C" {
 
 const char* rswa_last_error(void) { return g_last_error; }
 
-int32_t rswa_version(void) { return 3; }
+int32_t rswa_version(void) { return 4; }
 
 size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
   const char* fn = "rswa_workspace_bytes";
@@ -116,6 +122,20 @@ size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
         }
       return most;
     }
+    case RSWA_OP_SRSWA_ROUTED: {
+      // srswa_decode_routed / srswa_step: the SR-SWA decode plan (any topk, the step's extra
+      // token tile) followed by the fused router's area
+      size_t most = 0;
+      for (int k = 1; k <= rswa::kMaxTopk; ++k)
+        for (int64_t extra = 0; extra <= 1; ++extra) {
+          const size_t b = rswa::plan_decode_workspace(dims->batch, dims->heads,
+                                                       rswa::decode_max_tiles_sparse(k, dims->ring) + extra,
+                                                       rswa::device_sm_count())
+                               .bytes;
+          most = b > most ? b : most;
+        }
+      return align256(most) + rswa::route_area_bytes(dims->batch, dims->prefix_cap);
+    }
     case RSWA_OP_ROUTE:
     case RSWA_OP_PREFILL:
       return 256;
@@ -134,12 +154,25 @@ rswa_status rswa_check_status(void* workspace, size_t ws_bytes, int32_t* device_
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "rswa_check_status: reading the status word");
   if (host != 0) {
-    e = cudaMemsetAsync(workspace, 0, sizeof(int32_t), s);
+    // a timed-out wait can leave completion counters of the abandoned work items behind: the
+    // whole workspace goes back to its zero-filled initial state; otherwise only the status word
+    const size_t clear = (host & RSWA_DEVICE_WAIT_TIMEOUT) ? ws_bytes : sizeof(int32_t);
+    e = cudaMemsetAsync(workspace, 0, clear, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "rswa_check_status: clearing the status word");
   }
   if (device_status) *device_status = host;
   if (host != 0) return fail(RSWA_ERR_DEVICE_CHECK, "%s: device status 0x%x", fn, host);
+  return ok();
+}
+
+rswa_status rswa_test_arm_wait_timeout(int32_t drop_tile, int64_t wait_limit_ns) {
+  const char* fn = "rswa_test_arm_wait_timeout";
+  if (drop_tile < -1) return fail(RSWA_ERR_INVALID, "%s: drop_tile must be >= -1 (got %d)", fn, drop_tile);
+  if (wait_limit_ns < 1000 || wait_limit_ns > 10000000000ll)
+    return fail(RSWA_ERR_INVALID, "%s: wait_limit_ns must be in [1e3, 1e10] (got %lld)", fn, (long long)wait_limit_ns);
+  g_test_drop_tile = drop_tile;
+  g_test_wait_ns = (uint64_t)wait_limit_ns;
   return ok();
 }
 
@@ -193,6 +226,28 @@ struct AppendSrc {
   int32_t* slot_out;
 };
 constexpr AppendSrc kNoAppend{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+
+// An FP8 ring (codes + row scales) in place of the bf16 ring_k / ring_v.
+struct Ring8Src {
+  const void* k8;
+  const void* v8;
+  const float* ks;
+  const float* vs;
+  bool on;
+};
+constexpr Ring8Src kNoRing8{nullptr, nullptr, nullptr, nullptr, false};
+
+// The SR-SWA router fused into the decode launch: its inputs and the route outputs.
+struct RouteSrc {
+  const float* q_idx;
+  const float* kbar;
+  float idx_scale;
+  int32_t* blk_idx;
+  float* blk_logp;
+  float* tau;
+  bool on;
+};
+constexpr RouteSrc kNoRoute{nullptr, nullptr, 0.f, nullptr, nullptr, nullptr, false};
 constexpr size_t kGridCounterOffset = 128;  // an int32 inside the workspace's 256-byte status area
 
 // plan_budget > 0: plan the split-KV work to fit a workspace of that many bytes.
@@ -200,8 +255,14 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
                                  BandSrc band, AppendSrc app, const int32_t* prefix_len, const int32_t* blk_idx,
                                  const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                                  const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
-                                 void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0) {
+                                 void* workspace, size_t ws_bytes, void* stream, size_t plan_budget = 0,
+                                 Ring8Src r8 = kNoRing8, RouteSrc rt = kNoRoute) {
   const NvtxRange nvtx_range(fn);
+  // a wait-timeout test knob applies to this call only, whether or not it launches
+  const int test_drop_tile = g_test_drop_tile;
+  const uint64_t test_wait_ns = g_test_wait_ns;
+  g_test_drop_tile = -1;
+  g_test_wait_ns = 0;
   rswa_status st = check_dims(fn, dims, true);
   if (st != RSWA_OK) return st;
   REQUIRE_PTR(q);
@@ -229,6 +290,18 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
     REQUIRE_PTR_OR_NULL(ring_k);
     REQUIRE_PTR_OR_NULL(ring_v);
     if (prefix_len == nullptr) return fail(RSWA_ERR_INVALID, "%s: prefix_len must not be NULL", fn);
+  } else if (r8.on) {
+    const void* ring_k8 = r8.k8;
+    const void* ring_v8 = r8.v8;
+    const float* ring_kscale = r8.ks;
+    const float* ring_vscale = r8.vs;
+    REQUIRE_PTR(ring_k8);
+    REQUIRE_PTR(ring_v8);
+    REQUIRE_PTR(ring_kscale);
+    REQUIRE_PTR(ring_vscale);
+    if (!px.fp8) return fail(RSWA_ERR_UNSUPPORTED, "%s: an FP8 ring needs an FP8 prefix", fn);
+    if (prefix_len == nullptr || wp == nullptr || fill == nullptr)
+      return fail(RSWA_ERR_INVALID, "%s: prefix_len, wp and fill must not be NULL", fn);
   } else {
     REQUIRE_PTR(ring_k);
     REQUIRE_PTR(ring_v);
@@ -247,6 +320,18 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
     if (blk_idx == nullptr || blk_logp == nullptr)
       return fail(RSWA_ERR_INVALID, "%s: blk_idx and blk_logp must not be NULL", fn);
     if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
+  }
+  if (rt.on) {
+    const float* q_idx = rt.q_idx;
+    const float* kbar = rt.kbar;
+    REQUIRE_PTR(q_idx);
+    REQUIRE_PTR(kbar);
+    if (!std::isfinite(rt.idx_scale)) return fail(RSWA_ERR_INVALID, "%s: idx_scale must be finite", fn);
+    const int64_t nb_cap = (dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock;
+    if (nb_cap == 0) return fail(RSWA_ERR_INVALID, "%s: prefix_cap must be >= 1", fn);
+    if (nb_cap > rswa::kMaxRouteBlocks)
+      return fail(RSWA_ERR_UNSUPPORTED, "%s: %lld prefix blocks exceed the router's limit of %d", fn,
+                  (long long)nb_cap, rswa::kMaxRouteBlocks);
   }
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
   int64_t max_tiles = sparse ? rswa::decode_max_tiles_sparse(topk, dims->ring)
@@ -269,9 +354,22 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   } else {
     plan = rswa::plan_decode_workspace(dims->batch, dims->heads, max_tiles, rswa::device_sm_count(), plan_budget);
   }
-  if (ws_bytes < plan.bytes)
-    return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes,
-                plan.bytes);
+  size_t need = plan.bytes, route_off = 0;
+  int n_fin = 0;
+  if (rt.on) {
+    // the fused router's CTAs wait on one another: the grid must fit one resident wave of this
+    // kernel, and its last CTAs (item-free when there is room) finalise the routes
+    const int per_sm = rswa::routed_decode_ctas_per_sm();
+    if (per_sm < 1) return fail(RSWA_ERR_CUDA, "%s: occupancy query of the fused router kernel failed", fn);
+    const int64_t slots = (int64_t)rswa::device_sm_count() * per_sm;
+    const int64_t want = plan.items + dims->batch;
+    plan.grid = (int)(want < slots ? want : slots);
+    n_fin = dims->batch < plan.grid ? dims->batch : plan.grid;
+    route_off = align256(plan.bytes);
+    need = route_off + rswa::route_area_bytes(dims->batch, dims->prefix_cap);
+  }
+  if (ws_bytes < need)
+    return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required", fn, ws_bytes, need);
   rswa::DecodeArgs a;
   a.B = dims->batch;
   a.H = dims->heads;
@@ -304,6 +402,10 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.prefix_len = prefix_len;
   a.ring_k = static_cast<const uint16_t*>(ring_k);
   a.ring_v = static_cast<const uint16_t*>(ring_v);
+  a.ring_k8 = static_cast<const uint8_t*>(r8.k8);
+  a.ring_v8 = static_cast<const uint8_t*>(r8.v8);
+  a.ring_ks = r8.ks;
+  a.ring_vs = r8.vs;
   a.wp = wp;
   a.fill = fill;
   a.qscale = scale * 1.4426950408889634f;
@@ -316,6 +418,30 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.blk_idx = blk_idx;
   a.blk_logp = blk_logp;
   a.topk = sparse ? topk : 0;
+  a.wait_limit_ns = test_wait_ns > 0 ? test_wait_ns : rswa::kWaitLimitNs;
+  a.drop_tile = test_drop_tile;
+  a.q_idx = rt.q_idx;
+  a.kbar = rt.kbar;
+  a.idx_scale = rt.idx_scale;
+  a.nsl_cap = (int)(((dims->prefix_cap + rswa::kBlock - 1) / rswa::kBlock + 63) / 64);
+  a.n_fin = n_fin;
+  a.blk_idx_w = rt.blk_idx;
+  a.blk_logp_w = rt.blk_logp;
+  a.tau_w = rt.tau;
+  a.seq_count = a.route_ready = nullptr;
+  a.slice_max = a.slice_z = nullptr;
+  a.slice_i = nullptr;
+  if (rt.on) {  // route area: [seq_count, route_ready][slice_max][slice_z][slice_i]
+    uint8_t* r = ws + route_off;
+    const size_t B = (size_t)dims->batch, nsl = (size_t)a.nsl_cap;
+    a.seq_count = reinterpret_cast<int32_t*>(r);
+    a.route_ready = a.seq_count + B;
+    r += align256(B * 8);
+    a.slice_max = reinterpret_cast<float*>(r);
+    r += align256(B * nsl * 4);
+    a.slice_z = reinterpret_cast<float*>(r);
+    a.slice_i = reinterpret_cast<int32_t*>(a.slice_z + B * nsl * 64);
+  }
   cudaError_t e = rswa::launch_decode(a, plan.grid, sparse, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
@@ -347,6 +473,49 @@ rswa_status srswa_decode_fp8(const rswa_dims* dims, const void* q, const uint8_t
   return decode_common("srswa_decode_fp8", true, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
                        kNoAppend, prefix_len,
                        blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status rswa_decode_fp8kv(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                              const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                              const uint8_t* ring_k8, const uint8_t* ring_v8, const float* ring_kscale,
+                              const float* ring_vscale, const int32_t* wp, const int32_t* fill, float scale, float* out,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("rswa_decode_fp8kv", false, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
+                       kNoAppend, prefix_len, nullptr, nullptr, 0, nullptr, nullptr, wp, fill, scale, out, lse,
+                       workspace, ws_bytes, stream, 0, Ring8Src{ring_k8, ring_v8, ring_kscale, ring_vscale, true});
+}
+
+rswa_status srswa_decode_fp8kv(const rswa_dims* dims, const void* q, const uint8_t* pk8, const uint8_t* pv8,
+                               const float* k_scale, const float* v_scale, const int32_t* prefix_len,
+                               const int32_t* blk_idx, const float* blk_logp, int32_t topk, const uint8_t* ring_k8,
+                               const uint8_t* ring_v8, const float* ring_kscale, const float* ring_vscale,
+                               const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("srswa_decode_fp8kv", true, dims, q, PrefixSrc{pk8, pv8, k_scale, v_scale, true}, kNoBand,
+                       kNoAppend, prefix_len, blk_idx, blk_logp, topk, nullptr, nullptr, wp, fill, scale, out, lse,
+                       workspace, ws_bytes, stream, 0, Ring8Src{ring_k8, ring_v8, ring_kscale, ring_vscale, true});
+}
+
+rswa_status rswa_append_fp8(const rswa_dims* dims, uint8_t* ring_k8, uint8_t* ring_v8, float* ring_kscale,
+                            float* ring_vscale, const void* k_new, const void* v_new, int32_t* wp, int32_t* fill,
+                            int32_t* slot_out, int32_t* status, void* stream) {
+  const char* fn = "rswa_append_fp8";
+  const NvtxRange nvtx_range(fn);
+  rswa_status st = check_dims(fn, dims, false);
+  if (st != RSWA_OK) return st;
+  REQUIRE_PTR(ring_k8);
+  REQUIRE_PTR(ring_v8);
+  REQUIRE_PTR(ring_kscale);
+  REQUIRE_PTR(ring_vscale);
+  REQUIRE_PTR(k_new);
+  REQUIRE_PTR(v_new);
+  if (wp == nullptr || fill == nullptr) return fail(RSWA_ERR_INVALID, "%s: wp and fill must not be NULL", fn);
+  cudaError_t e = rswa::launch_append_fp8(dims->batch, dims->heads, dims->ring, ring_k8, ring_v8, ring_kscale,
+                                          ring_vscale, static_cast<const uint16_t*>(k_new),
+                                          static_cast<const uint16_t*>(v_new), wp, fill, slot_out, status,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
 }
 
 rswa_status rswa_quantize_prefix(const rswa_dims* dims, const void* pk, const void* pv, const int32_t* prefix_len,
@@ -464,6 +633,28 @@ rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, const void
   return decode_common("srswa_decode_append", true, dims, q, bf16_prefix(pk, pv), kNoBand,
                        AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, blk_idx, blk_logp,
                        topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_decode_routed(const rswa_dims* dims, const void* q, const float* q_idx, const float* kbar,
+                                float idx_scale, int32_t topk, const void* pk, const void* pv,
+                                const int32_t* prefix_len, const void* ring_k, const void* ring_v, const int32_t* wp,
+                                const int32_t* fill, float scale, int32_t* blk_idx, float* blk_logp, float* tau,
+                                float* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common("srswa_decode_routed", true, dims, q, bf16_prefix(pk, pv), kNoBand, kNoAppend, prefix_len,
+                       blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes,
+                       stream, 0, kNoRing8, RouteSrc{q_idx, kbar, idx_scale, blk_idx, blk_logp, tau, true});
+}
+
+rswa_status srswa_step(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new, const float* q_idx,
+                       const float* kbar, float idx_scale, int32_t topk, const void* pk, const void* pv,
+                       const int32_t* prefix_len, void* ring_k, void* ring_v, int32_t* wp, int32_t* fill,
+                       int32_t* slot_out, float scale, int32_t* blk_idx, float* blk_logp, float* tau, float* out,
+                       float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  if (k_new == nullptr || v_new == nullptr) return fail(RSWA_ERR_INVALID, "srswa_step: k_new and v_new must not be NULL");
+  return decode_common("srswa_step", true, dims, q, bf16_prefix(pk, pv), kNoBand,
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, blk_idx, blk_logp,
+                       topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream, 0, kNoRing8,
+                       RouteSrc{q_idx, kbar, idx_scale, blk_idx, blk_logp, tau, true});
 }
 
 rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,

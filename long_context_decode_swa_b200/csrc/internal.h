@@ -54,6 +54,34 @@ struct DecodeArgs {
   int32_t* fill_w;
   int32_t* slot_out;
   int32_t* grid_counter;
+  // FP8 ring (decode only): E4M3 code rows [B][H][n][D] with one f32 scale per row [B][H][n]
+  // for K and for V, in place of ring_k / ring_v (which are then null)
+  const uint8_t* ring_k8;
+  const uint8_t* ring_v8;
+  const float* ring_ks;
+  const float* ring_vs;
+  // every pipeline wait gives up after wait_limit_ns; drop_tile >= 0 (a test of that path
+  // only) makes CTA 0 skip the copy of its CTA-local tile drop_tile while still waiting on it
+  uint64_t wait_limit_ns;
+  int drop_tile;
+  // SR-SWA with the router fused into the launch: every warp of the grid scores 64-block
+  // slices of kbar against q_idx and publishes each slice sorted; the last n_fin CTAs each
+  // finalise the route of their sequences (entmax threshold, top-k, ln p) into blk_idx_w /
+  // blk_logp_w (tau_w nullable) and raise route_ready[b]; attention warps wait for that flag
+  // before they issue a routed block's copy (token and ring tiles need no route)
+  const float* q_idx;    // [B][32]
+  const float* kbar;     // [B][nb_cap][32]
+  float idx_scale;
+  int nsl_cap;           // slices per sequence: ceil(nb_cap / 64)
+  int n_fin;
+  float* slice_max;      // [B][nsl_cap]
+  float* slice_z;        // [B][nsl_cap][64], each slice sorted (larger score first, ties to the smaller block)
+  int32_t* slice_i;      // [B][nsl_cap][64]
+  int32_t* seq_count;    // [B]: slices published in this launch
+  int32_t* route_ready;  // [B]: the route was published in this launch
+  int32_t* blk_idx_w;    // [B][topk]
+  float* blk_logp_w;
+  float* tau_w;
 };
 
 // Workspace layout shared by every op: [status: 256 B][counters][partials].
@@ -74,6 +102,14 @@ cudaError_t launch_append(int B, int H, int n, uint16_t* ring_k, uint16_t* ring_
                           const uint16_t* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, int32_t* status,
                           cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int grid, bool sparse, cudaStream_t stream);
+// Resident CTAs per SM of the decode kernel with the router fused (occupancy query), and the
+// bytes of its route area in the workspace.
+int routed_decode_ctas_per_sm();
+size_t route_area_bytes(int B, int64_t cap);
+// Ring append into an FP8 ring: each written K / V row quantised with its own scale.
+cudaError_t launch_append_fp8(int B, int H, int n, uint8_t* ring_k8, uint8_t* ring_v8, float* ring_ks, float* ring_vs,
+                              const uint16_t* k_new, const uint16_t* v_new, int32_t* wp, int32_t* fill,
+                              int32_t* slot_out, int32_t* status, cudaStream_t stream);
 // page2d rotary encoding of rows x [H][D] of q (and k when not NULL); outputs may alias inputs.
 cudaError_t launch_rope(int64_t rows, int H, int D, const uint16_t* q, uint16_t* q_out, const uint16_t* k,
                         uint16_t* k_out, const int32_t* tok_pos, const int32_t* page, double base, int page_mod,

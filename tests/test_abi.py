@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     lib = rswa.load()
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.rswa_version() == 3
+    assert lib.rswa_version() == 4
 
 
 def _err():
@@ -200,3 +200,62 @@ def test_missing_library_fails_loudly(tmp_path):
     code = "import long_context_decode_swa_b200 as r\nr.load()"
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT, timeout=300)
     assert out.returncode != 0 and "not found" in out.stderr
+
+
+def test_fp8_ring_entry_points_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64)
+    ws = lib.rswa_workspace_bytes(ctypes.byref(d), 1)
+
+    def dec(ring_k8=A, ring_vscale=A, pk8=A, ws_bytes=ws):
+        return lib.rswa_decode_fp8kv(ctypes.byref(d), A, pk8, A, A, A, A, ring_k8, A, A, ring_vscale, A, A,
+                                     ctypes.c_float(0.088), A, None, A, ctypes.c_size_t(ws_bytes), None)
+
+    assert dec(ring_k8=None) == INVALID and "ring_k8" in _err()
+    assert dec(ring_vscale=MIS) == INVALID and "aligned" in _err()
+    assert dec(pk8=None) == INVALID
+    assert dec(ws_bytes=16) == INVALID and "workspace" in _err()
+
+    def app(ring_k8=A, k_new=A, wp=A, dims=d):
+        return lib.rswa_append_fp8(ctypes.byref(dims), ring_k8, A, A, A, k_new, A, wp, A, None, None, None)
+
+    assert app(ring_k8=None) == INVALID and "ring_k8" in _err()
+    assert app(k_new=MIS) == INVALID and "aligned" in _err()
+    assert app(wp=None) == INVALID and "wp and fill" in _err()
+    assert app(dims=Dims(2, 4, 64, 128, 0)) == UNSUPPORTED
+
+
+def test_wait_timeout_hook_validation():
+    lib = rswa.load()
+    assert lib.rswa_test_arm_wait_timeout(-2, 20_000_000) == INVALID and "drop_tile" in _err()
+    assert lib.rswa_test_arm_wait_timeout(0, 10) == INVALID and "wait_limit_ns" in _err()
+    assert lib.rswa_test_arm_wait_timeout(0, 20_000_000) == 0
+    # the armed knob is consumed by the next decode-family call even when that call fails validation
+    d = Dims(2, 4, 128, 128, 64)
+    assert lib.rswa_decode(ctypes.byref(d), None, A, A, A, A, A, A, A, ctypes.c_float(0.088), A, None, A,
+                           ctypes.c_size_t(1 << 20), None) == INVALID
+
+
+def test_fused_router_entry_points_validation():
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64 * 32)
+    ws = lib.rswa_workspace_bytes(ctypes.byref(d), 5)
+    assert ws > lib.rswa_workspace_bytes(ctypes.byref(d), 2)   # the decode plan plus the router's area
+
+    def routed(q_idx=A, kbar=A, topk=16, blk=A, idx_scale=1.0, dims=d):
+        return lib.srswa_decode_routed(ctypes.byref(dims), A, q_idx, kbar, ctypes.c_float(idx_scale), topk, A, A, A,
+                                       A, A, A, A, ctypes.c_float(0.088), blk, A, None, A, None, A,
+                                       ctypes.c_size_t(ws), None)
+
+    assert routed(q_idx=None) == INVALID and "q_idx" in _err()
+    assert routed(kbar=MIS) == INVALID and "aligned" in _err()
+    assert routed(topk=33) == INVALID and "topk" in _err()
+    assert routed(blk=None) == INVALID
+    assert routed(idx_scale=float("inf")) == INVALID and "idx_scale" in _err()
+    assert routed(dims=Dims(2, 4, 128, 128, 8193 * 32)) == UNSUPPORTED and "limit" in _err()
+
+    def step(k_new=A, slot_out=None):
+        return lib.srswa_step(ctypes.byref(d), A, k_new, A, A, A, ctypes.c_float(1.0), 16, A, A, A, A, A, A, A,
+                              slot_out, ctypes.c_float(0.088), A, A, None, A, None, A, ctypes.c_size_t(ws), None)
+
+    assert step(k_new=None) == INVALID and "k_new" in _err()
