@@ -10,7 +10,8 @@ A step is one decode step of the whole batch through the C ABI:
   configs 6, 7:           configs 2 and 4 over an FP8 (E4M3) prefix, quantised
                           once before timing: rswa_append + rswa_decode_fp8
                           (+ srswa_route + srswa_decode_fp8)
-  config 8 (SR-SWA chunked prefill): srswa_route_tokens + srswa_prefill
+  config 8 (SR-SWA chunked prefill): srswa_route_tokens + srswa_prefill (grouping by
+                          routed block set, band part and routed part on tcgen05)
   config 9 (page2d rotary encoding of a prefill chunk's q and k): rswa_rope_page2d
   config 10:              config 4 with the page2d encoding: rswa_append_rope +
                           srswa_route + srswa_decode
@@ -254,10 +255,11 @@ def measured_peak():
 
 
 def kernel_source_hash(kind: str) -> str:
-    """Hash of the code the measured kernel is built from (kind: dense, sparse, prefill or rope), with
+    """Hash of the code the measured kernel is built from (kind: dense, sparse, prefill, srswa_prefill or rope), with
     comments and blank lines removed: a traffic record stays valid across comment edits only."""
     import re
-    files = {"prefill": ["prefill.cu", "common.cuh"], "rope": ["rope.cu", "common.cuh"]}.get(
+    files = {"prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh"], "rope": ["rope.cu", "common.cuh"],
+             "srswa_prefill": ["srswa_prefill.cu", "prefill.cu", "tcgen05.cuh", "common.cuh"]}.get(
         kind, ["decode.cu", "common.cuh", "internal.h"])
     h = hashlib.sha256()
     for f in files:
@@ -508,7 +510,8 @@ class SrswaPrefillProblem:
         self.logp = torch.empty((B, T, 16), dtype=torch.float32, device="cuda")
         self.out = torch.empty((B, H, T, w["D"]), dtype=torch.float32, device="cuda")
         self.lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
-        self.ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        self.ws = rswa.srswa_prefill_workspace(B, H, T, w["cap"], ring=w["n"])
+        self.ws_route = torch.zeros(256, dtype=torch.uint8, device="cuda")
         self.sparse = True
         torch.cuda.synchronize()
 
@@ -516,7 +519,7 @@ class SrswaPrefillProblem:
         d, r = self.d, self.rswa
         if ev is not None:
             ev[2].record()
-        r.srswa_route_tokens(self.q_tok, self.kbar, d["prefix_len"], self.blk, self.logp, self.ws,
+        r.srswa_route_tokens(self.q_tok, self.kbar, d["prefix_len"], self.blk, self.logp, self.ws_route,
                              prefix_cap=self.w["cap"])
         if ev is not None:
             ev[3].record()
@@ -527,11 +530,6 @@ class SrswaPrefillProblem:
         if ev is not None:
             ev[1].record()
         return 2
-
-
-def alu_peak_tflops() -> float:
-    """FP32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the recipe's SM count and max clock)."""
-    return 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def measured_tensor_peak(sustained: bool):
@@ -704,13 +702,12 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
     kern_s = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1e3
     route_s = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) / 1e3 if sparse else 0.0
     del graph
+    sustained = ms_total > 1000.0
+    peak, src = measured_tensor_peak(sustained)
     if sparse:
         flops = srswa_prefill_flops(w, prob.blk.cpu().numpy(), prob.logp.cpu().numpy())
-        peak, src = alu_peak_tflops(), "derived"
     else:
         flops = prefill_flops(w)
-        sustained = ms_total > 1000.0
-        peak, src = measured_tensor_peak(sustained)
     achieved = flops / kern_s / 1e12
     e2e = run_prefill_e2e(prob, K, W) if not args.no_e2e else {"ms": float("nan"), "h2d": 0, "d2h": 0}
     e2e_ms = max_over_ranks(world, e2e["ms"])
@@ -719,16 +716,18 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
     return {
         "metric": METRIC, "value": value, "unit": "prefill chunks/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32" if sparse else "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "dtype": "bf16-mma/f32-acc", "storage_dtype": "bf16", "data": "synthetic", "impl": "ours",
         "config": config_of(w, args, world),
         "timing": TIMING_NOTE,
         "qtok_per_s": value * B * H * T,
-        "roofline": ({"bound": "alu", "kernel": "srswa decode_kernel<true, bf16> (chunked-prefill queries)",
+        "roofline": ({"bound": "tensor", "kernel": "SR-SWA prefill attention: group_kernel + prefill_kernel (band "
+                                                 "and ring, tcgen05) + routed_kernel (routed blocks, tcgen05)",
                       "achieved": achieved, "peak": peak,
-                      "peak_source": "derived: FP32 FMA, 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (no measured ALU "
-                                     "peak); gathered rows mostly hit L2",
+                      "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json); "
+                                     "FLOPs counted per query over its own routed rows and band",
                       "unit": "TFLOP/s", "frac": achieved / peak,
-                      "traffic": committed_traffic(f"srswa_prefill_config{args.config}", kernel_source_hash("sparse")),
+                      "traffic": committed_traffic(f"srswa_prefill_config{args.config}",
+                                                 kernel_source_hash("srswa_prefill")),
                       "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6} if sparse else
                      {"bound": "tensor", "kernel": "prefill_kernel (tcgen05)", "achieved": achieved, "peak": peak,
                       "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)",

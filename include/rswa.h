@@ -80,7 +80,7 @@ typedef struct {
 #define RSWA_OP_SRSWA_DECODE 2  /* srswa_decode, srswa_decode_fp8, srswa_decode_append
                                    (any topk in 1..32)                                      */
 #define RSWA_OP_ROUTE 3         /* srswa_route, srswa_route_tokens (256 bytes)               */
-#define RSWA_OP_PREFILL 4       /* rswa_prefill, srswa_prefill (256 bytes)                   */
+#define RSWA_OP_PREFILL 4       /* rswa_prefill (256 bytes); srswa_prefill: srswa_prefill_workspace_bytes */
 #define RSWA_OP_SRSWA_ROUTED 5  /* srswa_decode_routed, srswa_step (any topk in 1..32)       */
 
 /* Message of the last failed call on this host thread ("" if none). */
@@ -263,7 +263,9 @@ RSWA_API rswa_status srswa_decode(const rswa_dims* dims, const void* q, const vo
  * calls no cudaMalloc/cudaFree and no allocating library routine.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture on the device.
+ *   before any stream capture on the device. The address is kept for the
+ *   life of the process: do not use this entry point across a reset of the
+ *   device (cudaDeviceReset) or after its primary context was destroyed.
  * - Every call shares the one array per device: calls whose work overlaps on
  *   the GPU (other streams, other threads) race and give wrong results.
  *   Serialise them, e.g. on one stream.
@@ -357,18 +359,27 @@ RSWA_API rswa_status srswa_step(const rswa_dims* dims, const void* q, const void
  *   q_idx    : f32 [B][T][32];  kbar : f32 [B][ceil(prefix_cap / 32)][32]
  *   blk_idx  : int32 [B][T][topk];  blk_logp : f32 [B][T][topk]
  *   workspace: >= 256 bytes (status word).  Unsupported: B * T > 65535.
- * srswa_prefill: the attention of the chunk's T queries.
+ * srswa_prefill: the attention of the chunk's T queries (T <= 8192).
  *   q, k_out, v_out : bf16 [B][H][T][D] (the chunk's queries and output K/V)
  *   pk, pv, prefix_len : as srswa_decode;  blk_idx / blk_logp from srswa_route_tokens
  *   ring_k, ring_v, wp, fill : the previous chunk's ring, or all NULL for the first chunk
  *   out : f32 [B][H][T][D];  lse : f32 [B][H][T] or NULL
- *   workspace: >= 256 bytes (status word; every query is one work item).
- * Each query runs through the gathered-decode pipeline (its routed blocks, then the ring
- * part, then the band, as 32-row tiles).
+ *   workspace: srswa_prefill_workspace_bytes(dims, T) bytes, zero-initialised once
+ *   (status word, grouping scratch, and the band part's lse when lse is NULL).
+ * The routed blocks and the band are disjoint key sets, so the softmax over their union is
+ * the log-sum-exp merge of one over each: the band and ring part of every query runs on the
+ * tcgen05 prefill kernel (as rswa_prefill, prefix left out); the chunk's queries are grouped
+ * by the set of blocks their routes select, and each group of up to 128 queries runs, per
+ * head, as one 128-row tcgen05 tile against its blocks (passes of 16 blocks) with a per-
+ * (query, block) bias ln p, merged into the band result. P is rounded to bf16 for the P.V
+ * product, as in rswa_prefill. Route entries naming a block past prefix_len are flagged
+ * (RSWA_DEVICE_BAD_BLOCK_IDX) and attend to nothing.
  */
 RSWA_API rswa_status srswa_route_tokens(const rswa_dims* dims, int32_t T, const float* q_idx, const float* kbar,
                                         const int32_t* prefix_len, float idx_scale, int32_t topk, int32_t* blk_idx,
                                         float* blk_logp, void* workspace, size_t ws_bytes, void* stream);
+
+RSWA_API size_t srswa_prefill_workspace_bytes(const rswa_dims* dims, int32_t T);
 
 RSWA_API rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out,
                                    const void* v_out, const void* pk, const void* pv, const int32_t* prefix_len,

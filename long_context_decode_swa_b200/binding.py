@@ -40,7 +40,7 @@ EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_che
             "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill",
             "rswa_decode_append", "srswa_decode_append", "rswa_rope_page2d", "rswa_append_rope", "rswa_append_fp8",
             "rswa_decode_fp8kv", "srswa_decode_fp8kv", "rswa_test_arm_wait_timeout", "srswa_decode_routed",
-            "srswa_step")
+            "srswa_step", "srswa_prefill_workspace_bytes")
 
 
 class RswaError(RuntimeError):
@@ -92,6 +92,7 @@ def load(path: str | None = None):
                                     ctypes.c_int),
             "srswa_step": ([DP, P, P, P, P, P, F32, I32, P, P, P, P, P, P, P, P, F32, P, P, P, P, P, P, SZ, P],
                            ctypes.c_int),
+            "srswa_prefill_workspace_bytes": ([DP, I32], SZ),
             "rswa_append": ([DP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "rswa_decode": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_index_pool": ([DP, P, P, P, P], ctypes.c_int),
@@ -600,9 +601,19 @@ def srswa_route_tokens(q_idx, kbar, prefix_len, blk_idx, blk_logp, workspace, id
                                                            _stream(stream)))
 
 
+def srswa_prefill_workspace(batch: int, heads: int, T: int, prefix_cap: int, ring: int = 128, device=None):
+    """A zero-filled workspace for srswa_prefill over `batch` x `heads` chunks of T queries."""
+    dims = Dims(batch, heads, 128, ring, prefix_cap)
+    n = load().srswa_prefill_workspace_bytes(ctypes.byref(dims), int(T))
+    if n == 0:
+        raise RswaError("srswa_prefill_workspace_bytes", 1, load().rswa_last_error().decode())
+    return torch.zeros(int(n), dtype=torch.uint8, device=device or "cuda")
+
+
 def srswa_prefill(q, k_out, v_out, pk, pv, prefix_len, blk_idx, blk_logp, out, workspace, lse=None, ring_k=None,
                   ring_v=None, wp=None, fill=None, scale=None, ring: int = 128, stream=None):
-    """SR-SWA chunked prefill of T queries per (sequence, head), routes given per token."""
+    """SR-SWA chunked prefill of T queries per (sequence, head), routes given per token.
+    workspace: srswa_prefill_workspace(B, H, T, prefix_cap)."""
     B, H, T, D = q.shape
     cap = pk.shape[2]
     topk = blk_idx.shape[2]

@@ -716,6 +716,7 @@ rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const 
   L.wp_w = wp;
   L.fill_w = fill;
   L.status = ws_status(workspace);
+  L.ignore_prefix = 0;
   cudaError_t e = rswa::launch_prefill(L, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
@@ -782,15 +783,116 @@ rswa_status srswa_route_tokens(const rswa_dims* dims, int32_t T, const float* q_
                       nullptr, nullptr, workspace, ws_bytes, stream);
 }
 
+size_t srswa_prefill_workspace_bytes(const rswa_dims* dims, int32_t T) {
+  const char* fn = "srswa_prefill_workspace_bytes";
+  if (check_dims(fn, dims, true) != RSWA_OK) return 0;
+  if (T < 1) {
+    fail(RSWA_ERR_INVALID, "%s: T must be >= 1 (got %d)", fn, T);
+    return 0;
+  }
+  return 256 + rswa::srswa_prefill_scratch_bytes(dims->batch, dims->heads, T);
+}
+
 rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,
                           const void* pk, const void* pv, const int32_t* prefix_len, const int32_t* blk_idx,
                           const float* blk_logp, int32_t topk, const void* ring_k, const void* ring_v,
                           const int32_t* wp, const int32_t* fill, float scale, float* out, float* lse,
                           void* workspace, size_t ws_bytes, void* stream) {
-  return decode_common("srswa_prefill", true, dims, q, bf16_prefix(pk, pv), BandSrc{T, k_out, v_out}, kNoAppend,
-                       prefix_len,
-                       blk_idx, blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes,
-                       stream);
+  const char* fn = "srswa_prefill";
+  const NvtxRange nvtx_range(fn);
+  g_test_drop_tile = -1;  // the wait-timeout test hook covers the decode kernels only
+  g_test_wait_ns = 0;
+  rswa_status st = check_dims(fn, dims, true);
+  if (st != RSWA_OK) return st;
+  if (T < 1) return fail(RSWA_ERR_INVALID, "%s: T must be >= 1 (got %d)", fn, T);
+  if (T > 8192) return fail(RSWA_ERR_UNSUPPORTED, "%s: chunks of more than 8192 queries (got %d)", fn, T);
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k_out);
+  REQUIRE_PTR(v_out);
+  if (dims->prefix_cap > 0) {
+    REQUIRE_PTR(pk);
+    REQUIRE_PTR(pv);
+  }
+  REQUIRE_PTR(out);
+  REQUIRE_PTR(workspace);
+  REQUIRE_PTR_OR_NULL(lse);
+  if (prefix_len == nullptr) return fail(RSWA_ERR_INVALID, "%s: prefix_len must not be NULL", fn);
+  if (blk_idx == nullptr || blk_logp == nullptr)
+    return fail(RSWA_ERR_INVALID, "%s: blk_idx and blk_logp must not be NULL", fn);
+  if (topk < 1 || topk > rswa::kMaxTopk) return fail(RSWA_ERR_INVALID, "%s: topk must be in [1, 32] (got %d)", fn, topk);
+  if ((ring_k == nullptr) != (ring_v == nullptr))
+    return fail(RSWA_ERR_INVALID, "%s: ring_k and ring_v must both be given or both be NULL", fn);
+  const bool ring = ring_k != nullptr;
+  if (ring) {
+    REQUIRE_PTR(ring_k);
+    REQUIRE_PTR(ring_v);
+    if (wp == nullptr || fill == nullptr) return fail(RSWA_ERR_INVALID, "%s: a ring needs wp and fill", fn);
+  }
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(RSWA_ERR_INVALID, "%s: scale must be finite and > 0", fn);
+  const int64_t bh = (int64_t)dims->batch * dims->heads;
+  const int64_t lim = ((int64_t)1 << 31) - 1;
+  if (bh * T >= lim || bh * dims->prefix_cap >= lim || bh * dims->ring >= lim)
+    return fail(RSWA_ERR_UNSUPPORTED, "%s: more than 2^31 rows in one operand", fn);
+  const size_t need = 256 + rswa::srswa_prefill_scratch_bytes(dims->batch, dims->heads, T);
+  if (ws_bytes < need)
+    return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required "
+                "(srswa_prefill_workspace_bytes)", fn, ws_bytes, need);
+  // workspace: [status 256 B][counts 256 B][group records][query lists][sorted routes][biases][lse of the band part]
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t bt = (size_t)dims->batch * T;
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + 256);
+  int32_t* rec = reinterpret_cast<int32_t*>(ws + 512);
+  int32_t* gq = reinterpret_cast<int32_t*>(ws + 512 + align256(bt * rswa::srswa_prefill_group_rec_ints() * 4));
+  int32_t* gblk = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(gq) + align256(bt * 4));
+  float* gbias = reinterpret_cast<float*>(gblk + bt * rswa::kMaxTopk);
+  float* lse_scratch = gbias + bt * rswa::kMaxTopk;
+  float* lse_use = lse != nullptr ? lse : lse_scratch;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1. group the chunk's queries by routed block set
+  const bool routed = dims->prefix_cap > 0;  // with no prefix rows there is nothing to route to
+  cudaError_t e = cudaSuccess;
+  if (routed) {
+    e = cudaMemsetAsync(counts, 0, 16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "srswa_prefill: clearing the group counters");
+    e = rswa::launch_srswa_group(dims->batch, T, topk, dims->prefix_cap, prefix_len, blk_idx, blk_logp, rec, gq,
+                                 gblk, gbias, counts, ws_status(workspace), s);
+    if (e != cudaSuccess) return cuda_fail(e, "srswa_prefill: grouping");
+  }
+  // 2. the band (and previous-chunk ring) part of every query: the dense tcgen05 prefill, prefix left out
+  rswa::PrefillLaunch L;
+  L.B = dims->batch;
+  L.H = dims->heads;
+  L.n = dims->ring;
+  L.T = T;
+  L.cap = dims->prefix_cap;
+  L.q = q;
+  L.k_out = k_out;
+  L.v_out = v_out;
+  L.pk = pk;
+  L.pv = pv;
+  L.prefix_len = prefix_len;
+  L.ring_k = ring ? ring_k : nullptr;
+  L.ring_v = ring ? ring_v : nullptr;
+  L.wp = wp;
+  L.fill = fill;
+  L.scale = scale;
+  L.out = out;
+  L.lse = lse_use;
+  L.write_ring = 0;
+  L.ring_k_w = nullptr;
+  L.ring_v_w = nullptr;
+  L.wp_w = nullptr;
+  L.fill_w = nullptr;
+  L.status = ws_status(workspace);
+  L.ignore_prefix = 1;
+  e = rswa::launch_prefill(L, s);
+  if (e != cudaSuccess) return cuda_fail(e, "srswa_prefill: band part");
+  if (!routed) return ok();
+  // 3. the routed blocks of every group, per head, merged into (out, lse)
+  e = rswa::launch_srswa_routed(dims->batch, dims->heads, T, topk, dims->prefix_cap, prefix_len, q, pk, pv, rec, gq,
+                                gbias, counts, scale, out, lse_use, ws_status(workspace), s);
+  if (e != cudaSuccess) return cuda_fail(e, "srswa_prefill: routed part");
+  return ok();
 }
 
 // ---------------------------------------------------------------------------

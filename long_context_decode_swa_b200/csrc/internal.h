@@ -153,9 +153,22 @@ struct PrefillLaunch {
   int32_t* wp_w;
   int32_t* fill_w;
   int32_t* status;
+  int ignore_prefix;  // 1: attend to the band and the ring only (m = 0 for every sequence)
 };
 
 size_t prefill_smem_bytes();
 cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t stream);
+
+// SR-SWA chunked prefill on tensor cores: workspace bytes beyond the status area, the grouping
+// of a chunk's queries by routed block set, and the routed part merged into the band part.
+size_t srswa_prefill_scratch_bytes(int B, int H, int T);
+int srswa_prefill_group_rec_ints();
+cudaError_t launch_srswa_group(int B, int T, int topk, int64_t cap, const int32_t* prefix_len, const int32_t* blk,
+                               const float* logp, int32_t* rec, int32_t* gq, int32_t* gblk, float* gbias,
+                               int32_t* counts, int32_t* status, cudaStream_t stream);
+cudaError_t launch_srswa_routed(int B, int H, int T, int topk, int64_t cap, const int32_t* prefix_len, const void* q,
+                                const void* pk, const void* pv, const int32_t* rec, const int32_t* gq,
+                                const float* gbias, const int32_t* counts, float scale, float* out, float* lse,
+                                int32_t* status, cudaStream_t stream);
 
 }  // namespace rswa

@@ -140,6 +140,9 @@ def test_chunked_prefill_entry_points_validation():
     assert pf(k_out=MIS) == INVALID and "aligned" in _err()
     assert pf(ring_k=A) == INVALID and "both" in _err()
     assert pf(ring_k=A, ring_v=A2) == INVALID and "wp and fill" in _err()
+    assert pf(T=9000) == UNSUPPORTED and "8192" in _err()
+    assert pf() == INVALID and "srswa_prefill_workspace_bytes" in _err()      # 256 bytes are too few
+    assert lib.srswa_prefill_workspace_bytes(ctypes.byref(d), 8) > 256
 
 
 def test_fused_step_validation():
