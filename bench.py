@@ -13,8 +13,11 @@ A step is one decode step of the whole batch through the C ABI:
   config 8 (SR-SWA chunked prefill): srswa_route_tokens + srswa_prefill (grouping by
                           routed block set, band part and routed part on tcgen05)
   config 9 (page2d rotary encoding of a prefill chunk's q and k): rswa_rope_page2d
-  config 10:              config 4 with the page2d encoding: rswa_append_rope +
-                          srswa_route + srswa_decode
+  config 10:              config 4 with the page2d encoding of q and k_new inside the
+                          same launch: srswa_step_rope (--unfused: rswa_append_rope +
+                          srswa_route + srswa_decode)
+  config 13:              config 2 with the page2d encoding inside the fused step:
+                          rswa_decode_append_rope
   configs 11, 12:         configs 6 and 7 with an FP8 ring as well: rswa_append_fp8 +
                           rswa_decode_fp8kv (+ srswa_route + srswa_decode_fp8kv)
 (the router's block index keys are pooled once per prefix, before timing).
@@ -105,7 +108,12 @@ def workload(cfg: int) -> dict:
     if cfg == 10:
         w = workload(4)
         w["rope"] = True
-        w["name"] += "; page2d rotary encoding of q and the new key fused into the ring append (rswa_append_rope)"
+        w["name"] += "; page2d rotary encoding of q and the new key inside the same launch (srswa_step_rope)"
+        return w
+    if cfg == 13:
+        w = workload(2)
+        w["rope"] = True
+        w["name"] += "; page2d rotary encoding of q and the new key inside the fused step (rswa_decode_append_rope)"
         return w
     if cfg in (11, 12):  # configs 6 and 7 with the ring in FP8 too (row scales)
         w = workload(6 if cfg == 11 else 7)
@@ -338,8 +346,7 @@ class Problem:
         self.fp8 = bool(w.get("fp8"))
         # SR-SWA over a bf16 prefix and ring: the whole step (append + router + attention) in one
         # launch (srswa_step), unless unfused is asked for
-        self.fused_route = self.sparse and not self.fp8 and not w.get("rope") and not w.get("fp8_ring") and \
-            not w.get("unfused")
+        self.fused_route = self.sparse and not self.fp8 and not w.get("fp8_ring") and not w.get("unfused")
         if self.fp8:  # the stored cache: the bf16 prefix quantised once, by the library
             self.k8, self.v8, self.ks, self.vs = rswa.fp8_prefix_buffers(self.c.pk)
             rswa.rswa_quantize_prefix(self.c.pk, self.c.pv, self.c.prefix_len, self.k8, self.v8, self.ks, self.vs,
@@ -374,27 +381,40 @@ class Problem:
             del pl
         torch.cuda.synchronize()
 
-    def step(self, i: int, q=None, k_new=None, v_new=None, ev=None):
-        """Launches one decode step (1 to 3 kernels) on the current stream; returns the launch count."""
+    def step(self, i: int, q=None, k_new=None, v_new=None, ev=None, pos=None):
+        """Launches one decode step (1 to 3 kernels) on the current stream; returns the launch count.
+        pos: this step's (tok_pos, page) for the encoding configs (default: the device-resident ones)."""
         c, r = self.c, self.rswa
         q = c.q[i] if q is None else q
         k_new = c.k_new[i] if k_new is None else k_new
         v_new = c.v_new[i] if v_new is None else v_new
+        if self.rope:
+            tok, page = pos if pos is not None else (self.tok[i % self.tok.shape[0]], self.page[i % self.page.shape[0]])
         if self.fused_route:
             if ev is not None:
                 ev[0].record()
-            r.srswa_step(q, k_new, v_new, self.q_idx[i % self.n_dirs], self.kbar, c.pk, c.pv, c.prefix_len, c.ring_k,
-                         c.ring_v, c.wp, c.fill, self.blk, self.logp, self.out, self.ws, lse=self.lse, scale=c.scale)
+            if self.rope:
+                r.srswa_step_rope(q, k_new, v_new, self.q_idx[i % self.n_dirs], self.kbar, c.pk, c.pv, c.prefix_len,
+                                  c.ring_k, c.ring_v, c.wp, c.fill, tok, page, self.blk, self.logp, self.out, self.ws,
+                                  lse=self.lse, scale=c.scale)
+            else:
+                r.srswa_step(q, k_new, v_new, self.q_idx[i % self.n_dirs], self.kbar, c.pk, c.pv, c.prefix_len,
+                             c.ring_k, c.ring_v, c.wp, c.fill, self.blk, self.logp, self.out, self.ws, lse=self.lse,
+                             scale=c.scale)
             if ev is not None:
                 ev[1].record()
             return 1
-        if not self.fp8 and not self.sparse:
-            # R-SWA over a bf16 prefix: the fused step (ring append inside the decode launch),
-            # measured faster there; the SR-SWA steps keep append + route + decode
+        if not self.fp8 and not self.sparse and not (self.rope and self.w.get("unfused")):
+            # R-SWA over a bf16 prefix: the fused step (ring append, and the encoding when asked
+            # for, inside the decode launch), measured faster there
             if ev is not None:
                 ev[0].record()
-            r.rswa_decode_append(q, k_new, v_new, c.pk, c.pv, c.prefix_len, c.ring_k, c.ring_v, c.wp, c.fill,
-                                 self.out, self.ws, lse=self.lse, scale=c.scale)
+            if self.rope:
+                r.rswa_decode_append_rope(q, k_new, v_new, c.pk, c.pv, c.prefix_len, c.ring_k, c.ring_v, c.wp,
+                                          c.fill, tok, page, self.out, self.ws, lse=self.lse, scale=c.scale)
+            else:
+                r.rswa_decode_append(q, k_new, v_new, c.pk, c.pv, c.prefix_len, c.ring_k, c.ring_v, c.wp, c.fill,
+                                     self.out, self.ws, lse=self.lse, scale=c.scale)
             if ev is not None:
                 ev[1].record()
             return 1
@@ -421,8 +441,8 @@ class Problem:
         if self.rope:
             if ev is not None:
                 ev[4].record()
-            q = r.rswa_append_rope(c.ring_k, c.ring_v, k_new, v_new, c.wp, c.fill, q, self.tok[i % self.tok.shape[0]],
-                                   self.page[i % self.page.shape[0]], q_out=self.q_rot, status=self.ws)
+            q = r.rswa_append_rope(c.ring_k, c.ring_v, k_new, v_new, c.wp, c.fill, q, tok, page, q_out=self.q_rot,
+                                   status=self.ws)
             if ev is not None:
                 ev[5].record()
         else:
@@ -589,7 +609,7 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     ms_total = start.elapsed_time(end)
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     route_ms = [e[2].elapsed_time(e[3]) for e in evs] if prob.sparse and not prob.fused_route else []
-    rope_ms = [e[4].elapsed_time(e[5]) for e in evs] if prob.rope else []
+    rope_ms = [e[4].elapsed_time(e[5]) for e in evs] if prob.rope and w.get("unfused") else []
     ms_max = max_over_ranks(world, ms_total)
     del graph
 
@@ -606,6 +626,8 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
     if not prob.fp8 and (not prob.sparse or prob.fused_route):
         # the fused step also writes this step's K and V row into the ring
         nbytes["attn"] += w["B"] * w["H"] * 512
+        if prob.rope:  # and reads the step's two int32 positions per sequence
+            nbytes["attn"] += w["B"] * 8
     if prob.fused_route:  # one kernel moves the router's bytes too
         nbytes = dict(attn=nbytes["attn"] + nbytes["route"], route=0)
     attn_avg_s = statistics.mean(attn_ms) / 1e3
@@ -645,7 +667,9 @@ def run_ours(args, w: dict, world: int, rank: int, local: int) -> dict:
                                                 "the router fused" if prob.fused_route else
                                                 ("srswa decode_kernel<true" if prob.sparse else "rswa decode_kernel<false")
                                                 + (", fp8>" if prob.fp8 else (", bf16>" if prob.sparse else
-                                                                              ", bf16> with the fused ring append"))),
+                                                                              ", bf16> with the fused ring append")))
+                                               + (", the page2d encoding inside" if prob.rope and not w.get("unfused")
+                                                  else ""),
                      "achieved": achieved,
                      "peak": peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
@@ -922,11 +946,20 @@ def run_e2e(prob: Problem, K: int, W: int) -> dict:
     hlse = torch.empty((B, H), dtype=torch.float32, pin_memory=True)
     stream = torch.cuda.Stream()
 
+    if prob.rope:  # the step's token positions come from the host too
+        hpos = [torch.empty((2, B), dtype=torch.int32, pin_memory=True) for _ in range(pool)]
+        for j in range(pool):
+            hpos[j][0].copy_(prob.tok[j % prob.tok.shape[0]])
+            hpos[j][1].copy_(prob.page[j % prob.page.shape[0]])
+        dpos = torch.empty((2, B), dtype=torch.int32, device="cuda")
+
     def one(j):
         dq.copy_(hq[j % pool], non_blocking=True)
         dk.copy_(hk[j % pool], non_blocking=True)
         dv.copy_(hv[j % pool], non_blocking=True)
-        prob.step(0, q=dq, k_new=dk, v_new=dv)
+        if prob.rope:
+            dpos.copy_(hpos[j % pool], non_blocking=True)
+        prob.step(0, q=dq, k_new=dk, v_new=dv, pos=(dpos[0], dpos[1]) if prob.rope else None)
         hout.copy_(prob.out, non_blocking=True)
         hlse.copy_(prob.lse, non_blocking=True)
 
@@ -941,7 +974,7 @@ def run_e2e(prob: Problem, K: int, W: int) -> dict:
             one(j)
         e.record()
     e.synchronize()
-    h2d = 3 * B * H * D * 2
+    h2d = 3 * B * H * D * 2 + (2 * B * 4 if prob.rope else 0)
     d2h = B * H * D * 4 + B * H * 4
     return {"ms": s.elapsed_time(e), "h2d": h2d, "d2h": d2h}
 
@@ -1180,7 +1213,7 @@ def run_reference(args, w: dict) -> dict:
         unit = "prefill chunks/s"
         what = f"1 of {w['B']} sequences, {len(st['rows'])} of {w['T']} query rows per step (all heads)"
     else:
-        sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2, 10: 2, 11: 8, 12: 2}.get(args.config, 1))
+        sample = min(w["B"], {1: 1, 2: 8, 4: 2, 5: 1, 6: 8, 7: 2, 10: 2, 11: 8, 12: 2, 13: 8}.get(args.config, 1))
         st = oracle_sample_step(w, sample, seed=99)
         step = lambda: oracle_step(st, w)  # noqa: E731
         frac = sample / w["B"]
@@ -1281,7 +1314,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=None, choices=list(range(1, 13)),
+    ap.add_argument("--config", type=int, default=None, choices=list(range(1, 14)),
                     help="the workload (default 2, which also runs configs 1, 3, 4, 5 into `configs`)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

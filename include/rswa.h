@@ -90,7 +90,8 @@ RSWA_API const char* rswa_last_error(void);
  * FP8 prefix, the fused decode step and the SR-SWA chunked prefill to version 1; 3 adds
  * the page2d rotary encoding (rswa_rope_page2d, rswa_append_rope); 4 the FP8 ring
  * (rswa_append_fp8, rswa_decode_fp8kv, srswa_decode_fp8kv), the fused router
- * (srswa_decode_routed, srswa_step) and the wait-timeout test hook. */
+ * (srswa_decode_routed, srswa_step) and the wait-timeout test hook; 5 the fused steps
+ * with the page2d encoding (rswa_decode_append_rope, srswa_step_rope). */
 RSWA_API int32_t rswa_version(void);
 
 /*
@@ -494,8 +495,8 @@ RSWA_API rswa_status srswa_decode_fp8kv(const rswa_dims* dims, const void* q, co
  *   tok_pos, page : int32 [B] (this step's token positions), base, page_mod. q_out is
  *   written whatever the ring state; a sequence with wp / fill out of range is flagged
  *   and its ring left untouched, as in rswa_append.
- * A decode step with the encoding: rswa_append_rope, then srswa_route + srswa_decode (or
- * rswa_decode) on q_out; or rswa_rope_page2d on q and k_new, then rswa_decode_append.
+ * A decode step with the encoding: rswa_decode_append_rope or srswa_step_rope (one launch,
+ * below); or rswa_append_rope, then srswa_route + srswa_decode (or rswa_decode) on q_out.
  */
 RSWA_API rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, const void* q, void* q_out,
                                       const void* k, void* k_out, const int32_t* tok_pos, const int32_t* page,
@@ -505,6 +506,42 @@ RSWA_API rswa_status rswa_append_rope(const rswa_dims* dims, void* ring_k, void*
                                       const void* v_new, int32_t* wp, int32_t* fill, int32_t* slot_out, const void* q,
                                       void* q_out, const int32_t* tok_pos, const int32_t* page, double base,
                                       int32_t page_mod, int32_t* status, void* stream);
+
+/*
+ * The fused decode steps with the page2d encoding inside the same launch: this step's
+ * query is encoded where the attention loads it, and its key where the step appends it
+ * (into ring slot wp[b] and into the step's key set); values are not encoded. Results are
+ * bit-identical to rswa_rope_page2d (or rswa_append_rope) on q and k_new followed by
+ * rswa_decode_append (resp. srswa_step) on the encoded rows: the same fp64 angles, the
+ * same f32 cos / sin and the same f32 rotation rounded to bf16. The router (srswa_step_rope)
+ * reads q_idx, which is not encoded.
+ *   rope : host pointer to an rswa_rope (read during the call only):
+ *          tok_pos, page : int32 device arrays [batch], this step's positions (any values;
+ *                          4-byte aligned, read on the device)
+ *          base          : finite > 0;  page_mod : >= 0 (as rswa_rope_page2d)
+ *   The other arguments, the workspace and the error behaviour are those of
+ *   rswa_decode_append (resp. srswa_step); head_dim 128. A sequence whose ring state is
+ *   out of range is flagged and not appended, and its query is still encoded.
+ */
+typedef struct rswa_rope {
+  const int32_t* tok_pos;
+  const int32_t* page;
+  double base;
+  int32_t page_mod;
+} rswa_rope;
+
+RSWA_API rswa_status rswa_decode_append_rope(const rswa_dims* dims, const rswa_rope* rope, const void* q,
+                                             const void* k_new, const void* v_new, const void* pk, const void* pv,
+                                             const int32_t* prefix_len, void* ring_k, void* ring_v, int32_t* wp,
+                                             int32_t* fill, int32_t* slot_out, float scale, float* out, float* lse,
+                                             void* workspace, size_t ws_bytes, void* stream);
+
+RSWA_API rswa_status srswa_step_rope(const rswa_dims* dims, const rswa_rope* rope, const void* q, const void* k_new,
+                                     const void* v_new, const float* q_idx, const float* kbar, float idx_scale,
+                                     int32_t topk, const void* pk, const void* pv, const int32_t* prefix_len,
+                                     void* ring_k, void* ring_v, int32_t* wp, int32_t* fill, int32_t* slot_out,
+                                     float scale, int32_t* blk_idx, float* blk_logp, float* tau, float* out,
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -12,7 +12,7 @@ from .binding import (  # noqa: F401
     rswa_quantize_prefix, srswa_decode, srswa_decode_append, srswa_decode_fp8, srswa_index_pool, srswa_prefill,
     srswa_route,
     srswa_route_tokens, test_arm_wait_timeout, workspace_bytes, srswa_decode_routed, srswa_step,
-    srswa_prefill_workspace,
+    srswa_prefill_workspace, rswa_decode_append_rope, srswa_step_rope,
 )
 
 __all__ = ["load", "Dims", "RswaError", "rswa_append", "rswa_decode", "rswa_prefill", "srswa_index_pool", "srswa_route",
@@ -20,5 +20,5 @@ __all__ = ["load", "Dims", "RswaError", "rswa_append", "rswa_decode", "rswa_pref
            "srswa_route_tokens", "srswa_prefill", "rswa_decode_append", "srswa_decode_append",
            "rswa_rope_page2d", "rswa_append_rope", "rswa_append_fp8", "rswa_decode_fp8kv", "srswa_decode_fp8kv",
            "fp8_ring_buffers", "test_arm_wait_timeout", "srswa_decode_routed", "srswa_step",
-           "srswa_prefill_workspace",
+           "srswa_prefill_workspace", "rswa_decode_append_rope", "srswa_step_rope",
            "workspace_bytes", "new_workspace", "route_workspace", "check_status", "dims_of"]

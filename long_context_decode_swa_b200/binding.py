@@ -40,7 +40,7 @@ EXPORTED = ("rswa_last_error", "rswa_version", "rswa_workspace_bytes", "rswa_che
             "rswa_quantize_prefix", "rswa_decode_fp8", "srswa_decode_fp8", "srswa_route_tokens", "srswa_prefill",
             "rswa_decode_append", "srswa_decode_append", "rswa_rope_page2d", "rswa_append_rope", "rswa_append_fp8",
             "rswa_decode_fp8kv", "srswa_decode_fp8kv", "rswa_test_arm_wait_timeout", "srswa_decode_routed",
-            "srswa_step", "srswa_prefill_workspace_bytes")
+            "srswa_step", "srswa_prefill_workspace_bytes", "rswa_decode_append_rope", "srswa_step_rope")
 
 
 class RswaError(RuntimeError):
@@ -56,6 +56,12 @@ class Dims(ctypes.Structure):
     def __repr__(self):
         return (f"Dims(batch={self.batch}, heads={self.heads}, head_dim={self.head_dim}, ring={self.ring}, "
                 f"prefix_cap={self.prefix_cap})")
+
+
+class Rope(ctypes.Structure):
+    """rswa_rope: the page2d encoding of a fused decode step (device position arrays)."""
+    _fields_ = [("tok_pos", ctypes.c_void_p), ("page", ctypes.c_void_p), ("base", ctypes.c_double),
+                ("page_mod", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -82,6 +88,7 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(p)
         P, I32, I64, F32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
         DP = ctypes.POINTER(Dims)
+        RP = ctypes.POINTER(Rope)
         sig = {
             "rswa_last_error": ([], ctypes.c_char_p),
             "rswa_version": ([], I32),
@@ -93,6 +100,9 @@ def load(path: str | None = None):
             "srswa_step": ([DP, P, P, P, P, P, F32, I32, P, P, P, P, P, P, P, P, F32, P, P, P, P, P, P, SZ, P],
                            ctypes.c_int),
             "srswa_prefill_workspace_bytes": ([DP, I32], SZ),
+            "rswa_decode_append_rope": ([DP, RP, P, P, P, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
+            "srswa_step_rope": ([DP, RP, P, P, P, P, P, F32, I32, P, P, P, P, P, P, P, P, F32, P, P, P, P, P, P, SZ,
+                                 P], ctypes.c_int),
             "rswa_append": ([DP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "rswa_decode": ([DP, P, P, P, P, P, P, P, P, F32, P, P, P, SZ, P], ctypes.c_int),
             "srswa_index_pool": ([DP, P, P, P, P], ctypes.c_int),
@@ -547,6 +557,44 @@ def rswa_decode_append(q, k_new, v_new, pk, pv, prefix_len, ring_k, ring_v, wp, 
                                                            _stream(stream)))
 
 
+def _rope_arg(tok_pos, page, base, page_mod, B: int) -> Rope:
+    _want(tok_pos, "tok_pos", torch.int32, (B,))
+    _want(page, "page", torch.int32, (B,))
+    return Rope(_ptr(tok_pos), _ptr(page), float(base), int(page_mod))
+
+
+def rswa_decode_append_rope(q, k_new, v_new, pk, pv, prefix_len, ring_k, ring_v, wp, fill, tok_pos, page, out,
+                            workspace, lse=None, slot_out=None, base: float = 10000.0, page_mod: int = 2, scale=None,
+                            stream=None):
+    """rswa_decode_append with q and k_new page2d-encoded inside the same launch (tok_pos, page:
+    int32 [B], this step's positions)."""
+    B, H, cap, D = pk.shape
+    n = ring_k.shape[2]
+    _want(q, "q", torch.bfloat16, (B, H, D))
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    _want(pk, "pk", torch.bfloat16)
+    _want(pv, "pv", torch.bfloat16, pk.shape)
+    _want(prefix_len, "prefix_len", torch.int32, (B,))
+    _want(ring_k, "ring_k", torch.bfloat16, (B, H, n, D))
+    _want(ring_v, "ring_v", torch.bfloat16, (B, H, n, D))
+    _want(wp, "wp", torch.int32, (B,))
+    _want(fill, "fill", torch.int32, (B,))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    _want(out, "out", torch.float32, (B, H, D))
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (B, H))
+    _want(workspace, "workspace", torch.uint8)
+    rope = _rope_arg(tok_pos, page, base, page_mod, B)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("rswa_decode_append_rope", load().rswa_decode_append_rope(
+        ctypes.byref(dims), ctypes.byref(rope), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(pk), _ptr(pv),
+        _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp), _ptr(fill), _ptr(slot_out), scale, _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
 def srswa_decode_append(q, k_new, v_new, pk, pv, prefix_len, blk_idx, blk_logp, ring_k, ring_v, wp, fill, out,
                         workspace, lse=None, slot_out=None, scale=None, stream=None):
     """rswa_append + srswa_decode in one launch (same results; wp / fill / ring updated)."""
@@ -735,3 +783,25 @@ def srswa_step(q, k_new, v_new, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v,
         _ptr(pk), _ptr(pv), _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp), _ptr(fill), _ptr(slot_out), scale,
         _ptr(blk_idx), _ptr(blk_logp), _ptr(tau), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)))
+
+
+def srswa_step_rope(q, k_new, v_new, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, tok_pos, page,
+                    blk_idx, blk_logp, out, workspace, lse=None, tau=None, slot_out=None, base: float = 10000.0,
+                    page_mod: int = 2, idx_scale=1.0, scale=None, stream=None):
+    """srswa_step with q and k_new page2d-encoded inside the same launch (tok_pos, page: int32 [B],
+    this step's positions; the router's q_idx is not encoded). workspace: new_workspace(dims,
+    OP_SRSWA_ROUTED)."""
+    B, H, cap, D, n, topk = _want_routed(q, q_idx, kbar, pk, pv, prefix_len, ring_k, ring_v, wp, fill, blk_idx,
+                                         blk_logp, tau, out, lse, workspace)
+    _want(k_new, "k_new", torch.bfloat16, (B, H, D))
+    _want(v_new, "v_new", torch.bfloat16, (B, H, D))
+    if slot_out is not None:
+        _want(slot_out, "slot_out", torch.int32, (B,))
+    rope = _rope_arg(tok_pos, page, base, page_mod, B)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dims = Dims(B, H, D, n, cap)
+    _check("srswa_step_rope", load().srswa_step_rope(
+        ctypes.byref(dims), ctypes.byref(rope), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_idx), _ptr(kbar),
+        float(idx_scale), topk, _ptr(pk), _ptr(pv), _ptr(prefix_len), _ptr(ring_k), _ptr(ring_v), _ptr(wp),
+        _ptr(fill), _ptr(slot_out), scale, _ptr(blk_idx), _ptr(blk_logp), _ptr(tau), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel(), _stream(stream)))

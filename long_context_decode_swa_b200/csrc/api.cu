@@ -92,7 +92,7 @@ extern "C" {
 
 const char* rswa_last_error(void) { return g_last_error; }
 
-int32_t rswa_version(void) { return 4; }
+int32_t rswa_version(void) { return 5; }
 
 size_t rswa_workspace_bytes(const rswa_dims* dims, int32_t op) {
   const char* fn = "rswa_workspace_bytes";
@@ -224,8 +224,9 @@ struct AppendSrc {
   int32_t* wp;
   int32_t* fill;
   int32_t* slot_out;
+  const rswa_rope* rope;  // page2d encoding of this step's query and key, or null
 };
-constexpr AppendSrc kNoAppend{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+constexpr AppendSrc kNoAppend{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
 
 // An FP8 ring (codes + row scales) in place of the bf16 ring_k / ring_v.
 struct Ring8Src {
@@ -249,6 +250,15 @@ struct RouteSrc {
 };
 constexpr RouteSrc kNoRoute{nullptr, nullptr, 0.f, nullptr, nullptr, nullptr, false};
 constexpr size_t kGridCounterOffset = 128;  // an int32 inside the workspace's 256-byte status area
+
+// page2d rotary encoding: the checks shared by the entry points that encode.
+static rswa_status check_rope_params(const char* fn, const int32_t* tok_pos, const int32_t* page, double base,
+                                     int32_t page_mod) {
+  if (tok_pos == nullptr || page == nullptr) return fail(RSWA_ERR_INVALID, "%s: tok_pos and page must not be NULL", fn);
+  if (!(base > 0.0) || !std::isfinite(base)) return fail(RSWA_ERR_INVALID, "%s: base must be finite and > 0", fn);
+  if (page_mod < 0) return fail(RSWA_ERR_INVALID, "%s: page_mod must be >= 0 (got %d)", fn, page_mod);
+  return RSWA_OK;
+}
 
 // plan_budget > 0: plan the split-KV work to fit a workspace of that many bytes.
 static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* dims, const void* q, PrefixSrc px,
@@ -315,6 +325,10 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
     const void* v_new = app.v_new;
     REQUIRE_PTR(k_new);
     REQUIRE_PTR(v_new);
+    if (app.rope != nullptr) {
+      st = check_rope_params(fn, app.rope->tok_pos, app.rope->page, app.rope->base, app.rope->page_mod);
+      if (st != RSWA_OK) return st;
+    }
   }
   if (sparse) {
     if (blk_idx == nullptr || blk_logp == nullptr)
@@ -398,6 +412,10 @@ static rswa_status decode_common(const char* fn, bool sparse, const rswa_dims* d
   a.wp_w = app.wp;
   a.fill_w = app.fill;
   a.slot_out = app.slot_out;
+  a.rope_tok = app.rope ? app.rope->tok_pos : nullptr;
+  a.rope_page = app.rope ? app.rope->page : nullptr;
+  a.rope_log2_base = app.rope ? std::log2(app.rope->base) : 0.0;
+  a.rope_page_mod = app.rope ? app.rope->page_mod : 0;
   a.grid_counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kGridCounterOffset);
   a.prefix_len = prefix_len;
   a.ring_k = static_cast<const uint16_t*>(ring_k);
@@ -542,15 +560,6 @@ rswa_status rswa_quantize_prefix(const rswa_dims* dims, const void* pk, const vo
   return ok();
 }
 
-// page2d rotary encoding: the checks shared by both entry points.
-static rswa_status check_rope_params(const char* fn, const int32_t* tok_pos, const int32_t* page, double base,
-                                     int32_t page_mod) {
-  if (tok_pos == nullptr || page == nullptr) return fail(RSWA_ERR_INVALID, "%s: tok_pos and page must not be NULL", fn);
-  if (!(base > 0.0) || !std::isfinite(base)) return fail(RSWA_ERR_INVALID, "%s: base must be finite and > 0", fn);
-  if (page_mod < 0) return fail(RSWA_ERR_INVALID, "%s: page_mod must be >= 0 (got %d)", fn, page_mod);
-  return RSWA_OK;
-}
-
 rswa_status rswa_rope_page2d(int64_t rows, int32_t heads, int32_t head_dim, const void* q, void* q_out, const void* k,
                              void* k_out, const int32_t* tok_pos, const int32_t* page, double base, int32_t page_mod,
                              void* stream) {
@@ -619,8 +628,8 @@ rswa_status rswa_decode_append(const rswa_dims* dims, const void* q, const void*
   if (k_new == nullptr || v_new == nullptr)
     return fail(RSWA_ERR_INVALID, "rswa_decode_append: k_new and v_new must not be NULL");
   return decode_common("rswa_decode_append", false, dims, q, bf16_prefix(pk, pv), kNoBand,
-                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, nullptr, nullptr, 0,
-                       ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out, nullptr}, prefix_len, nullptr,
+                       nullptr, 0, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
 rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, const void* k_new, const void* v_new,
@@ -631,8 +640,8 @@ rswa_status srswa_decode_append(const rswa_dims* dims, const void* q, const void
   if (k_new == nullptr || v_new == nullptr)
     return fail(RSWA_ERR_INVALID, "srswa_decode_append: k_new and v_new must not be NULL");
   return decode_common("srswa_decode_append", true, dims, q, bf16_prefix(pk, pv), kNoBand,
-                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, blk_idx, blk_logp,
-                       topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out, nullptr}, prefix_len, blk_idx,
+                       blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
 }
 
 rswa_status srswa_decode_routed(const rswa_dims* dims, const void* q, const float* q_idx, const float* kbar,
@@ -652,9 +661,37 @@ rswa_status srswa_step(const rswa_dims* dims, const void* q, const void* k_new, 
                        float* lse, void* workspace, size_t ws_bytes, void* stream) {
   if (k_new == nullptr || v_new == nullptr) return fail(RSWA_ERR_INVALID, "srswa_step: k_new and v_new must not be NULL");
   return decode_common("srswa_step", true, dims, q, bf16_prefix(pk, pv), kNoBand,
-                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out}, prefix_len, blk_idx, blk_logp,
-                       topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream, 0, kNoRing8,
-                       RouteSrc{q_idx, kbar, idx_scale, blk_idx, blk_logp, tau, true});
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out, nullptr}, prefix_len, blk_idx,
+                       blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream, 0,
+                       kNoRing8, RouteSrc{q_idx, kbar, idx_scale, blk_idx, blk_logp, tau, true});
+}
+
+rswa_status rswa_decode_append_rope(const rswa_dims* dims, const rswa_rope* rope, const void* q, const void* k_new,
+                                    const void* v_new, const void* pk, const void* pv, const int32_t* prefix_len,
+                                    void* ring_k, void* ring_v, int32_t* wp, int32_t* fill, int32_t* slot_out,
+                                    float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  const char* fn = "rswa_decode_append_rope";
+  if (rope == nullptr) return fail(RSWA_ERR_INVALID, "%s: rope must not be NULL", fn);
+  if (k_new == nullptr || v_new == nullptr) return fail(RSWA_ERR_INVALID, "%s: k_new and v_new must not be NULL", fn);
+  return decode_common(fn, false, dims, q, bf16_prefix(pk, pv), kNoBand,
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out, rope}, prefix_len, nullptr, nullptr,
+                       0, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream);
+}
+
+rswa_status srswa_step_rope(const rswa_dims* dims, const rswa_rope* rope, const void* q, const void* k_new,
+                            const void* v_new, const float* q_idx, const float* kbar, float idx_scale, int32_t topk,
+                            const void* pk, const void* pv, const int32_t* prefix_len, void* ring_k, void* ring_v,
+                            int32_t* wp, int32_t* fill, int32_t* slot_out, float scale, int32_t* blk_idx,
+                            float* blk_logp, float* tau, float* out, float* lse, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  const char* fn = "srswa_step_rope";
+  if (rope == nullptr) return fail(RSWA_ERR_INVALID, "%s: rope must not be NULL", fn);
+  if (k_new == nullptr || v_new == nullptr) return fail(RSWA_ERR_INVALID, "%s: k_new and v_new must not be NULL", fn);
+  return decode_common(fn, true, dims, q, bf16_prefix(pk, pv), kNoBand,
+                       AppendSrc{k_new, v_new, ring_k, ring_v, wp, fill, slot_out, rope}, prefix_len, blk_idx,
+                       blk_logp, topk, ring_k, ring_v, wp, fill, scale, out, lse, workspace, ws_bytes, stream, 0,
+                       kNoRing8, RouteSrc{q_idx, kbar, idx_scale, blk_idx, blk_logp, tau, true});
 }
 
 rswa_status rswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const void* k_out, const void* v_out,

@@ -34,6 +34,7 @@
 // is read as a one-row tile and written into its ring slot inside the launch, whose last
 // CTA advances wp / fill); and the SR-SWA chunked prefill (items are single queries of a
 // chunk, whose key sets end with their causal band of the chunk's outputs).
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -77,6 +78,8 @@ struct DecodeSmem {
   int fin_redi[kWarps];
   int fin_n;
   int fin_ok;
+  // page2d encoding in the fused step: the 64 pair frequencies base^(-i/64), fp64
+  double rope_th[kHeadDim / 2];
 };
 
 constexpr int kDecodeMinBlocks =
@@ -329,6 +332,7 @@ struct ItemView {
   int t0;
   int b;
   bool routed;  // (c, lp) hold the route (fused router: read once the route is published)
+  int rope_tok, rope_pg;  // fused step with the page2d encoding: the sequence's positions
   SeqView v;
   int c;
   float lp;
@@ -343,6 +347,10 @@ __device__ __forceinline__ void load_item(const DecodeArgs& a, int item, int lan
   iv.item = item;
   iv.t0 = split * a.tiles_per_item;
   iv.b = b;
+  if (mode_appends(kMode) && a.rope_tok != nullptr && split == 0) {  // loaded beside the view's reads
+    iv.rope_tok = a.rope_tok[b];
+    iv.rope_pg = a.rope_page[b];
+  }
   iv.v = make_view<kSparse, kFp8, kMode>(a, b, h, i, lane == 0 && split == 0 && h == 0 && i == 0);
   iv.c = -1;
   iv.lp = -INFINITY;
@@ -377,6 +385,59 @@ __device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
 // observed, e.g. its warp's or CTA's writes before a barrier), then a relaxed atomic add.
 __device__ __forceinline__ void red_release_gpu(int32_t* p, int v) {
   asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// page2d rotary encoding of this step's query and key rows inside the fused step
+// (Unlimited-OCR-2 SR-SWA explainer, 2D 位置编码; constants as read for rswa_rope_page2d:
+// pair i couples dims i and i + 64 and turns by pos * base^(-i/64), pos = the page number
+// when i mod page_mod == page_mod - 1, else the token position; th[i] = base^(-i/64) from
+// the CTA's table). Warp-collective: lane l
+// takes the fp64 angles and sincos of pairs 2l and 2l + 1, and every lane then gathers the
+// cos / sin (rounded to f32) of the eight pairs its 16-byte chunk c = lane & 15 touches,
+// pairs 8 (c & 7) + e: the same values, and the same rotation arithmetic below, as the
+// stand-alone encoding kernels, so the fused step gives their results bit for bit.
+__device__ __forceinline__ void rope_lane_cos_sin(const DecodeArgs& a, const double* th, int tok, int pg, int lane,
+                                                  float2 (&cs)[8]) {
+  float2 mine[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = 2 * lane + u;
+    const bool on_page = a.rope_page_mod > 0 && i % a.rope_page_mod == a.rope_page_mod - 1;
+    double s, c;
+    sincos((double)(on_page ? pg : tok) * th[i], &s, &c);
+    mine[u] = make_float2((float)c, (float)s);
+  }
+  const int src = 4 * (lane & 7);  // lane holding pairs 8 (c & 7) + 0, 1
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    cs[e].x = __shfl_sync(0xffffffffu, mine[e & 1].x, src + (e >> 1));
+    cs[e].y = __shfl_sync(0xffffffffu, mine[e & 1].y, src + (e >> 1));
+  }
+}
+
+// Rotates the 16-byte chunk w (dims 8c..8c+7, c = lane & 15, of a row spread over a half
+// warp) with its partner chunk c ^ 8, rounding to bf16. Warp-collective (every lane
+// shuffles); lanes with rotate == false keep w.
+__device__ __forceinline__ uint4 rope_rotate_chunk(uint4 w, const float2 (&cs)[8], int lane, bool rotate) {
+  uint32_t own[4] = {w.x, w.y, w.z, w.w};
+  uint32_t other[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) other[k] = __shfl_xor_sync(0xffffffffu, own[k], 8);
+  if (!rotate) return w;
+  const bool first_half = (lane & 8) == 0;  // dims below 64: x of y_i = x_i cos - x_{i+64} sin
+  uint32_t r[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t lo = first_half ? own[k] : other[k];  // dims i (8 (c & 7) + 2k, + 1)
+    const uint32_t hi = first_half ? other[k] : own[k];  // dims i + 64
+    const float2 a0 = cs[2 * k], a1 = cs[2 * k + 1];
+    const float x0 = bf16lo(lo), x1 = bf16hi(lo), y0 = bf16lo(hi), y1 = bf16hi(hi);
+    const __nv_bfloat162 v = first_half
+        ? __floats2bfloat162_rn(fmaf(x0, a0.x, -y0 * a0.y), fmaf(x1, a1.x, -y1 * a1.y))
+        : __floats2bfloat162_rn(fmaf(y0, a0.x, x0 * a0.y), fmaf(y1, a1.x, x1 * a1.y));
+    r[k] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 // Fused router: waits (bounded) until the route of the item's sequence is published, then
@@ -445,10 +506,25 @@ __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& 
   const int c = __shfl_sync(0xffffffffu, iv.c, ridx & 31);
   const float lp = __shfl_sync(0xffffffffu, iv.lp, ridx & 31);
   const TileRef r = tile_at<kSparse, kFp8, kMode>(iv.v, tile, c, lp, lane == 0 ? a.status : nullptr);
+  const bool rope_key = mode_appends(kMode) && r.blk == -2 && a.rope_tok != nullptr;
   if (r.blk == -2) {  // fused append: the warp writes this step's row into its ring slot
     const uint4* src = reinterpret_cast<const uint4*>(lane < 16 ? iv.v.nk : iv.v.nv);
     uint4* dst = reinterpret_cast<uint4*>(lane < 16 ? iv.v.wk : iv.v.wv);
-    dst[lane & 15] = src[lane & 15];
+    uint4 w = src[lane & 15];
+    if (rope_key) {
+      // the key is encoded on its way: lanes 0-15 rotate it, write it into the ring slot and
+      // into the stage themselves (its bulk copy is left out below; V is copied as usual)
+      float2 cs[8];
+      rope_lane_cos_sin(a, sm.rope_th, iv.rope_tok, iv.rope_pg, lane, cs);
+      w = rope_rotate_chunk(w, cs, lane, lane < 16);
+      if (lane < 16) {
+        reinterpret_cast<uint4*>(sm.stage[s][0])[lane] = w;
+        // ordered before the bulk copy that refills this stage after the tile is read
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      __syncwarp();
+    }
+    dst[lane & 15] = w;
     if (lane == 0 && iv.v.slot_out) *iv.v.slot_out = iv.v.wslot;
   }
   f.rows = r.rows;
@@ -471,7 +547,7 @@ __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& 
   f.armed = r.rows > 0;
   if (r.rows > 0 && lane == 0) {
     const uint32_t bytes = (uint32_t)r.rows * (f.fp8 ? (uint32_t)kHeadDim : (uint32_t)kRowBytes);
-    mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+    mbar_arrive_expect_tx(&sm.full[s], rope_key ? bytes : 2 * bytes);  // an encoded key is in the stage already
     if (kSparse && r.blk >= 0) {
       // routed blocks change from step to step: mark them first to leave L2, so the ring,
       // which every step reads again, stays there (measured: 32K-history attention
@@ -481,7 +557,7 @@ __device__ __forceinline__ InFlight issue_tile(const DecodeArgs& a, DecodeSmem& 
       bulk_copy_g2s_stream(sm.stage[s][0], r.k, bytes, &sm.full[s], pol);
       bulk_copy_g2s_stream(sm.stage[s][1], r.v, bytes, &sm.full[s], pol);
     } else {
-      bulk_copy_g2s(sm.stage[s][0], r.k, bytes, &sm.full[s]);
+      if (!rope_key) bulk_copy_g2s(sm.stage[s][0], r.k, bytes, &sm.full[s]);
       bulk_copy_g2s(sm.stage[s][1], r.v, bytes, &sm.full[s]);
     }
   }
@@ -1022,6 +1098,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
     fence_mbar_init();
   }
+  if constexpr (mode_appends(kMode)) {
+    if (a.rope_tok != nullptr && tid < kHeadDim / 2)
+      sm.rope_th[tid] = exp2(-(2.0 * tid / kHeadDim) * a.rope_log2_base);
+  }
   __syncthreads();
   griddep_wait();               // inputs may be written by the previous kernel in the stream
   griddep_launch_dependents();  // the next kernel may start its prologue
@@ -1068,15 +1148,35 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeMinBlocks) decode_kerne
   const int g = lane >> 4, c = lane & 15;
   // the next item's query is loaded while the current item streams
   uint4 q_next = make_uint4(0, 0, 0, 0);
-  if (blockIdx.x < a.items)
+  int2 pos_next = make_int2(0, 0);  // fused step with the encoding: the next item's positions
+  const bool rope_q = mode_appends(kMode) && a.rope_tok != nullptr;
+  if (blockIdx.x < a.items) {
     q_next = *reinterpret_cast<const uint4*>(a.q + (int64_t)(blockIdx.x / a.splits) * kHeadDim + c * 8);
+    if (rope_q) {
+      const int bn = (int)blockIdx.x / a.splits / a.H;
+      pos_next = make_int2(a.rope_tok[bn], a.rope_page[bn]);
+    }
+  }
   int li_base = 0;
   for (int item = blockIdx.x; item < a.items; item += gridDim.x, li_base += P) {
     // vq: the item's query, (b * H + h) * T + i; q, out, lse and the split partials are per query
     const int vq = item / a.splits, split = item - vq * a.splits;
-    const uint4 q_cur = q_next;
-    if (item + (int)gridDim.x < a.items)
+    uint4 q_cur = q_next;
+    const int2 pos_cur = pos_next;
+    if (item + (int)gridDim.x < a.items) {
       q_next = *reinterpret_cast<const uint4*>(a.q + (int64_t)((item + gridDim.x) / a.splits) * kHeadDim + c * 8);
+      if (rope_q) {
+        const int bn = (item + (int)gridDim.x) / a.splits / a.H;
+        pos_next = make_int2(a.rope_tok[bn], a.rope_page[bn]);
+      }
+    }
+    if constexpr (mode_appends(kMode)) {
+      if (rope_q) {  // the query encoded at its sequence's position (one query per item)
+        float2 cs[8];
+        rope_lane_cos_sin(a, sm.rope_th, pos_cur.x, pos_cur.y, lane, cs);
+        q_cur = rope_rotate_chunk(q_cur, cs, lane, true);
+      }
+    }
     float2 q2[4];
     {
       const uint32_t ws[4] = {q_cur.x, q_cur.y, q_cur.z, q_cur.w};

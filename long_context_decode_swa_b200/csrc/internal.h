@@ -54,6 +54,13 @@ struct DecodeArgs {
   int32_t* fill_w;
   int32_t* slot_out;
   int32_t* grid_counter;
+  // page2d rotary encoding inside the fused append (null rope_tok: none): this step's query
+  // and key rows of sequence b are encoded at positions (rope_tok[b], rope_page[b]) on the
+  // way into the attention (the query) and into the ring slot and the key set (the key)
+  const int32_t* rope_tok;
+  const int32_t* rope_page;
+  double rope_log2_base;
+  int rope_page_mod;
   // FP8 ring (decode only): E4M3 code rows [B][H][n][D] with one f32 scale per row [B][H][n]
   // for K and for V, in place of ring_k / ring_v (which are then null)
   const uint8_t* ring_k8;

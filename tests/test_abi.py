@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     lib = rswa.load()
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.rswa_version() == 4
+    assert lib.rswa_version() == 5
 
 
 def _err():
@@ -262,3 +262,38 @@ def test_fused_router_entry_points_validation():
                               slot_out, ctypes.c_float(0.088), A, A, None, A, None, A, ctypes.c_size_t(ws), None)
 
     assert step(k_new=None) == INVALID and "k_new" in _err()
+
+
+def test_fused_steps_with_encoding_validation():
+    from long_context_decode_swa_b200.binding import Rope
+    lib = rswa.load()
+    d = Dims(2, 4, 128, 128, 64 * 32)
+    ws_dec = lib.rswa_workspace_bytes(ctypes.byref(d), 1)
+    ws_step = lib.rswa_workspace_bytes(ctypes.byref(d), 5)
+
+    def dec(rope=True, tok=A, page=A2, base=1e4, page_mod=2, k_new=A, ws_bytes=ws_dec):
+        r = Rope(tok, page, base, page_mod)
+        return lib.rswa_decode_append_rope(ctypes.byref(d), ctypes.byref(r) if rope else None, A, k_new, A, A, A, A,
+                                           A, A, A, A, None, ctypes.c_float(0.088), A, None, A,
+                                           ctypes.c_size_t(ws_bytes), None)
+
+    assert dec(rope=False) == INVALID and "rope" in _err()
+    assert dec(tok=None) == INVALID and "tok_pos" in _err()
+    assert dec(page=None) == INVALID and "page" in _err()
+    assert dec(base=0.0) == INVALID and "base" in _err()
+    assert dec(base=float("nan")) == INVALID and "base" in _err()
+    assert dec(page_mod=-1) == INVALID and "page_mod" in _err()
+    assert dec(k_new=None) == INVALID and "k_new" in _err()
+    assert dec(ws_bytes=255) == INVALID and "workspace" in _err()
+
+    def step(rope=True, tok=A, base=1e4, page_mod=2, q_idx=A, ws_bytes=ws_step):  # the size check needs a GPU
+        r = Rope(tok, A2, base, page_mod)
+        return lib.srswa_step_rope(ctypes.byref(d), ctypes.byref(r) if rope else None, A, A, A, q_idx, A,
+                                   ctypes.c_float(1.0), 16, A, A, A, A, A, A, A, None, ctypes.c_float(0.088), A, A,
+                                   None, A, None, A, ctypes.c_size_t(ws_bytes), None)
+
+    assert step(rope=False) == INVALID and "rope" in _err()
+    assert step(tok=None) == INVALID and "tok_pos" in _err()
+    assert step(base=-3.0) == INVALID and "base" in _err()
+    assert step(page_mod=-5) == INVALID and "page_mod" in _err()
+    assert step(q_idx=None) == INVALID and "q_idx" in _err()

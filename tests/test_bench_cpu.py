@@ -13,7 +13,7 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-@pytest.mark.parametrize("cfg", list(range(1, 13)))
+@pytest.mark.parametrize("cfg", list(range(1, 14)))
 def test_workloads_are_complete(cfg):
     w = bench.workload(cfg)
     for key in ("kind", "B", "H", "D", "n", "plen", "cap", "name"):
