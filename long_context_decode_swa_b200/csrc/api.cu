@@ -875,6 +875,7 @@ rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const
     return fail(RSWA_ERR_INVALID, "%s: workspace of %zu bytes is smaller than the %zu required "
                 "(srswa_prefill_workspace_bytes)", fn, ws_bytes, need);
   // workspace: [status 256 B][counts 256 B][group records][query lists][sorted routes][biases][lse of the band part]
+  // [sort keys]
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t bt = (size_t)dims->batch * T;
   int32_t* counts = reinterpret_cast<int32_t*>(ws + 256);
@@ -883,6 +884,8 @@ rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const
   int32_t* gblk = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(gq) + align256(bt * 4));
   float* gbias = reinterpret_cast<float*>(gblk + bt * rswa::kMaxTopk);
   float* lse_scratch = gbias + bt * rswa::kMaxTopk;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(lse_scratch) +
+                                               align256((size_t)dims->batch * dims->heads * T * 4));
   float* lse_use = lse != nullptr ? lse : lse_scratch;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // 1. group the chunk's queries by routed block set
@@ -892,7 +895,7 @@ rswa_status srswa_prefill(const rswa_dims* dims, int32_t T, const void* q, const
     e = cudaMemsetAsync(counts, 0, 16, s);
     if (e != cudaSuccess) return cuda_fail(e, "srswa_prefill: clearing the group counters");
     e = rswa::launch_srswa_group(dims->batch, T, topk, dims->prefix_cap, prefix_len, blk_idx, blk_logp, rec, gq,
-                                 gblk, gbias, counts, ws_status(workspace), s);
+                                 gblk, gbias, counts, keys, ws_status(workspace), s);
     if (e != cudaSuccess) return cuda_fail(e, "srswa_prefill: grouping");
   }
   // 2. the band (and previous-chunk ring) part of every query: the dense tcgen05 prefill, prefix left out

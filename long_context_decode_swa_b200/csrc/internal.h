@@ -172,7 +172,7 @@ size_t srswa_prefill_scratch_bytes(int B, int H, int T);
 int srswa_prefill_group_rec_ints();
 cudaError_t launch_srswa_group(int B, int T, int topk, int64_t cap, const int32_t* prefix_len, const int32_t* blk,
                                const float* logp, int32_t* rec, int32_t* gq, int32_t* gblk, float* gbias,
-                               int32_t* counts, int32_t* status, cudaStream_t stream);
+                               int32_t* counts, uint64_t* keys, int32_t* status, cudaStream_t stream);
 cudaError_t launch_srswa_routed(int B, int H, int T, int topk, int64_t cap, const int32_t* prefix_len, const void* q,
                                 const void* pk, const void* pv, const int32_t* rec, const int32_t* gq,
                                 const float* gbias, const int32_t* counts, float scale, float* out, float* lse,

@@ -535,6 +535,298 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Per-token router of the chunked prefill (T router queries per sequence, at most 1024
+// blocks): the same result as route_kernel row by row (the same z arithmetic; the same
+// sort-based threshold whenever at most 32 blocks are candidates), organised for many rows
+// that share one sequence's block keys. A CTA takes one sequence and a run of its tokens:
+// it stages the sequence's keys in shared memory once (bulk copies on an mbarrier), and each
+// warp routes two tokens at a time from there: both rows' scores come from the same key
+// loads (the octet layout of route_kernel), go to the warp's two score rows in shared
+// memory, and each row is then finished by the warp alone, without block barriers:
+//   * max z and the candidate count (z > max z - 2) by warp reductions;
+//   * at most 32 candidates (the usual case): compacted by ballots, sorted by one warp
+//     bitonic network (larger score first, ties to the smaller block), the threshold by the
+//     sort-based rule over a warp scan; the top-k is the front of that list, completed, when
+//     fewer than k blocks are candidates, by argmax rounds over the rest of the row;
+//   * more than 32 candidates: the root of sum (y - tau)_+^2 = 1 (y = z/2 - max z/2) is
+//     bracketed by bisection on [-1, 0], the support is {y > the bracket's low end}, and tau
+//     is the closed form over that support (the value the sort-based rule reaches); the top-k
+//     comes from argmax rounds.
+// ---------------------------------------------------------------------------------------
+constexpr int kTokWarps = 12;
+constexpr int kTokThreads = kTokWarps * 32;
+constexpr int kTokMaxBlocks = 1024;       // 32 scores per lane per row
+constexpr uint32_t kTokCopyBytes = 32768;  // bulk copies of the keys in pieces of this size
+
+__host__ __device__ __forceinline__ int tok_padded_blocks(int nb_cap) { return (nb_cap + 63) / 64 * 64; }
+
+__host__ __device__ __forceinline__ size_t tok_smem_bytes(int nb_cap) {
+  const size_t nbr = (size_t)tok_padded_blocks(nb_cap);
+  return nbr * kIndexDim * 4 + (size_t)kTokWarps * 2 * nbr * 4 + 16;
+}
+
+// Finishes one router row from its scores zs[0, NB) in shared memory (warp-collective; the
+// row's buffer is reused as scratch).
+__device__ void tok_finish_row(const RouteArgs& a, float* zs, int NB, int64_t row, int lane) {
+  float zr[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    const int c = lane + 32 * t;
+    zr[t] = c < NB ? zs[c] : -INFINITY;
+  }
+  float mx = zr[0];
+#pragma unroll
+  for (int t = 1; t < 32; ++t) mx = fmaxf(mx, zr[t]);
+  const float zmax = warp_max(mx);
+  const float cut = zmax - 2.f;  // candidates: z / 2 > max z / 2 - 1
+  int cnt = 0;
+#pragma unroll
+  for (int t = 0; t < 32; ++t) cnt += zr[t] > cut ? 1 : 0;
+  const int C = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);  // >= 1: the maximum
+  const float xmax = 0.5f * zmax;
+  __syncwarp();  // the row is in registers: its buffer now holds the candidate list
+  float* lz = zs;
+  int* li = reinterpret_cast<int*>(zs + 32);
+  float sz = -INFINITY;  // lane r: the r-th entry of the top list (best first)
+  int si = kNone;
+  int have = 0;          // entries of the top list already in place
+  float tau_y;
+  if (C <= 32) {
+    int base = 0;
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const bool in = zr[t] > cut;
+      const unsigned bal = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const int k = base + __popc(bal & lt);
+        lz[k] = zr[t];
+        li[k] = lane + 32 * t;
+      }
+      base += __popc(bal);
+    }
+    __syncwarp();
+    if (lane < C) {
+      sz = lz[lane];
+      si = li[lane];
+    }
+    warp_sort(sz, si, lane);
+    // sort-based rule: prefix sums of y and y^2 in rank order, tau_k per rank, support size =
+    // the largest k with delta_k >= 0 and tau_k < y_(k)
+    const float y = lane < C ? fmaf(sz, 0.5f, -xmax) : 0.f;
+    float s1 = y, s2 = y * y;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float t1 = __shfl_up_sync(0xffffffffu, s1, o), t2 = __shfl_up_sync(0xffffffffu, s2, o);
+      if (lane >= o) {
+        s1 += t1;
+        s2 += t2;
+      }
+    }
+    const float k = (float)(lane + 1);
+    const float mean = s1 / k;
+    const float delta = (1.f - (s2 - s1 * mean)) / k;
+    const float tk = mean - sqrtf(fmaxf(delta, 0.f));
+    const unsigned ok = __ballot_sync(0xffffffffu, lane < C && delta >= 0.f && tk < y);
+    const int best = ok ? 32 - __clz(ok) : 0;
+    const float tb = __shfl_sync(0xffffffffu, tk, best > 0 ? best - 1 : 0);
+    tau_y = best > 0 ? tb : 0.f;
+    have = C;
+  } else {
+    // f(tau) = sum (y - tau)_+^2 falls from f(-1) >= 1 (the maximum has y = 0) to f(0) = 0
+    float lo = -1.f, hi = 0.f;
+#pragma unroll 1
+    for (int it = 0; it < 30; ++it) {
+      const float mid = 0.5f * (lo + hi);
+      float f = 0.f;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const float d = fmaf(zr[t], 0.5f, -xmax) - mid;
+        f = d > 0.f ? fmaf(d, d, f) : f;
+      }
+      if (warp_sum(f) >= 1.f)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    float n = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const float y = fmaf(zr[t], 0.5f, -xmax);
+      if (y > lo) {
+        n += 1.f;
+        s1 += y;
+        s2 = fmaf(y, y, s2);
+      }
+    }
+    n = warp_sum(n);
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    const float mean = s1 / n;
+    const float delta = (1.f - (s2 - s1 * mean)) / n;
+    tau_y = mean - sqrtf(fmaxf(delta, 0.f));
+  }
+  if (have < a.topk) {
+    // argmax rounds: each takes the best entry ranking after the previous round's
+    float pz = have > 0 ? __shfl_sync(0xffffffffu, sz, have - 1) : INFINITY;
+    int pi = have > 0 ? __shfl_sync(0xffffffffu, si, have - 1) : -1;
+#pragma unroll 1
+    for (int r = have; r < a.topk; ++r) {
+      float bz = -INFINITY;
+      int bi = kNone;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const float z = zr[t];
+        const int i = lane + 32 * t;
+        const bool after = z < pz || (z == pz && i > pi);
+        if (after && i < NB && ranks_before(z, i, bz, bi)) {
+          bz = z;
+          bi = i;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ranks_before(oz, oi, bz, bi)) {
+          bz = oz;
+          bi = oi;
+        }
+      }
+      if (lane == r) {
+        sz = bz;
+        si = bi;
+      }
+      pz = bz;
+      pi = bi;
+    }
+  }
+  if (lane < a.topk) {
+    const int64_t o = row * a.topk + lane;
+    if (si == kNone) {
+      a.blk_idx[o] = -1;
+      a.blk_logp[o] = -INFINITY;
+    } else {
+      const float d = fmaf(sz, 0.5f, -xmax) - tau_y;
+      const float pr = d > 0.f ? d * d : 0.f;
+      a.blk_idx[o] = si;
+      a.blk_logp[o] = pr > 0.f ? logf(pr) : -INFINITY;
+    }
+  }
+  __syncwarp();  // the buffer is rewritten by the warp's next rows
+}
+
+__global__ void __launch_bounds__(kTokThreads, 1) route_tokens_kernel(const RouteArgs a, int rows_per_cta) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int nbr = tok_padded_blocks(a.nb_cap);
+  float* kb = reinterpret_cast<float*>(smem_raw);                                    // [nbr][32] keys
+  float* zb = kb + (size_t)nbr * kIndexDim;                                          // [warps][2][nbr]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(zb + (size_t)kTokWarps * 2 * nbr);
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t_begin = blockIdx.x * rows_per_cta;
+  const int t_end = min(a.tokens, t_begin + rows_per_cta);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+  int64_t m64 = a.prefix_len[b];
+  if (m64 < 0 || m64 > a.cap) {
+    if (tid == 0 && blockIdx.x == 0) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
+    m64 = 0;
+  }
+  const int NB = (int)((m64 + kBlock - 1) / kBlock);
+  bool staged = true;
+  if (NB > 0) {
+    if (tid == 0) {
+      const uint32_t bytes = (uint32_t)NB * kIndexDim * 4;
+      mbar_arrive_expect_tx(bar, bytes);
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.kbar + (int64_t)b * a.nb_cap * kIndexDim);
+      for (uint32_t off = 0; off < bytes; off += kTokCopyBytes)
+        bulk_copy_g2s(reinterpret_cast<uint8_t*>(kb) + off, src + off, min(kTokCopyBytes, bytes - off), bar);
+    }
+    staged = mbar_wait(bar, 0);
+  }
+  if (!__syncthreads_and(staged)) {  // the whole CTA gives up together
+    if (tid == 0) set_status(a.status, RSWA_DEVICE_WAIT_TIMEOUT);
+    if (!staged) (void)mbar_wait(bar, 0);  // the copies in flight land before the CTA leaves
+    return;
+  }
+  const int o = lane >> 3, j = lane & 7;
+  float* zw = zb + (size_t)warp * 2 * nbr;
+  const int n_pairs = (max(0, t_end - t_begin) + 1) / 2;
+  for (int p = warp; p < n_pairs; p += kTokWarps) {
+    const int r0 = t_begin + 2 * p;
+    const bool two = r0 + 1 < t_end;
+    const int64_t row0 = (int64_t)b * a.tokens + r0;
+    if (NB == 0) {
+      if (lane < a.topk) {
+        a.blk_idx[row0 * a.topk + lane] = -1;
+        a.blk_logp[row0 * a.topk + lane] = -INFINITY;
+        if (two) {
+          a.blk_idx[(row0 + 1) * a.topk + lane] = -1;
+          a.blk_logp[(row0 + 1) * a.topk + lane] = -INFINITY;
+        }
+      }
+      continue;
+    }
+    const float4 qa = reinterpret_cast<const float4*>(a.q_idx + row0 * kIndexDim)[j];
+    const float4 qb = two ? reinterpret_cast<const float4*>(a.q_idx + (row0 + 1) * kIndexDim)[j] : qa;
+    for (int base = 0; base < NB; base += 64) {
+      // octet o reads block base + 4i + o, lane j its dims 4j..4j+3 (512 contiguous bytes per
+      // warp load); both rows' 16 partial dots are reduce-scattered over the octet, leaving
+      // lane j the dots of blocks base + 8j + o and base + 8j + 4 + o, as in route_kernel
+      float4 kv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        kv[i] = reinterpret_cast<const float4*>(kb)[(size_t)(base + 4 * i + o) * 8 + j];
+      float va[16], vb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float d = qa.x * kv[i].x;
+        d = fmaf(qa.y, kv[i].y, d);
+        d = fmaf(qa.z, kv[i].z, d);
+        va[i] = fmaf(qa.w, kv[i].w, d);
+        float e = qb.x * kv[i].x;
+        e = fmaf(qb.y, kv[i].y, e);
+        e = fmaf(qb.z, kv[i].z, e);
+        vb[i] = fmaf(qb.w, kv[i].w, e);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool up = j & 4;
+        va[i] = (up ? va[i + 8] : va[i]) + __shfl_xor_sync(0xffffffffu, up ? va[i] : va[i + 8], 4);
+        vb[i] = (up ? vb[i + 8] : vb[i]) + __shfl_xor_sync(0xffffffffu, up ? vb[i] : vb[i + 8], 4);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool up = j & 2;
+        va[i] = (up ? va[i + 4] : va[i]) + __shfl_xor_sync(0xffffffffu, up ? va[i] : va[i + 4], 2);
+        vb[i] = (up ? vb[i + 4] : vb[i]) + __shfl_xor_sync(0xffffffffu, up ? vb[i] : vb[i + 4], 2);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const bool up = j & 1;
+        va[i] = (up ? va[i + 2] : va[i]) + __shfl_xor_sync(0xffffffffu, up ? va[i] : va[i + 2], 1);
+        vb[i] = (up ? vb[i + 2] : vb[i]) + __shfl_xor_sync(0xffffffffu, up ? vb[i] : vb[i + 2], 1);
+      }
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int c = base + 8 * j + 4 * s2 + o;
+        zw[c] = c < NB ? a.idx_scale * va[s2] : -INFINITY;
+        zw[nbr + c] = c < NB ? a.idx_scale * vb[s2] : -INFINITY;
+      }
+    }
+    __syncwarp();
+    tok_finish_row(a, zw, NB, row0, lane);
+    if (two) tok_finish_row(a, zw + nbr, NB, row0 + 1, lane);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_index_pool(int B, int64_t cap, const uint16_t* k_idx, const int32_t* prefix_len, float* kbar,
@@ -569,6 +861,25 @@ cudaError_t launch_route(int B, int tokens, int64_t cap, const float* q_idx, con
   a.probs = probs;
   a.tau = tau;
   a.status = status;
+  if (tokens > 1 && a.nb_cap <= kTokMaxBlocks && probs == nullptr && tau == nullptr) {
+    // many router queries per sequence: the per-token kernel; CTAs per sequence so that the
+    // grid fills the SMs, each with a run of the sequence's tokens
+    const size_t smem = tok_smem_bytes(a.nb_cap);
+    static unsigned long long tok_done = 0;
+    cudaError_t e = ensure_smem_limit(route_tokens_kernel, tok_smem_bytes(kTokMaxBlocks), &tok_done);
+    if (e != cudaSuccess) return e;
+    const int slots = device_sm_count();  // one CTA per SM (its registers alone fill most of one)
+    const int by_rows = (tokens + 2 * kTokWarps - 1) / (2 * kTokWarps);  // a full pass of every warp at least
+    const int by_sms = (slots + B - 1) / B;
+    int gx = by_rows < by_sms ? by_rows : by_sms;
+    if (gx < 1) gx = 1;
+    const int rows_per_cta = (tokens + gx - 1) / gx;
+    gx = (tokens + rows_per_cta - 1) / rows_per_cta;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    fill_launch_config(cfg, attr, dim3(gx, B), dim3(kTokThreads), smem, stream);
+    return cudaLaunchKernelEx(&cfg, route_tokens_kernel, a, rows_per_cta);
+  }
   const size_t smem = (size_t)a.csize * kRouteThreads * 2 * 8 + (size_t)route_sort_capacity(a.csize) * 8;
   static unsigned long long done = 0;
   cudaError_t e = ensure_smem_limit(

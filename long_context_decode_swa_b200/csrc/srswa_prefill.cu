@@ -107,6 +107,7 @@ struct GroupArgs {
   int32_t* gblk;         // [B * T][kMaxTopk]: per query, its route's blocks ascending (INT_MAX past them)
   float* gbias;          // [B * T][kMaxTopk]: per query, ln p of those blocks in that order
   int32_t* counts;       // [0] groups, [1] gq entries (zeroed before the launch)
+  uint64_t* keys;        // [B * T]: per query, its sort key (group_prep_kernel -> group_kernel)
 };
 
 // Block-wide inclusive prefix sum of three counters over the threads
@@ -142,10 +143,46 @@ __device__ __forceinline__ int3 block_scan3(int3 v, int3* wsum, int3& total) {
   return make_int3(before.x + inc.x, before.y + inc.y, before.z + inc.z);
 }
 
-// One CTA per sequence: sorts the chunk's queries by a hash of their block sets (the hash
-// only brings equal sets together; adjacent queries are compared set for set) and cuts every
-// run of equal sets into groups of up to 128 queries. Queries with an empty route join none.
-__global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a) {
+// One thread per query of the chunk, over the whole grid: the query's route sorted by block into
+// its scratch rows (blocks ascending, INT_MAX past them; ln p in the same order) and its sort
+// key: a hash of the sorted block list in the high bits (equal sets, equal hashes) and the
+// position in the low 13 (keys of empty routes sort last). Route entries past the prefix are
+// flagged (their rows lie outside it: they are read as masked).
+constexpr int kPrepThreads = 128;
+
+__global__ void __launch_bounds__(kPrepThreads) group_prep_kernel(const GroupArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t qi = (int64_t)blockIdx.x * kPrepThreads + threadIdx.x;
+  if (qi >= (int64_t)a.B * a.T) return;
+  const int b = (int)(qi / a.T), t = (int)(qi - (int64_t)b * a.T);
+  const int m_b = a.prefix_len[b];
+  const int NB = (m_b < 0 || m_b > a.cap) ? 0 : (m_b + 31) / 32;
+  RouteRegs rq;
+  load_route(a.blk, a.logp, qi * a.topk, a.topk, rq);
+  int4* gb = reinterpret_cast<int4*>(a.gblk + qi * kMaxTopk);
+  float4* gl = reinterpret_cast<float4*>(a.gbias + qi * kMaxTopk);
+#pragma unroll
+  for (int j = 0; j < kMaxTopk; j += 4) {
+    gb[j / 4] = make_int4(rq.blk[j], rq.blk[j + 1], rq.blk[j + 2], rq.blk[j + 3]);
+    gl[j / 4] = make_float4(rq.lp[j], rq.lp[j + 1], rq.lp[j + 2], rq.lp[j + 3]);
+  }
+  uint64_t h = 0;
+  int top = -1;
+#pragma unroll
+  for (int j = 0; j < kMaxTopk; ++j)
+    if (j < rq.k) {
+      h = mix64(h ^ (uint64_t)(uint32_t)rq.blk[j]);
+      top = rq.blk[j];
+    }
+  a.keys[qi] = rq.k > 0 ? (mix64(h + (uint64_t)rq.k) & ~0x1FFFull) | (uint64_t)t : ~0ull;
+  if (top >= NB) set_status(a.status, RSWA_DEVICE_BAD_BLOCK_IDX);  // the largest valid block lies past the prefix
+}
+
+// One CTA per sequence: sorts the chunk's queries by their keys (the hash only brings equal
+// sets together; adjacent queries are compared set for set) and cuts every run of equal sets
+// into groups of up to 128 queries. Queries with an empty route join none.
+__global__ void __launch_bounds__(kGroupThreads, 1) group_kernel(const GroupArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ int3 wsum[kGroupThreads / 32];
   __shared__ int s_base[3];
@@ -157,38 +194,9 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
   int* hp = reinterpret_cast<int*>(keys + np2);              // segment starts (T + 1)
   griddep_wait();
   griddep_launch_dependents();
-  // route entries past the prefix are flagged (their rows lie outside it: they are read as masked)
   const int m_b = a.prefix_len[b];
-  const int NB = (m_b < 0 || m_b > a.cap) ? 0 : (m_b + 31) / 32;
   if (tid == 0 && (m_b < 0 || m_b > a.cap)) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
-  bool bad = false;
-  // each query's route sorted by block into the scratch rows, and its sort key
-  for (int t = tid; t < np2; t += kGroupThreads) {
-    uint64_t key = ~0ull;  // empty routes and padding sort last
-    if (t < T) {
-      RouteRegs rq;
-      load_route(a.blk, a.logp, ((int64_t)b * T + t) * a.topk, a.topk, rq);
-      int4* gb = reinterpret_cast<int4*>(a.gblk + ((int64_t)b * T + t) * kMaxTopk);
-      float4* gl = reinterpret_cast<float4*>(a.gbias + ((int64_t)b * T + t) * kMaxTopk);
-      uint64_t h = 0;
-#pragma unroll
-      for (int j = 0; j < kMaxTopk; j += 4) {
-        gb[j / 4] = make_int4(rq.blk[j], rq.blk[j + 1], rq.blk[j + 2], rq.blk[j + 3]);
-        gl[j / 4] = make_float4(rq.lp[j], rq.lp[j + 1], rq.lp[j + 2], rq.lp[j + 3]);
-      }
-      int top = -1;
-#pragma unroll
-      for (int j = 0; j < kMaxTopk; ++j)
-        if (j < rq.k) {
-          h = mix64(h ^ (uint64_t)(uint32_t)rq.blk[j]);  // the sorted list: equal sets, equal hashes
-          top = rq.blk[j];
-        }
-      if (rq.k > 0) key = (mix64(h + (uint64_t)rq.k) & ~0x1FFFull) | (uint64_t)t;
-      bad |= top >= NB;  // the largest valid block lies past the prefix
-    }
-    keys[t] = key;
-  }
-  if (bad) set_status(a.status, RSWA_DEVICE_BAD_BLOCK_IDX);
+  for (int t = tid; t < np2; t += kGroupThreads) keys[t] = t < T ? a.keys[(int64_t)b * T + t] : ~0ull;
   for (int k2 = 2; k2 <= np2; k2 <<= 1)
     for (int j = k2 >> 1; j > 0; j >>= 1) {
       __syncthreads();
@@ -724,15 +732,24 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
 size_t srswa_prefill_scratch_bytes(int B, int H, int T) {
   const size_t bt = (size_t)B * T;
   return 256 + (bt * kRec * 4 + 255) / 256 * 256 + (bt * 4 + 255) / 256 * 256 + bt * kMaxTopk * 8 +
-         ((size_t)B * H * T * 4 + 255) / 256 * 256;
+         ((size_t)B * H * T * 4 + 255) / 256 * 256 + bt * 8;
 }
 
 int srswa_prefill_group_rec_ints() { return kRec; }
 
 cudaError_t launch_srswa_group(int B, int T, int topk, int64_t cap, const int32_t* prefix_len, const int32_t* blk,
                                const float* logp, int32_t* rec, int32_t* gq, int32_t* gblk, float* gbias,
-                               int32_t* counts, int32_t* status, cudaStream_t stream) {
-  GroupArgs a{B, T, topk, cap, prefix_len, status, blk, logp, rec, gq, gblk, gbias, counts};
+                               int32_t* counts, uint64_t* keys, int32_t* status, cudaStream_t stream) {
+  GroupArgs a{B, T, topk, cap, prefix_len, status, blk, logp, rec, gq, gblk, gbias, counts, keys};
+  {  // the per-query part over the whole grid, then the per-sequence sort and cut
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    const int64_t queries = (int64_t)B * T;
+    fill_launch_config(cfg, attr, dim3((unsigned)((queries + kPrepThreads - 1) / kPrepThreads)), dim3(kPrepThreads),
+                       0, stream);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, group_prep_kernel, a);
+    if (e != cudaSuccess) return e;
+  }
   int np2 = 1;
   while (np2 < T) np2 <<= 1;
   const size_t smem = (size_t)np2 * 8 + (size_t)(T + 1) * 4 + (size_t)T;
