@@ -84,17 +84,6 @@ __device__ __forceinline__ void load_route(const int32_t* blk, const float* logp
   q.k = k;
 }
 
-// Two queries' sorted block lists (rows of the grouping scratch) agree: the same set.
-__device__ __forceinline__ bool same_set(const int32_t* x, const int32_t* y) {
-  bool same = true;
-#pragma unroll
-  for (int j = 0; j < kMaxTopk; j += 4) {
-    const int4 u = *reinterpret_cast<const int4*>(x + j), v = *reinterpret_cast<const int4*>(y + j);
-    same &= u.x == v.x && u.y == v.y && u.z == v.z && u.w == v.w;
-  }
-  return same;
-}
-
 struct GroupArgs {
   int B, T, topk;
   int64_t cap;
@@ -179,6 +168,71 @@ __global__ void __launch_bounds__(kPrepThreads) group_prep_kernel(const GroupArg
   if (top >= NB) set_status(a.status, RSWA_DEVICE_BAD_BLOCK_IDX);  // the largest valid block lies past the prefix
 }
 
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Stage (k2, J) of the bitonic network for the pairs inside one thread's registers (J < E).
+template <int E, int J>
+__device__ __forceinline__ void sort_stage_regs(uint64_t (&x)[E], int t, int k2) {
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if ((e & J) == 0) {
+      const bool ascending = ((t * E + e) & k2) == 0;
+      const uint64_t u = x[e], v = x[e | J];
+      if ((u > v) == ascending) {
+        x[e] = v;
+        x[e | J] = u;
+      }
+    }
+}
+
+// Ascending bitonic sort of the chunk's keys of sequence b (padded with ~0 to
+// kGroupThreads * E), held E per thread: thread t holds logical elements t * E + e. Strides
+// below E are exchanged in registers, strides up to 32 E between the lanes of a warp by
+// shuffles, larger ones through shared memory (element-major there: logical t * E + e at
+// e * kGroupThreads + t, so the writes and the partner reads are both conflict-free).
+// The sorted keys end in keys[0, kGroupThreads * E) in logical order. Every thread calls it.
+template <int E>
+__device__ void sort_keys(const uint64_t* g, int T, uint64_t* keys) {
+  const int t = threadIdx.x;
+  constexpr int N = kGroupThreads * E;
+  uint64_t x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = t * E + e < T ? g[t * E + e] : ~0ull;
+  for (int k2 = 2; k2 <= N; k2 <<= 1)
+    for (int j = k2 >> 1; j > 0; j >>= 1) {
+      if (j < E) {
+        if (j == 1) sort_stage_regs<E, 1>(x, t, k2);
+        if constexpr (E > 2) if (j == 2) sort_stage_regs<E, 2>(x, t, k2);
+        if constexpr (E > 4) if (j == 4) sort_stage_regs<E, 4>(x, t, k2);
+        if constexpr (E > 8) if (j == 8) sort_stage_regs<E, 8>(x, t, k2);
+      } else {
+        const bool in_warp = j < 32 * E;
+        if (!in_warp) {  // partner in another warp
+          __syncthreads();  // the previous stage's readers are done
+#pragma unroll
+          for (int e = 0; e < E; ++e) keys[e * kGroupThreads + t] = x[e];
+          __syncthreads();
+        }
+        const int m = j / E;  // the partner thread: t ^ m
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = t * E + e;
+          const uint64_t y = in_warp ? shfl_xor_u64(x[e], m) : keys[e * kGroupThreads + (t ^ m)];
+          const bool keep_min = ((i & k2) == 0) == ((i & j) == 0);
+          x[e] = keep_min ? (x[e] < y ? x[e] : y) : (x[e] < y ? y : x[e]);
+        }
+      }
+    }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < E; ++e) keys[t * E + e] = x[e];
+  __syncthreads();
+}
+
 // One CTA per sequence: sorts the chunk's queries by their keys (the hash only brings equal
 // sets together; adjacent queries are compared set for set) and cuts every run of equal sets
 // into groups of up to 128 queries. Queries with an empty route join none.
@@ -188,7 +242,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) group_kernel(const GroupArgs
   __shared__ int s_base[3];
   const int b = blockIdx.x, tid = threadIdx.x;
   const int T = a.T;
-  int np2 = 1;
+  int np2 = kGroupThreads;
   while (np2 < T) np2 <<= 1;
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem_raw);  // np2 sort keys: hash (high bits) | position
   int* hp = reinterpret_cast<int*>(keys + np2);              // segment starts (T + 1)
@@ -196,34 +250,42 @@ __global__ void __launch_bounds__(kGroupThreads, 1) group_kernel(const GroupArgs
   griddep_launch_dependents();
   const int m_b = a.prefix_len[b];
   if (tid == 0 && (m_b < 0 || m_b > a.cap)) set_status(a.status, RSWA_DEVICE_BAD_PREFIX_LEN);
-  for (int t = tid; t < np2; t += kGroupThreads) keys[t] = t < T ? a.keys[(int64_t)b * T + t] : ~0ull;
-  for (int k2 = 2; k2 <= np2; k2 <<= 1)
-    for (int j = k2 >> 1; j > 0; j >>= 1) {
-      __syncthreads();
-      for (int i = tid; i < np2; i += kGroupThreads) {
-        const int p = i ^ j;
-        if (p > i) {
-          const uint64_t x = keys[i], y = keys[p];
-          if ((x > y) == ((i & k2) == 0)) {
-            keys[i] = y;
-            keys[p] = x;
-          }
-        }
-      }
-    }
-  __syncthreads();
+  const uint64_t* gkeys = a.keys + (int64_t)b * T;
+  switch (np2 / kGroupThreads) {  // uniform over the CTA
+    case 1: sort_keys<1>(gkeys, T, keys); break;
+    case 2: sort_keys<2>(gkeys, T, keys); break;
+    case 4: sort_keys<4>(gkeys, T, keys); break;
+    case 8: sort_keys<8>(gkeys, T, keys); break;
+    default: sort_keys<16>(gkeys, T, keys); break;
+  }
   // positions [p0, p1) per thread (contiguous, so the scans give ranks in position order)
   const int per = (T + kGroupThreads - 1) / kGroupThreads;
   const int p0 = min(T, tid * per), p1 = min(T, p0 + per);
   auto valid_at = [&](int p) { return keys[p] != ~0ull; };
   auto pos_at = [&](int p) { return (int)(keys[p] & 0x1FFFull); };
   uint8_t* hf = reinterpret_cast<uint8_t*>(hp + T + 1);  // per position: segment head
-  for (int p = p0; p < p1; ++p) {
+  // a position starts a segment unless its neighbour below has the same hash and, compared
+  // block by block, the same set (rows hold the blocks ascending, INT_MAX past the valid
+  // ones, so the first topk entries decide); positions strided over the threads, so that each
+  // thread's row loads are independent
+  const int chunks = (a.topk + 3) / 4;
+#pragma unroll 2
+  for (int p = tid; p < T; p += kGroupThreads) {
     bool head = false;
     if (valid_at(p)) {
-      head = p == 0 || (keys[p] >> 13) != (keys[p - 1] >> 13) ||
-             !same_set(a.gblk + ((int64_t)b * T + pos_at(p)) * kMaxTopk,
-                       a.gblk + ((int64_t)b * T + pos_at(p - 1)) * kMaxTopk);
+      head = p == 0 || (keys[p] >> 13) != (keys[p - 1] >> 13);
+      if (!head) {
+        const int4* u = reinterpret_cast<const int4*>(a.gblk + ((int64_t)b * T + pos_at(p)) * kMaxTopk);
+        const int4* v = reinterpret_cast<const int4*>(a.gblk + ((int64_t)b * T + pos_at(p - 1)) * kMaxTopk);
+        bool same = true;
+#pragma unroll
+        for (int c = 0; c < kMaxTopk / 4; ++c)
+          if (c < chunks) {
+            const int4 x = u[c], y = v[c];
+            same &= x.x == y.x && x.y == y.y && x.z == y.z && x.w == y.w;
+          }
+        head = !same;
+      }
     }
     hf[p] = head ? 1 : 0;
   }
@@ -752,6 +814,7 @@ cudaError_t launch_srswa_group(int B, int T, int topk, int64_t cap, const int32_
   }
   int np2 = 1;
   while (np2 < T) np2 <<= 1;
+  if (np2 < kGroupThreads) np2 = kGroupThreads;
   const size_t smem = (size_t)np2 * 8 + (size_t)(T + 1) * 4 + (size_t)T;
   static unsigned long long done = 0;
   cudaError_t e = ensure_smem_limit(group_kernel, (size_t)8192 * 8 + 8193 * 4 + 8192, &done);
