@@ -373,7 +373,8 @@ struct __align__(1024) RoutedSmem {
   uint8_t kv[kKV][kTileR];
   uint64_t q_full, q_empty;
   uint64_t kv_full[kKV], kv_empty[kKV];
-  uint64_t s_full, p_full, o_full, o_free;
+  uint64_t s_full[kChunkBlocks / 4];  // S of key tile t of the pass is in TMEM
+  uint64_t p_full, o_full, o_free;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    mbar_init(&sm.s_full, 1);
+    for (int t = 0; t < kChunkBlocks / 4; ++t) mbar_init(&sm.s_full[t], 1);
     mbar_init(&sm.p_full, 128);
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_free, 128);
@@ -499,8 +500,11 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
       // ---------------- producer: K tiles then V tiles of each pass ----------------
       int idx = 0;  // tiles through the ring so far
       bool ok = true;
+      Unit wn;  // the next unit's record, loaded one unit ahead
+      if ((int)blockIdx.x < n_units) wn = unit_at(a, blockIdx.x);
       for (int u = blockIdx.x; ok && u < n_units; u += grid) {
-        const Unit w = unit_at(a, u);
+        const Unit w = wn;
+        if (u + grid < n_units) wn = unit_at(a, u + grid);
         const int64_t row0 = ((int64_t)w.b * a.H + w.h) * a.cap;
         for (int c = 0; ok && c < unit_passes(w); ++c) {
           const int nkt = (pass_blocks(w, c) + 3) / 4;
@@ -534,8 +538,11 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
     constexpr uint32_t kIdescPV = idesc_bf16_m128_n128(1);
     int idx = 0, it = 0;
     bool ok = true;
+    Unit wn;  // the next unit's record, loaded one unit ahead
+    if ((int)blockIdx.x < n_units) wn = unit_at(a, blockIdx.x);
     for (int u = blockIdx.x; ok && u < n_units; u += grid) {
-      const Unit w = unit_at(a, u);
+      const Unit w = wn;
+      if (u + grid < n_units) wn = unit_at(a, u + grid);
       for (int c = 0; ok && c < unit_passes(w); ++c, ++it) {
         const int nkt = (pass_blocks(w, c) + 3) / 4;
         ok = __all_sync(0xffffffffu, routed_wait(sm, &sm.q_full, it & 1, a.status));
@@ -559,6 +566,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
                         smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0);
             }
             tc_commit(&sm.kv_empty[s]);
+            tc_commit(&sm.s_full[t]);  // the softmax's first pass follows tile by tile
           }
           __syncwarp();
         }
@@ -566,10 +574,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
         // a pass of fewer than 3 key tiles still frees the previous O before PV writes it
         if (nkt < 3 && it > 0) ok = __all_sync(0xffffffffu, routed_wait(sm, &sm.o_free, (it - 1) & 1, a.status));
         if (!ok) break;
-        if (lane == 0) {
-          tc_commit(&sm.s_full);
-          tc_commit(&sm.q_empty);
-        }
+        if (lane == 0) tc_commit(&sm.q_empty);
         __syncwarp();
         ok = __all_sync(0xffffffffu, routed_wait(sm, &sm.p_full, it & 1, a.status));
         if (!ok) break;
@@ -655,6 +660,7 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
     const int r = tid - 128;
     const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
     int it = 0;
+    uint32_t s_phase = 0;  // bit t: parity of the next completion of s_full[t]
     bool ok = true;
     for (int u = blockIdx.x; ok && u < n_units; u += grid) {
       const Unit w = unit_at(a, u);
@@ -683,61 +689,71 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
             if (!live) bias[j] = -INFINITY;
           }
         }
-        if (!(ok = __all_sync(0xffffffffu, routed_wait(sm, &sm.s_full, it & 1, a.status)))) break;
-        tc_fence_after();
-        // pass 1: the row maximum over every routed key of the pass
+        // pass 1: the row maximum over every routed key of the pass, key tile by key tile as the
+        // tensor core finishes them; two 32-column chunks (block slots) per TMEM wait
         float mx = -INFINITY;
-        // one 32-column chunk (one block slot) per iteration; not unrolled: a compact loop body
 #pragma unroll 1
-        for (int j = 0; j < 4 * nkt; ++j) {
-          {
-            uint32_t rv[32];
-            tmem_ld32(tmem + lane_base + (uint32_t)(j * 32), rv);
-            tmem_wait_ld();
-            const float bj = pick16(bias, j);
-            const int nr = pick16(rows, j);
+        for (int j = 0; j < 4 * nkt; j += 2) {
+          if ((j & 3) == 0) {
+            // s_full[t] completes once per pass that has key tile t: its own phase bit
+            const int t = j >> 2;
+            if (!(ok = __all_sync(0xffffffffu, routed_wait(sm, &sm.s_full[t], (s_phase >> t) & 1u, a.status))))
+              break;
+            s_phase ^= 1u << t;
+            tc_fence_after();
+          }
+          uint32_t rv[32], rw[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)(j * 32), rv);
+          tmem_ld32(tmem + lane_base + (uint32_t)(j * 32 + 32), rw);
+          tmem_wait_ld();
+          const float bj = pick16(bias, j), bk = pick16(bias, j + 1);
+          const int nr = pick16(rows, j), ns = pick16(rows, j + 1);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (e < nr) mx = fmaxf(mx, fmaf(__uint_as_float(rv[e]), a.qk_scale_log2, bj));
+          for (int e = 0; e < 32; ++e) {
+            if (e < nr) mx = fmaxf(mx, fmaf(__uint_as_float(rv[e]), a.qk_scale_log2, bj));
+            if (e < ns) mx = fmaxf(mx, fmaf(__uint_as_float(rw[e]), a.qk_scale_log2, bk));
           }
         }
+        if (!ok) break;
         const float msub = mx == -INFINITY ? 0.f : mx;
-        // pass 2: P = 2^(s - max) as bf16 pairs over the S columns already read
+        // pass 2: P = 2^(s - max) as bf16 pairs over the S columns already read; two chunks per
+        // TMEM wait (P of chunk j lands in columns [16 j, 16 j + 16), inside chunks already read)
         float l = 0.f, lu = 0.f;
-#pragma unroll 1
-        for (int j = 0; j < 4 * nkt; ++j) {
-          {
-            uint32_t rv[32];
-            tmem_ld32(tmem + lane_base + (uint32_t)(j * 32), rv);
-            tmem_wait_ld();
-            const float bj = pick16(bias, j);
-            const int nr = pick16(rows, j);
-            uint32_t pk[16];
+        auto p_chunk = [&](const uint32_t (&rv)[32], float bj, int nr, uint32_t (&pk)[16]) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = 2 * e < nr ? fmaf(__uint_as_float(rv[2 * e]), a.qk_scale_log2, bj) - msub : -INFINITY;
-              const float x1 =
-                  2 * e + 1 < nr ? fmaf(__uint_as_float(rv[2 * e + 1]), a.qk_scale_log2, bj) - msub : -INFINITY;
-              const float p0 = ex2(x0), p1 = ex2(x1);  // MUFU 2^x (2^-inf = 0), as in the dense prefill
-              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
-              l += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
-              lu += p0 + p1;
-            }
-            tmem_st16(tmem + lane_base + (uint32_t)(j * 16), pk);  // P of chunk j: 16 packed columns
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = 2 * e < nr ? fmaf(__uint_as_float(rv[2 * e]), a.qk_scale_log2, bj) - msub : -INFINITY;
+            const float x1 =
+                2 * e + 1 < nr ? fmaf(__uint_as_float(rv[2 * e + 1]), a.qk_scale_log2, bj) - msub : -INFINITY;
+            const float p0 = ex2(x0), p1 = ex2(x1);  // MUFU 2^x (2^-inf = 0), as in the dense prefill
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
+            l += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+            lu += p0 + p1;
           }
+        };
+#pragma unroll 1
+        for (int j = 0; j < 4 * nkt; j += 2) {
+          uint32_t rv[32], rw[32], pk[16];
+          tmem_ld32(tmem + lane_base + (uint32_t)(j * 32), rv);
+          tmem_ld32(tmem + lane_base + (uint32_t)(j * 32 + 32), rw);
+          tmem_wait_ld();
+          p_chunk(rv, pick16(bias, j), pick16(rows, j), pk);
+          tmem_st16(tmem + lane_base + (uint32_t)(j * 16), pk);
+          p_chunk(rw, pick16(bias, j + 1), pick16(rows, j + 1), pk);
+          tmem_st16(tmem + lane_base + (uint32_t)(j * 16 + 16), pk);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full);
-        // the band part's row, read while the tensor core runs P.V
+        // the band part's row: brought into L1 while the tensor core runs P.V, read at the merge
+        // (held in registers instead, it would leave too few for the paired TMEM loads)
         const int64_t vq = ((int64_t)w.b * a.H + w.h) * a.T + t_q;
         float* orow = a.out + vq * kHeadDim;
-        float4 oa[kHeadDim / 4];
         float lse_a = -INFINITY;
         if (live) {
 #pragma unroll
-          for (int e = 0; e < kHeadDim / 4; ++e) oa[e] = reinterpret_cast<const float4*>(orow)[e];
+          for (int e = 0; e < kHeadDim; e += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(orow + e));
           lse_a = a.lse[vq];
         }
         if (!(ok = __all_sync(0xffffffffu, routed_wait(sm, &sm.o_full, it & 1, a.status)))) break;
@@ -763,9 +779,12 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
           tmem_ld32(tmem + lane_base + kColOR + (uint32_t)ch * 32u, rv);
           tmem_wait_ld();
           if (live) {
+            float4 ob[8];  // the band part's values of these 32 columns
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ob[e] = reinterpret_cast<const float4*>(orow + ch * 32)[e];
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              float4 o = oa[(ch * 32 + e) / 4];
+              float4 o = ob[e / 4];
               o.x = fmaf(o.x, wa, __uint_as_float(rv[e]) * inv_l);
               o.y = fmaf(o.y, wa, __uint_as_float(rv[e + 1]) * inv_l);
               o.z = fmaf(o.z, wa, __uint_as_float(rv[e + 2]) * inv_l);
@@ -790,7 +809,8 @@ __global__ void __launch_bounds__(kRoutedThreads, 1)
 
 }  // namespace
 
-// Workspace of srswa_prefill past its status area: [counts 256 B][group records][gq][gblk][gbias][lse scratch].
+// Workspace of srswa_prefill past its status area: [counts 256 B][group records][gq][gblk][gbias][lse scratch]
+// [sort keys].
 size_t srswa_prefill_scratch_bytes(int B, int H, int T) {
   const size_t bt = (size_t)B * T;
   return 256 + (bt * kRec * 4 + 255) / 256 * 256 + (bt * 4 + 255) / 256 * 256 + bt * kMaxTopk * 8 +
