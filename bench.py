@@ -744,8 +744,9 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
         "config": config_of(w, args, world),
         "timing": TIMING_NOTE,
         "qtok_per_s": value * B * H * T,
-        "roofline": ({"bound": "tensor", "kernel": "SR-SWA prefill attention: group_kernel + prefill_kernel (band "
-                                                 "and ring, tcgen05) + routed_kernel (routed blocks, tcgen05)",
+        "roofline": ({"bound": "tensor", "kernel": "SR-SWA prefill attention: group_prep_kernel + group_kernel + "
+                                                 "prefill_kernel (band and ring, tcgen05) + routed_kernel (routed "
+                                                 "blocks, tcgen05)",
                       "achieved": achieved, "peak": peak,
                       "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json); "
                                      "FLOPs counted per query over its own routed rows and band",
@@ -759,7 +760,8 @@ def run_prefill(args, w: dict, world: int, rank: int, local: int) -> dict:
                       "traffic": committed_traffic(f"rswa_prefill_config{args.config}", kernel_source_hash("prefill")),
                       "algorithmic_flops_per_launch": flops, "avg_launch_us": kern_s * 1e6}),
         "kernels_us": {"prefill": kern_s * 1e6, **({"route": route_s * 1e6} if sparse else {})},
-        "gpu_launches": K * (2 if sparse else 1),
+        # SR-SWA: route_tokens, group_prep, group, band prefill, routed; dense: the prefill kernel
+        "gpu_launches": K * (5 if sparse else 1),
         "clocks": clk,
         "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": "prefill chunks/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms / K},
