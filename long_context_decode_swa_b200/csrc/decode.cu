@@ -183,9 +183,12 @@ __device__ __forceinline__ SeqView make_view(const DecodeArgs& a, int b, int h, 
   int cnt = f;  // ring slots read: the cnt most recently written, (w - cnt + i) mod n for i < cnt
   if (band) cnt = min(max(a.n - 1 - i, 0), f);
   // fused append: the oldest slot of a full ring (slot w) is overwritten by this step's token,
-  // which is read from k_new / v_new as the last tile instead
+  // which is read from k_new / v_new as the item's first tile instead
   // (a sequence with a bad ring state is left untouched, as rswa_append leaves it). A full
-  // ring is still read as [0, n) in aligned tiles, with the overwritten slot masked.
+  // ring is still read as [0, n) in aligned tiles, with the overwritten slot masked: the bulk
+  // copy of the tile holding slot w may read that row while the token's warp writes it (an
+  // unsynchronised cross-proxy read and write of one row), and the mask keeps whatever it
+  // reads out of every score and of P.V.
   const bool app = mode_appends(kMode) && ring_ok;
   // a full ring is read as [0, n)
   int a0 = cnt == a.n ? 0 : (w - cnt) % a.n;
