@@ -204,3 +204,48 @@ def test_srswa_step_rope_matches_unfused_and_oracle(cuda_lib, plen, H, steps):
         assert_attention_close(to_np(fused.out), want, f"encoded SR-SWA step {s}")
         assert np.abs(to_np(fused.lse) - want_lse).max() <= LSE_ABS
     assert rswa.check_status(fused.ws) == 0 and rswa.check_status(ref.ws) == 0
+
+
+def test_srswa_step_rope_full_size_sampled(cuda_lib):
+    # the benchmarked encoded SR-SWA step: 64 sequences x 16 heads, 32K-token histories, two
+    # steps; every output bit-equal to the unfused sequence, the route of every sequence against
+    # the oracle's router, sampled sequences against the oracle's encoding, append and decode
+    rswa = cuda_lib
+    B, H, cap, steps = 64, 16, 32768, 2
+    plen = [cap] * B
+    c = synth.decode_case(B, H, 128, plen, cap, 128, steps, seed=990, device="cuda")
+    pl = synth.plant_router_keys(plen, cap, n_dirs=4, seed=991, device="cuda")
+    pt = torch.tensor(plen, dtype=torch.int32, device="cuda")
+    kbar = torch.empty((B, cap // 32, 32), dtype=torch.float32, device="cuda")
+    rswa.srswa_index_pool(pl.k_idx, pt, kbar)
+    o_kbar = oracle.index_pool(to_np(pl.k_idx), np.array(plen, np.int32))
+    tok, page = synth.page_positions(B, steps, seed=992)
+    fused, ref = Arm(rswa, c, rswa.OP_SRSWA_ROUTED), Arm(rswa, c, rswa.OP_SRSWA_ROUTED)
+    sample = np.array([0, 9, 31, 63])
+    sel = torch.as_tensor(sample, device="cuda")
+    o_pk, o_pv = to_np(c.pk.index_select(0, sel)), to_np(c.pv.index_select(0, sel))
+    o_rk, o_rv = to_np(c.ring_k)[sample].copy(), to_np(c.ring_v)[sample].copy()
+    o_wp, o_fill = to_np(c.wp)[sample].copy(), to_np(c.fill)[sample].copy()
+    for s in range(steps):
+        t_s, p_s = tok[:, s].contiguous().cuda(), page[:, s].contiguous().cuda()
+        rswa.srswa_step_rope(c.q[s], c.k_new[s], c.v_new[s], pl.q_idx[s], kbar, c.pk, c.pv, c.prefix_len,
+                             fused.ring_k, fused.ring_v, fused.wp, fused.fill, t_s, p_s, fused.blk, fused.logp,
+                             fused.out, fused.ws, lse=fused.lse, tau=fused.tau, slot_out=fused.slot, scale=c.scale)
+        q_rot, k_rot = _encode(rswa, c.q[s], c.k_new[s], t_s, p_s, 10000.0, 2)
+        rswa.srswa_step(q_rot, k_rot, c.v_new[s], pl.q_idx[s], kbar, c.pk, c.pv, c.prefix_len, ref.ring_k,
+                        ref.ring_v, ref.wp, ref.fill, ref.blk, ref.logp, ref.out, ref.ws, lse=ref.lse, tau=ref.tau,
+                        slot_out=ref.slot, scale=c.scale)
+        fused.assert_same(ref, f"full-size SR-SWA step {s}", route=True)
+        ro = oracle.route(to_np(pl.q_idx[s]), o_kbar, np.array(plen, np.int32))
+        np.testing.assert_array_equal(to_np(fused.blk), ro["blk_idx"], err_msg=f"route step {s}")
+        ts, ps = tok[sample, s].numpy(), page[sample, s].numpy()
+        qo = oracle.bf16_round(oracle.rope_page2d(to_np(c.q[s])[sample], ts, ps))
+        ko = oracle.bf16_round(oracle.rope_page2d(to_np(c.k_new[s])[sample], ts, ps))
+        oracle.append(o_rk, o_rv, ko, to_np(c.v_new[s])[sample], o_wp, o_fill)
+        want, want_lse = oracle.srswa_decode(qo, o_pk, o_pv, np.array(plen, np.int32)[sample],
+                                             np.ascontiguousarray(ro["blk_idx"][sample]),
+                                             np.ascontiguousarray(ro["blk_logp"][sample]), o_rk, o_rv, o_wp, o_fill,
+                                             c.scale)
+        assert_attention_close(to_np(fused.out)[sample], want, f"full-size encoded SR-SWA step {s}")
+        assert np.abs(to_np(fused.lse)[sample] - want_lse).max() <= LSE_ABS
+    assert rswa.check_status(fused.ws) == 0 and rswa.check_status(ref.ws) == 0

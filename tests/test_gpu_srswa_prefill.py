@@ -155,3 +155,30 @@ def test_srswa_prefill_bad_block_is_flagged(cuda_lib):
     cuda_lib.srswa_prefill(d["q"], d["k_out"], d["v_out"], d["pk"], d["pv"], d["prefix_len"],
                            torch.from_numpy(blk).cuda(), torch.from_numpy(logp).cuda(), out, ws, scale=d["scale"])
     assert cuda_lib.check_status(ws) & cuda_lib.binding.DEVICE_BAD_BLOCK_IDX
+
+
+def test_srswa_prefill_chunk_full_size_sampled(cuda_lib):
+    # the benchmarked chunk: 4 sequences x 16 heads x 4096 queries over a 32K-token history,
+    # every query routed by srswa_route_tokens (planted keys, 32 directions cycled over the
+    # tokens, so 32 block sets of 128 queries per sequence); routes of sampled tokens against
+    # the oracle's router, attention rows sampled against the oracle's prefill
+    B, H, T, cap = 4, 16, 4096, 32768
+    plen = [cap] * B
+    pl = synth.plant_router_keys(plen, cap, n_dirs=32, seed=81, device="cuda")
+    q_tok = pl.q_idx[torch.arange(T, device="cuda") % 32].permute(1, 0, 2).contiguous()
+    pt = torch.tensor(plen, dtype=torch.int32, device="cuda")
+    kbar = torch.empty((B, cap // 32, 32), dtype=torch.float32, device="cuda")
+    cuda_lib.srswa_index_pool(pl.k_idx, pt, kbar)
+    blk = torch.empty((B, T, 16), dtype=torch.int32, device="cuda")
+    logp = torch.empty((B, T, 16), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    cuda_lib.srswa_route_tokens(q_tok, kbar, pt, blk, logp, ws, prefix_cap=cap)
+    assert cuda_lib.check_status(ws) == 0
+    rows = np.concatenate([np.arange(0, 4), np.arange(126, 131), np.arange(2047, 2050), np.arange(T - 4, T)])
+    plen_np = np.array(plen, np.int32)
+    r_idx, r_logp = oracle.route_tokens(to_np(q_tok)[:, rows], oracle.index_pool(to_np(pl.k_idx), plen_np), plen_np)
+    np.testing.assert_array_equal(to_np(blk)[:, rows], r_idx)
+    np.testing.assert_allclose(np.exp(to_np(logp)[:, rows]), np.exp(r_logp), rtol=0, atol=ROUTER_P_ABS)
+    del pl
+    d = synth.prefill_case(B, H, 128, plen, cap, T, seed=82, device="cuda", poison=False)
+    _check(cuda_lib, d, to_np(blk), to_np(logp), 128, rows, tag="srswa prefill full chunk")
