@@ -48,3 +48,35 @@ def test_cpu_baseline_reports_threads_and_a_one_thread_figure():
     r = bench.cpu_baseline(bench.workload(1), budget_s=0.5, budget_1thread_s=0.3)
     assert r["kind"] == "oracle" and r["value"] > 0 and r["value_1thread"] > 0
     assert r["cores"] >= 1 and r["host_cpus"] >= 1 and r["cpu_model"]
+
+
+def test_traffic_records_follow_the_kernel_source():
+    # a committed DRAM-traffic record is reported only while the kernel source it was captured on
+    # is unchanged (comments and blank lines aside); every record names a known workload key
+    kinds = {"rswa_decode": "dense", "srswa_decode": "sparse", "srswa_step_decode": "sparse",
+             "rswa_prefill": "prefill", "srswa_prefill": "srswa_prefill", "rope": "rope"}
+    lines = [ln.split() for ln in open(os.path.join(ROOT, "profiles", "ncu_traffic.txt"))
+             if ln.strip() and not ln.startswith("#")]
+    assert lines
+    for parts in lines:
+        key, src_hash, nbytes = parts[0], parts[1], float(parts[2])
+        kind = kinds[key.rsplit("_config", 1)[0]]
+        assert nbytes > 0
+        assert bench.committed_traffic(key, src_hash) == nbytes
+        assert bench.committed_traffic(key, "0" * 16) is None           # another source: no record
+        assert len(bench.kernel_source_hash(kind)) == 16
+
+
+def test_kernel_source_hash_ignores_comments(tmp_path, monkeypatch):
+    # the hash strips comments and blank lines: a comment edit keeps a traffic record valid,
+    # a code edit does not
+    csrc = tmp_path / "long_context_decode_swa_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in ("rope.cu", "common.cuh"):
+        (csrc / name).write_text(open(os.path.join(ROOT, "long_context_decode_swa_b200", "csrc", name)).read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash("rope")
+    (csrc / "rope.cu").write_text((csrc / "rope.cu").read_text() + "\n// a note\n\n/* another */\n")
+    assert bench.kernel_source_hash("rope") == h0
+    (csrc / "rope.cu").write_text((csrc / "rope.cu").read_text() + "\nstatic int extra_symbol;\n")
+    assert bench.kernel_source_hash("rope") != h0
