@@ -87,7 +87,6 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 2^x on the MUFU unit (the hardware's approximate base-2 exponential, flush-to-zero).
 // max of three (one instruction on sm_100)
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -95,6 +94,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
+// 2^x on the MUFU unit (the hardware's approximate base-2 exponential, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
